@@ -1,0 +1,447 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each pin is written so that a plausible slip anywhere in the oracle (a swapped
+nibble order, a dropped -8 offset, a wrong sign, a transposed operand, an
+off-by-one in the rolling window, a wrong GQA mapping) fails at least one of
+them; ``test_planted_mistakes_are_caught`` plants such slips into copies of the
+oracle's functions and checks that the pins notice.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import ref
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------- fixtures
+def load_handbuilt():
+    cases, cur = [], None
+    with open(os.path.join(GOLDEN, "q4_handbuilt_blocks.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, _, rest = line.partition(" ")
+            if key == "case":
+                cur = {"name": rest}
+                cases.append(cur)
+            elif key == "d":
+                cur["d"] = int(rest, 16)
+            elif key == "qs":
+                cur["qs"] = np.array([int(b, 16) for b in rest.split()], np.uint8)
+            elif key == "w":
+                cur["w"] = np.array([float.fromhex(v) if v.lstrip("-").startswith("0x") else float(v)
+                                     for v in rest.split()])
+    return cases
+
+
+HANDBUILT = load_handbuilt()
+
+
+def same_bits_or_nan(a, b):
+    """Equal as IEEE values including the sign of zero; NaN matches NaN."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    both_nan = np.isnan(a) & np.isnan(b)
+    eq = (a == b) & (np.signbit(a) == np.signbit(b))
+    return bool(np.all(both_nan | eq))
+
+
+# ------------------------------------------------------------ pin functions
+def pin_handbuilt(decode):
+    """decode(qs[1,1,16], d[1,1]) -> 32 weights; must equal the hand-worked values."""
+    for c in HANDBUILT:
+        w = decode(c["qs"].reshape(1, 1, 16), np.array([[c["d"]]], np.uint16)).reshape(-1)
+        assert same_bits_or_nan(w, c["w"]), c["name"]
+
+
+def pin_single_block_dot(matvec):
+    """K = 32: y = d * sum_j (q_j - 8) x_j, worked by hand for the ramp block."""
+    qs = np.array([0xF0, 0xE1, 0xD2, 0xC3, 0xB4, 0xA5, 0x96, 0x87,
+                   0x78, 0x69, 0x5A, 0x4B, 0x3C, 0x2D, 0x1E, 0x0F], np.uint8).reshape(1, 1, 16)
+    d = np.array([[0x4000]], np.uint16)                  # d = 2
+    x = np.zeros((1, 32), np.float32)
+    x[0, 0] = 1.0                                        # w_0 = -8*2 = -16
+    x[0, 15] = 0.5                                       # w_15 = 7*2 = 14 -> 7
+    x[0, 16] = -1.0                                      # w_16 = 7*2 = 14 -> -14
+    x[0, 31] = 0.25                                      # w_31 = -8*2 = -16 -> -4
+    y = np.asarray(matvec(qs, d, x)).reshape(-1)
+    assert y[0] == -16.0 + 7.0 - 14.0 - 4.0
+
+
+def pin_one_hot_columns(matvec, qs, d):
+    """One-hot x picks column j of the exactly dequantised W."""
+    n, nb, _ = qs.shape
+    k = nb * 32
+    W = np.stack([HAND_ROW(qs[r], d[r]) for r in range(n)])
+    for j in (0, 5, 15, 16, 31, 32, k - 1):
+        x = np.zeros((1, k), np.float32)
+        x[0, j] = 1.0
+        y = np.asarray(matvec(qs, d, x)).reshape(-1)
+        assert np.array_equal(y, W[:, j]), j
+
+
+def HAND_ROW(qs_row, d_row):
+    """Straight-line decode of one row, scalar Python, for the one-hot pin."""
+    out = []
+    for b in range(qs_row.shape[0]):
+        scale = float(np.array([d_row[b]], np.uint16).view(np.float16)[0])
+        for j in range(32):
+            byte = int(qs_row[b][j % 16])
+            q = (byte & 15) if j < 16 else (byte >> 4)
+            out.append((q - 8) * scale)
+    return np.array(out)
+
+
+def pin_integer_matrix(matvec):
+    """With d = 1 every weight is the integer q - 8, and with integer x the fp64
+    product is exact: compare with numpy's int64 matmul."""
+    rng = np.random.default_rng(7)
+    n, k = 19, 96
+    qs = rng.integers(0, 256, (n, k // 32, 16), dtype=np.uint8)
+    d = np.full((n, k // 32), 0x3C00, np.uint16)
+    x = rng.integers(-50, 51, (3, k)).astype(np.float32)
+    codes = np.concatenate([qs & 15, qs >> 4], axis=-1).astype(np.int64).reshape(n, k) - 8
+    want = x.astype(np.int64) @ codes.T
+    got = np.asarray(matvec(qs, d, x))
+    assert np.array_equal(got, want.astype(np.float64))
+
+
+def pin_attention_list_model(attn, configs):
+    """Brute force: simulate the rolling window as a plain list of the last W
+    (k, v) pairs in arrival order, attend in pure Python, compare."""
+    for (n_q, n_kv, hd, W) in configs:
+        rng = np.random.default_rng([n_q, n_kv, hd, W])
+        group = n_q // n_kv
+        k_cache = np.zeros((n_kv, W, hd), np.uint16)
+        v_cache = np.zeros((n_kv, W, hd), np.uint16)
+        history = []                                      # list of (k, v) fp32 [n_kv, hd]
+        for P in range(3 * W + 1):
+            k_new = rng.standard_normal((n_kv, hd)).astype(np.float32)
+            v_new = rng.standard_normal((n_kv, hd)).astype(np.float32)
+            ref.c_kv_append(k_cache, v_cache, k_new, v_new, P)
+            history.append((ref.bf16_to_f64(ref.f32_to_bf16(k_new)), ref.bf16_to_f64(ref.f32_to_bf16(v_new))))
+            window = history[-W:]
+            q = rng.standard_normal((n_q, hd)).astype(np.float32)
+            got = attn(q, k_cache, v_cache, P)
+            for h in range(n_q):
+                kvh = h // group
+                s = [sum(float(q[h, c]) * kv[0][kvh, c] for c in range(hd)) / math.sqrt(hd) for kv in window]
+                m = max(s)
+                e = [math.exp(v - m) for v in s]
+                tot = sum(e)
+                want = [sum(e[j] * window[j][1][kvh, c] for j in range(len(window))) / tot for c in range(hd)]
+                np.testing.assert_allclose(got[h], want, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------- tests
+def test_half_decode_all_patterns(oracle_c):
+    """The C oracle's hand-written fp16 decode equals numpy's cast on all 65536 patterns."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    want = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle_c.vr_half_to_double(int(b)) for b in bits])
+    assert same_bits_or_nan(got, want)
+
+
+def test_bf16_rounding_matches_torch(oracle_c):
+    """Both oracle bf16 roundings equal torch's CPU cast (RNE) away from NaN."""
+    import torch
+
+    rng = np.random.default_rng(1)
+    f = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-39).astype(np.float32),     # subnormals
+        np.array([0.0, -0.0, np.inf, -np.inf, 3.4028235e38, -3.4028235e38, 1.0 + 2**-8,
+                  1.0 + 3 * 2**-8], np.float32),
+        # exact ties at every exponent: a kept part plus 0x8000 in the dropped bits
+        (rng.integers(0, 0x7F7F, 2000, dtype=np.uint32) << 16 | 0x8000).astype(np.uint32).view(np.float32),
+    ])
+    want = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got_np = ref.f32_to_bf16(f)
+    got_c = np.array([oracle_c.vr_f32_to_bf16(float(v)) for v in f], np.uint16)
+    assert np.array_equal(got_np, want)
+    assert np.array_equal(got_c, want)
+    assert oracle_c.vr_f32_to_bf16(float("nan")) == 0x7FC0
+    assert ref.f32_to_bf16(np.array([np.nan], np.float32))[0] == 0x7FC0
+
+
+def test_handbuilt_blocks_c_and_numpy():
+    pin_handbuilt(lambda qs, d: ref.c_dequant_f32(qs, d))
+    pin_handbuilt(lambda qs, d: ref.dequant_f32(qs, d))
+
+
+def test_bf16_dequant_ties():
+    rows = []
+    with open(os.path.join(GOLDEN, "bf16_ties.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                a, b = line.split()
+                rows.append((int(a, 16), int(b, 16)))
+    qs = np.full((len(rows), 1, 16), 0x99, np.uint8)       # every code 9 -> q - 8 = 1
+    d = np.array([[a] for a, _ in rows], np.uint16)
+    want = np.array([b for _, b in rows], np.uint16)
+    assert np.all(ref.c_dequant_bf16(qs, d) == want[:, None])
+    assert np.all(ref.dequant_bf16(qs, d) == want[:, None])
+
+
+def test_dequant_fp32_is_exact():
+    """(q-8)*d is exactly representable in fp32 for every fp16 d: the fp32
+    output widened back to float64 equals the float64 product."""
+    rng = np.random.default_rng(3)
+    qs = rng.integers(0, 256, (64, 8, 16), dtype=np.uint8)
+    d = rng.integers(0, 0x7C00, (64, 8), dtype=np.uint16)   # all finite non-negative fp16
+    d[::2] |= 0x8000
+    exact = ref.q4_weights(qs, d)
+    assert np.array_equal(ref.c_dequant_f32(qs, d).astype(np.float64), exact)
+
+
+def test_matvec_single_block_by_hand():
+    pin_single_block_dot(ref.c_matvec)
+    pin_single_block_dot(ref.matvec)
+    pin_single_block_dot(ref.c_matvec_blocksum)
+
+
+def test_matvec_one_hot_columns():
+    rng = np.random.default_rng(11)
+    qs = rng.integers(0, 256, (9, 3, 16), dtype=np.uint8)
+    d = (np.abs(rng.standard_normal((9, 3))) * 0.5).astype(np.float16).view(np.uint16)
+    pin_one_hot_columns(ref.c_matvec, qs, d)
+    pin_one_hot_columns(ref.matvec, qs, d)
+
+
+def test_matvec_zero_codes():
+    qs = np.full((5, 4, 16), 0x88, np.uint8)
+    d = np.full((5, 4), 0x3C00, np.uint16)
+    x = np.ones((2, 128), np.float32)
+    assert np.all(ref.c_matvec(qs, d, x) == 0.0)
+
+
+def test_matvec_integer_exact():
+    pin_integer_matrix(ref.c_matvec)
+    pin_integer_matrix(ref.matvec)
+    pin_integer_matrix(ref.c_matvec_blocksum)
+
+
+def test_matvec_routes_agree():
+    """Dense route (dequantise then fp64 matmul) == block-sum identity == numpy twin."""
+    import synth
+
+    qs, d = synth.q4_blocks(300, 3072, 0, 12345)
+    x = synth.activations(3, 3072, 0, 54321)
+    y_dense = ref.c_matvec(qs, d, x)
+    y_block = ref.c_matvec_blocksum(qs, d, x)
+    y_np = ref.matvec(qs, d, x)
+    scale = np.abs(y_dense).max()
+    assert np.max(np.abs(y_dense - y_block)) <= 1e-12 * scale
+    assert np.max(np.abs(y_dense - y_np)) <= 1e-12 * scale
+    # row sampling of the C oracle returns the same rows
+    y_rows = ref.c_matvec(qs, d, x, row0=17, nrows=40)
+    assert np.array_equal(y_rows, y_dense[:, 17:57])
+
+
+def test_rolling_slots_bruteforce():
+    """slot = pos mod W: after appending 0..P the slots hold exactly the last
+    min(P+1, W) positions, each once (list model)."""
+    for W in (1, 2, 3, 5, 8192):
+        slots = {}
+        last = []
+        top = 3 * W + 5 if W < 100 else 2 * W + 300
+        for P in range(top + 1):
+            s = int(ref.c_lib().vr_kv_slot(P, W))
+            assert s == ref.kv_slot(P, W)
+            slots[s] = P
+            last.append(P)
+            last = last[-W:]
+            assert sorted(slots.values()) == last
+            assert len(slots) == ref.valid_slots(P, W)
+            assert set(slots.keys()) == set(range(ref.valid_slots(P, W)))
+
+
+def test_kv_append_c_equals_numpy():
+    rng = np.random.default_rng(5)
+    kc1 = np.zeros((3, 7, 16), np.uint16); vc1 = kc1.copy()
+    kc2 = kc1.copy(); vc2 = kc1.copy()
+    for P in range(20):
+        k = rng.standard_normal((3, 16)).astype(np.float32)
+        v = rng.standard_normal((3, 16)).astype(np.float32)
+        ref.c_kv_append(kc1, vc1, k, v, P)
+        ref.kv_append(kc2, vc2, k, v, P)
+    assert np.array_equal(kc1, kc2) and np.array_equal(vc1, vc2)
+
+
+TINY_ATTN = [(1, 1, 1, 1), (2, 1, 4, 3), (4, 2, 8, 5), (2, 2, 4, 1), (4, 1, 8, 3)]
+
+
+def test_attention_bruteforce_c():
+    pin_attention_list_model(lambda q, kc, vc, P: ref.c_gqa_attn(q, kc, vc, P), TINY_ATTN)
+
+
+def test_attention_bruteforce_numpy():
+    pin_attention_list_model(lambda q, kc, vc, P: ref.gqa_attn(q, kc, vc, P), TINY_ATTN)
+
+
+def test_attention_invariants():
+    import synth
+
+    n_q, n_kv, hd, W = 8, 2, 16, 37
+    kc = synth.bf16_normal((n_kv, W, hd), 0, 1)
+    vc = synth.bf16_normal((n_kv, W, hd), 0, 2)
+    q = synth.activations(n_q, hd, 0, 3)
+    V = ref.bf16_to_f64(vc)
+    # one valid key -> o = v exactly
+    o = ref.c_gqa_attn(q, kc, vc, 0)
+    for h in range(n_q):
+        assert np.array_equal(o[h], V[h // 4, 0])
+    # q = 0 -> mean of the valid V rows
+    P = 20
+    o = ref.c_gqa_attn(np.zeros_like(q), kc, vc, P)
+    for h in range(n_q):
+        np.testing.assert_allclose(o[h], V[h // 4, :P + 1].mean(axis=0), rtol=1e-12, atol=1e-13)
+    # wrapped: permuting the slots leaves o unchanged (ring == compaction)
+    P = 3 * W + 4
+    perm = np.random.default_rng(0).permutation(W)
+    o1 = ref.c_gqa_attn(q, kc, vc, P)
+    o2 = ref.c_gqa_attn(q, np.ascontiguousarray(kc[:, perm]), np.ascontiguousarray(vc[:, perm]), P)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
+    # group size 1 is plain multi-head attention: head h reads kv head h
+    o_mha = ref.c_gqa_attn(q[:2], kc, vc, P)
+    for h in range(2):
+        o_single = ref.c_gqa_attn(q[h:h + 1], np.ascontiguousarray(kc[h:h + 1]), np.ascontiguousarray(vc[h:h + 1]), P)
+        np.testing.assert_allclose(o_mha[h], o_single[0], rtol=1e-12, atol=1e-13)
+    # split-KV combine with any split count equals the unsplit result
+    for ns in (1, 2, 3, 7, W):
+        np.testing.assert_allclose(ref.combine_partials(ref.split_partials(q, kc, vc, P, ns)), o1,
+                                   rtol=1e-12, atol=1e-13)
+    # C and numpy twins agree
+    np.testing.assert_allclose(ref.gqa_attn(q, kc, vc, P), o1, rtol=1e-12, atol=1e-13)
+
+
+def test_rmsnorm_silu_gelu_closed_forms():
+    eps = ref.RMS_EPS
+    for c in (0.1, 1.0, -3.0, 250.0):
+        r = ref.rmsnorm(np.full(3072, c))
+        np.testing.assert_allclose(r, np.sign(c) / np.sqrt(1 + eps / c ** 2), rtol=1e-14)
+    assert ref.silu(0.0) == 0.0
+    np.testing.assert_allclose(ref.silu(np.array([30.0, -30.0, 1.0])),
+                               [30.0 - 30.0 * math.exp(-30.0) / (1 + math.exp(-30.0)),
+                                -30.0 * math.exp(-30.0) / (1 + math.exp(-30.0)), 1 / (1 + math.exp(-1))],
+                               rtol=1e-14)
+    assert ref.gelu(0.0) == 0.0
+    xs = np.array([-6.0, -1.0, -0.3, 0.5, 2.0, 9.0])
+    want = [0.5 * v * (1 + math.erf(v / math.sqrt(2))) for v in xs]
+    np.testing.assert_allclose(ref.gelu(xs), want, rtol=1e-14)
+    assert abs(ref.gelu(40.0) - 40.0) < 1e-12
+
+
+def test_window_attention_bruteforce():
+    """Encoder sliding window: query i (position q0+i) sees j with p-W < j <= p."""
+    rng = np.random.default_rng(9)
+    nh, hd, W, nhist, nq = 2, 3, 4, 5, 3
+    Q = rng.standard_normal((nq, nh * hd))
+    K = rng.standard_normal((nhist + nq, nh * hd))
+    V = rng.standard_normal((nhist + nq, nh * hd))
+    got = ref.window_attn(Q, K, V, nhist, W, nh, hd)
+    for i in range(nq):
+        p = nhist + i
+        vis = [j for j in range(nhist + nq) if p - W < j <= p]
+        assert len(vis) == W
+        for h in range(nh):
+            sl = slice(h * hd, (h + 1) * hd)
+            s = [float(Q[i, sl] @ K[j, sl]) / math.sqrt(hd) for j in vis]
+            e = [math.exp(v - max(s)) for v in s]
+            want = sum(e[t] * V[vis[t], sl] for t in range(W)) / sum(e)
+            np.testing.assert_allclose(got[i, sl], want, rtol=1e-12)
+
+
+def test_downsample_order():
+    X = np.arange(8 * 3).reshape(8, 3)
+    Y = ref.downsample_rows(X, 4)
+    assert Y.shape == (2, 12)
+    assert list(Y[1]) == list(range(12, 24))
+
+
+def test_argmax_lowest_index():
+    assert ref.argmax_lowest([1.0, 3.0, 3.0, 2.0]) == 1
+    assert ref.argmax_lowest([-1.0, -1.0]) == 0
+
+
+def test_shape_readings_match_page_footprints():
+    """Parameter-count cross-check of the shape readings against the pages'
+    footprints (tests/golden/footprint.txt): untied embedding + LM head and an
+    ungated encoder FFN fit; the alternatives fit worse."""
+    fp = {}
+    with open(os.path.join(GOLDEN, "footprint.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                key, val, unit, tol = line.split()[:4]
+                fp[key] = (float(val), unit, float(tol))
+    dec_layer = 4096 * 3072 + 2 * 1024 * 3072 + 3072 * 4096 + 3 * 9216 * 3072
+    assert dec_layer == 116_391_936
+    enc_layer = 3 * 1280 * 1280 + 1280 * 1280 + 2 * 5120 * 1280
+    vocab = int(fp["vocab"][0])
+    embed = vocab * 3072
+    adapter = 5120 * 3072 + 3072 * 3072
+    total = 26 * dec_layer + 2 * embed + 32 * enc_layer + adapter
+    assert total == 4_485_808_128
+
+    def within(key, value):
+        want, _, tol = fp[key]
+        return abs(value - want) <= tol * want
+
+    assert within("bf16_weights", total * 2 / 1e9)
+    assert within("f16_gpu_cache", total * 2 / 2 ** 30)
+    assert within("q4_gguf", total * 18 / 32 / 1e9)
+    assert within("kv_cache_max", 26 * 8192 * 1024 * 2 * 4 / 1e9)
+    assert within("embedding_f32", embed * 4 / 2 ** 30)
+    gated = total + 32 * 5120 * 1280
+    tied = total - embed
+    assert abs(gated * 2 / 1e9 - 8.9) > abs(total * 2 / 1e9 - 8.9)
+    assert abs(tied * 2 / 1e9 - 8.9) > abs(total * 2 / 1e9 - 8.9)
+
+
+# ------------------------------------------------------- planted mistakes
+def test_planted_mistakes_are_caught():
+    """Copies of the oracle's functions with one plausible slip each must fail a pin."""
+    def swapped_nibbles(qs, d):
+        codes = np.concatenate([qs >> 4, qs & 0x0F], axis=-1).astype(np.int64)
+        return ((codes - 8) * ref.half_to_f64(d)[:, :, None]).reshape(qs.shape[0], -1)
+
+    def no_offset(qs, d):
+        codes = np.concatenate([qs & 0x0F, qs >> 4], axis=-1).astype(np.int64)
+        return (codes * ref.half_to_f64(d)[:, :, None]).reshape(qs.shape[0], -1)
+
+    def interleaved_nibbles(qs, d):
+        codes = np.stack([qs & 0x0F, qs >> 4], axis=-1).reshape(qs.shape[0], qs.shape[1], 32).astype(np.int64)
+        return ((codes - 8) * ref.half_to_f64(d)[:, :, None]).reshape(qs.shape[0], -1)
+
+    for bad in (swapped_nibbles, no_offset, interleaved_nibbles):
+        with pytest.raises(AssertionError):
+            pin_handbuilt(bad)
+
+    def transposed_matvec(qs, d, x):
+        W = ref.q4_weights(qs, d)
+        x = np.atleast_2d(x).astype(np.float64)
+        return (W[:, :x.shape[1]] @ x[:, :W.shape[0]].T).T if W.shape[0] == W.shape[1] else x @ W[:, ::-1].T
+
+    with pytest.raises(AssertionError):
+        pin_integer_matrix(transposed_matvec)
+
+    def attn_off_by_one(q, kc, vc, P):           # drops the newest position
+        return ref.gqa_attn(q, kc, vc, max(P - 1, 0))
+
+    with pytest.raises(AssertionError):
+        pin_attention_list_model(attn_off_by_one, [(2, 1, 4, 3)])
+
+    def attn_wrong_group(q, kc, vc, P):          # interleaved head -> kv mapping
+        n_kv = kc.shape[0]
+        out = np.empty((q.shape[0], kc.shape[2]))
+        for h in range(q.shape[0]):
+            out[h] = ref.gqa_attn(q[h:h + 1], kc[h % n_kv:h % n_kv + 1], vc[h % n_kv:h % n_kv + 1], P)[0]
+        return out
+
+    with pytest.raises(AssertionError):
+        pin_attention_list_model(attn_wrong_group, [(4, 2, 8, 5)])
