@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of the Q4_0 decode hot path on B200: prints ONE JSON line.
+
+Workload (default, N=1): the full synthetic 26-layer decoder token step of
+Voxtral Mini 4B Realtime (dim 3072, GQA 32/8, FFN 9216, Q4_0 weights, 131072 x
+3072 LM head and embedding), rolling KV cache of 8192 positions filled to
+8192 + 300 (wrapped), M = 1.  One step = one replay of the captured
+vox_decoder_step graph: embedding row, 26 x (RMSNorm+QKV GEMV+rolling append,
+split-KV GQA attention, Wo GEMV+residual, RMSNorm+W1||W3 GEMV+SiLU*mul, W2
+GEMV+residual), RMSNorm+LM-head GEMV+argmax, position advance.  Every step
+streams 2.8 GB (> 126 MB L2), so no flush is needed between steps.
+
+value      = algorithmic bytes of all steps of all ranks / max-over-ranks time (GB/s)
+ms_per_step= the decoder ms/step
+roofline   = the dominant kernel (the Q4_0 GEMV, ~69% of the step's bytes),
+             timed inside this run over the step's own 105 GEMV launches
+e2e        = the same metric through the Python API with the token copied
+             host->device before and device->host after every step
+cpu_baseline / --impl reference = the CPU oracle (oracle/) on the host cores
+
+Multi-GPU: one process per GPU (torchrun), independent replicas (the path
+does not shard), barrier + max-over-ranks device time; "scaling": "weak".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Q4_0 GEMV weight GB/s (% of HBM peak); 26-layer decoder ms/step on 1 B200"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+FILLED = 8192 + 300
+# dram bytes per launch of the dominant kernel from the committed ncu capture
+# (profiles/q4_gemv_decoder_step.md); None until a capture of the current kernel exists
+GEMV_TRAFFIC_BYTES_PER_LAUNCH = None
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
+    return p.parse_args(argv)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
+
+
+# ------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu)],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ------------------------------------------------------- distributed
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def dist_init(world, backend):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+
+
+def aggregate(local_ms: float, steps: int, bytes_per_step: int, world: int):
+    """Max-over-ranks time and the whole-job throughput (GB/s) of `world`
+    independent replicas that each ran `steps` steps."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([local_ms], dtype=torch.float64)
+    if world > 1 and dist.is_initialized():
+        if dist.get_backend() == "nccl":
+            t = t.cuda()
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    value = world * steps * bytes_per_step / (max_ms / 1e3) / 1e9
+    return max_ms, value
+
+
+def barrier(world):
+    import torch.distributed as dist
+
+    if world > 1 and dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------ timing
+def time_replays(g, n, world):
+    import torch
+
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(n):
+        g.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    return e0.elapsed_time(e1)
+
+
+# ------------------------------------------------------- CPU oracle
+def oracle_decoder_sample(budget_s: float, layers=None):
+    """The oracle's decoder layer (C oracle matvec + attention, numpy norms) on
+    consecutive layers of the same workload until `budget_s` of CPU time is
+    spent.  Returns (bytes processed, seconds, layers done, threads)."""
+    import numpy as np
+
+    import synth
+    from oracle import ref
+
+    shape = synth.DecoderShape()
+    D, QD, KVD = shape.dim, shape.q_dim, shape.kv_dim
+    done, t_tot, bytes_tot = 0, 0.0, 0
+    x = synth.activations(1, D, 0, synth.X_ID)[0]
+    for l in range(shape.n_layers if layers is None else layers):
+        w = synth.decoder_layer_weights(shape, l, 0)
+        kc, vc = synth.decoder_layer_cache(shape, l, 0)
+        t0 = time.perf_counter()
+        n = ref.rmsnorm(x).astype(np.float32)
+        qkv = np.concatenate([ref.c_matvec(*w[k], n)[0] for k in ("wq", "wk", "wv")])
+        ref.c_kv_append(kc, vc, qkv[QD:QD + KVD].reshape(shape.n_kv_heads, -1),
+                        qkv[QD + KVD:].reshape(shape.n_kv_heads, -1), FILLED)
+        o = ref.c_gqa_attn(qkv[:QD].reshape(shape.n_q_heads, -1).astype(np.float32), kc, vc, FILLED).reshape(-1)
+        h = x + ref.c_matvec(*w["wo"], o.astype(np.float32))[0]
+        n2 = ref.rmsnorm(h).astype(np.float32)
+        a = ref.silu(ref.c_matvec(*w["w1"], n2)[0]) * ref.c_matvec(*w["w3"], n2)[0]
+        x = (h + ref.c_matvec(*w["w2"], a.astype(np.float32))[0]).astype(np.float32)
+        t_tot += time.perf_counter() - t0
+        done += 1
+        nw = sum(v[0].shape[0] * v[0].shape[1] * 32 for v in w.values())
+        bytes_tot += nw * 18 // 32 + 2 * shape.n_kv_heads * min(FILLED + 1, shape.window) * shape.head_dim * 2
+        if t_tot >= budget_s:
+            break
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return bytes_tot, t_tot, done, threads
+
+
+def cpu_baseline(budget_s):
+    b, t, n, threads = oracle_decoder_sample(budget_s)
+    return {"value": b / t / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} of 26 decoder layers of the same step (fp64 C oracle, OpenMP over rows), "
+                      f"{b / 1e6:.1f} MB in {t:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle on the host cores, timed as the reference arm."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    budget = max(0.05, 90.0 / max(1, args.steps + args.warmup))
+    import numpy as np
+
+    import synth
+    from oracle import ref
+
+    shape = synth.DecoderShape()
+    w = synth.decoder_layer_weights(shape, 0, 0)
+    kc, vc = synth.decoder_layer_cache(shape, 0, 0)
+    x = synth.activations(1, shape.dim, 0, synth.X_ID)[0]
+    mats = [w[k] for k in ("wq", "wk", "wv", "wo", "w1", "w3", "w2")]
+    # calibrate rows per step so one step takes about `budget` seconds
+    t0 = time.perf_counter()
+    ref.c_matvec(*w["w1"], ref.rmsnorm(x).astype(np.float32), row0=0, nrows=512)
+    per_row = (time.perf_counter() - t0) / 512
+    rows = int(max(16, min(9216, budget / max(per_row, 1e-9))))
+    tot_bytes, tot_t = 0, 0.0
+    xin = {3072: ref.rmsnorm(x).astype(np.float32), 4096: synth.activations(1, 4096, 0, 1)[0],
+           9216: synth.activations(1, 9216, 0, 2)[0]}
+    for it in range(args.warmup + args.steps):
+        qs, d = mats[it % len(mats)]
+        r0 = (it * rows) % max(1, qs.shape[0] - rows + 1)
+        nr = min(rows, qs.shape[0])
+        t0 = time.perf_counter()
+        ref.c_matvec(qs, d, xin[qs.shape[1] * 32], row0=r0, nrows=nr)
+        dt = time.perf_counter() - t0
+        if it >= args.warmup:
+            tot_t += dt
+            tot_bytes += nr * qs.shape[1] * 18
+    value = tot_bytes / tot_t / 1e9
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = f"per step {rows} rows of one decoder projection ({rows * 3072 * 18 // 32 / 1e6:.2f} MB Q4_0), fp64 C oracle"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "decoder_step_q4_26L_kv8192wrapped_M1 (oracle row sample)", "l2": "n/a (host)"},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------- ours
+def run_ours(args):
+    import torch
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist_init(world, "nccl")
+    from bit_quantized_transformer_b200 import build
+
+    if rank == 0 or not os.path.exists(build.LIB):
+        build.build()
+    barrier(world)
+    import synth
+    from bit_quantized_transformer_b200 import workloads as WL
+
+    shape = synth.DecoderShape()
+    dm = WL.DecoderModel(shape, seed=0, filled=FILLED, token=17)
+    g = dm.capture()
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    step_bytes = dm.weight_bytes() + dm.kv_bytes(FILLED)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    local_ms = time_replays(g, args.steps, world)
+    clk = clocks.stop()
+    max_ms, value = aggregate(local_ms, args.steps, step_bytes, world)
+    ms_step = max_ms / args.steps
+
+    # dominant kernel: the step's 105 GEMV launches captured alone, same chaining
+    gg = dm.capture(dm.gemv_chain)
+    for _ in range(3):
+        gg.replay()
+    reps = max(20, min(400, args.steps // 4))
+    ms_g = time_replays(gg, reps, world)
+    launches = dm.gemv_chain_launches()
+    per_launch_bytes = dm.gemv_chain_bytes() / launches
+    per_launch_ms = ms_g / (reps * launches)
+    achieved = per_launch_bytes / (per_launch_ms / 1e3) / 1e9
+    peak, peak_src = measured_peaks()
+
+    # attention alone (reported beside the roofline)
+    pos_now = int(dm.pos.item())
+    ga = dm.capture(lambda: dm.attn_chain(pos_now))
+    for _ in range(3):
+        ga.replay()
+    ms_a = time_replays(ga, reps, world)
+    attn_bytes = dm.kv_bytes(pos_now)
+    attn_gbs = attn_bytes * reps / (ms_a / 1e3) / 1e9
+
+    # end to end through the Python API: token H2D, graph replay, token D2H
+    e2e_steps = max(10, min(args.steps, 500))
+    tok_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
+    out_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
+    tok_h[0] = 17
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(e2e_steps):
+        dm.token.copy_(tok_h, non_blocking=True)
+        g.replay()
+        out_h.copy_(dm.token, non_blocking=True)
+        s.synchronize()
+        tok_h[0] = out_h[0]                                   # the host feeds the next token back
+    e1.record(s)
+    torch.cuda.synchronize()
+    e2e_local = e0.elapsed_time(e1)
+    _, e2e_value = aggregate(e2e_local, e2e_steps, step_bytes, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "q4_0 weights, fp16/bf16 tensor-core inputs, f32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": "decoder_step_q4_26L_kv8192wrapped_M1", "layers": shape.n_layers,
+                       "dim": shape.dim, "heads": "32q/8kv x 128", "ffn": shape.ffn, "vocab": shape.vocab,
+                       "kv_window": shape.window, "kv_filled": FILLED, "bytes_per_step": step_bytes,
+                       "weight_bytes_per_step": dm.weight_bytes(), "kv_bytes_per_step": dm.kv_bytes(FILLED),
+                       "l2": "inputs larger than L2 (2.8 GB per step, no flush)",
+                       "replicas": world, "graph": "one CUDA graph per step, PDL between kernels"},
+            "roofline": {"bound": "hbm", "kernel": "q4_gemv_kernel", "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": GEMV_TRAFFIC_BYTES_PER_LAUNCH,
+                         "peak_source": peak_src, "launches_timed": reps * launches,
+                         "algorithmic_bytes_per_launch": per_launch_bytes,
+                         "avg_launch_us": per_launch_ms * 1e3},
+            "attention": {"kernel": "gqa_decode_attn_kernel+attn_combine_kernel", "gbs": attn_gbs,
+                          "frac": attn_gbs / peak, "bytes_per_step": attn_bytes,
+                          "us_per_layer": ms_a / reps / dm.L * 1e3},
+            "decoder_ms_per_step": ms_step,
+            "hbm_frac_step": value / world / peak,
+            "gpu_launches": dm.step_launches() * args.steps,
+            "clocks": clk,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4,
+                    "ms_per_step": e2e_local / e2e_steps, "api": "DecoderModel graph replay via vox_decoder_step"},
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    del g, gg, ga
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,148 @@
+// Host plumbing (error state, device queries, tensor-map encoding) and the
+// small glue kernels: RMSNorm with fp32/bf16 output and the end-of-step
+// position advance.
+#include <mutex>
+#include <stdio.h>
+#include <string.h>
+
+#include "tma.cuh"
+
+namespace vox {
+
+__device__ int32_t g_vox_device_status = 0;
+
+static thread_local char t_last_error[256] = "";
+
+void set_cuda_error(cudaError_t e)
+{
+    snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+const char* last_error_text() { return t_last_error; }
+
+vox_status check_launch()
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        set_cuda_error(e);
+        return VOX_ERR_CUDA;
+    }
+    return VOX_OK;
+}
+
+int device_sm_count()
+{
+    static int cached[64];
+    static bool init[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!init[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+        init[dev] = true;
+    }
+    return cached[dev];
+}
+
+// ------------------------------------------------------------ tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+vox_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+                        uint64_t cols, uint64_t rows, uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows,
+                        CUtensorMapSwizzle swizzle)
+{
+    (void)elem_bytes;
+    auto fn = get_encode_fn();
+    if (!fn) {
+        snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled unavailable");
+        return VOX_ERR_CUDA;
+    }
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {pitch_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return VOX_ERR_CUDA;
+    }
+    return VOX_OK;
+}
+
+// ------------------------------------------------------------------ RMSNorm
+// One CTA per row: y = x / sqrt(mean(x^2) + eps) * g (g = 1 when NULL);
+// with normalize == 0 the row is only converted (y = x * g).
+__global__ void rmsnorm_kernel(const float* __restrict__ x, int64_t n, int64_t ldx, float eps,
+                               const float* __restrict__ g, void* __restrict__ out, int out_bf16, int64_t ldo,
+                               int normalize)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    __shared__ float red[32];
+    const int64_t row = blockIdx.x;
+    const float* xr = x + row * ldx;
+    float ssq = 0.f;
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) ssq = fmaf(xr[i], xr[i], ssq);
+    for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ssq;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float s = 0.f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += red[w];
+        red[0] = normalize ? 1.0f / sqrtf(s / (float)n + eps) : 1.0f;
+    }
+    __syncthreads();
+    const float r = red[0];
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+        float v = xr[i] * r;
+        if (g) v *= g[i];
+        if (out_bf16)
+            static_cast<uint16_t*>(out)[row * ldo + i] = f32_to_bf16_bits(v);
+        else
+            static_cast<float*>(out)[row * ldo + i] = v;
+    }
+}
+
+vox_status launch_rmsnorm(const float* x, int64_t m, int64_t n, int64_t ldx, float eps, const float* g, void* out,
+                          int out_dtype, int64_t ldo, cudaStream_t s)
+{
+    return launch_pdl(rmsnorm_kernel, dim3((unsigned)m), dim3(256), 0, s, x, n, ldx, eps, g, out,
+                      (int)(out_dtype == VOX_BF16), ldo, 1);
+}
+
+vox_status launch_cast_rows(const float* x, int64_t m, int64_t n, int64_t ldx, void* out, int out_dtype,
+                            int64_t ldo, cudaStream_t s)
+{
+    return launch_pdl(rmsnorm_kernel, dim3((unsigned)m), dim3(256), 0, s, x, n, ldx, 0.0f,
+                      static_cast<const float*>(nullptr), out, (int)(out_dtype == VOX_BF16), ldo, 0);
+}
+
+// --------------------------------------------------------- position advance
+__global__ void advance_pos_kernel(int64_t* pos)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    if (threadIdx.x == 0) *pos += 1;
+}
+
+vox_status launch_advance_pos(int64_t* pos, cudaStream_t s)
+{
+    return launch_pdl(advance_pos_kernel, dim3(1), dim3(32), 0, s, pos);
+}
+
+}  // namespace vox

@@ -1,0 +1,317 @@
+// K2: fused Q4_0 dequantise + GEMM on the 5th-generation tensor cores
+// (tcgen05), for M >= 16 activation rows: encoder chunks and batched decode.
+//
+// Y[i][j] = sum_c X[i][c] W[j][c], W = (q - 8) * d (GGUF Q4_0, "Voxtral Mini
+// 4B Realtime (Rust)", page 5 "Arquitetura"), with the dequantisation fused
+// into the matmul ("브라우저에서 도는 4B 음성인식: Voxtral Rust+WASM 구현 해부",
+// "F32(9GB) vs Q4 GGUF(2.5GB)").  Encoder shapes: voxtral.c page, "모델
+// 아키텍처" (dim 1280, FFN 5120, adapter 5120 -> 3072).
+//
+// One CTA computes a 128-weight-row x BN-token tile of Y^T in tensor memory:
+//   warp 0      producer: bulk copies of the 8 packed 576-byte records of the
+//               128 rows for one 64-column chunk, and a TMA tile (128-byte
+//               swizzle) of BN activation rows x 64 columns;
+//   warp 1      allocates BN tensor-memory columns and, from one thread,
+//               issues tcgen05.mma kind::f16 (M=128, N=BN, K=16, bf16 in, fp32
+//               accumulate) on shared-memory descriptors, committing each
+//               stage back to the producer;
+//   warps 2-9   dequantise: thread (row, block) turns 32 codes into bf16
+//               (q - 8) * d and writes them in the canonical K-major
+//               128-byte-swizzled layout the MMA reads; after the last chunk
+//               they read the accumulator with tcgen05.ld and run the
+//               epilogue (residual add, GELU, fp32 or bf16 store).
+#include "tma.cuh"
+
+namespace vox {
+
+constexpr int kGemmThreads = 320;
+constexpr int kGemmRows = 128;                      // MMA M (weight rows per CTA)
+constexpr int kGemmRawBytes = 8 * kChunkBytes;      // 4608
+constexpr int kGemmABytes = kGemmRows * 128;        // 16 KB bf16 tile, 64 columns
+
+struct GemmArgs {
+    const uint8_t* w;
+    int64_t n, k;
+    int32_t tiles, kc;
+    int64_t m;
+    void* y;
+    int32_t y_bf16;
+    int64_t ldy;
+    int32_t op;
+    const float* res;
+    int64_t ldr;
+};
+
+template <int BN>
+struct GemmCfg {
+    static constexpr int xbytes = BN * 128;
+    static constexpr int stage = ((xbytes + kGemmABytes + kGemmRawBytes) + 1023) / 1024 * 1024;
+    static constexpr int stages = (200 * 1024 / stage) > 6 ? 6 : (200 * 1024 / stage);
+    static constexpr int bars = stages * stage;
+    static constexpr int smem = bars + (3 * stages + 2) * 8 + 16 + 1024;
+    static constexpr int tmem_cols = BN < 32 ? 32 : BN;
+};
+
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr)
+{
+    // start address >> 4 (bits 0-13), LBO 16 B (unused for swizzled K-major),
+    // SBO 1024 B between 8-row groups, version 1, 128-byte swizzle.
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(dtmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8])
+{
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ float gelu_erf_g(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a)
+{
+    using C = GemmCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::bars);
+    uint64_t* aready = full + C::stages;
+    uint64_t* empty = aready + C::stages;
+    uint64_t* accb = empty + C::stages;
+    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(accb + 2);
+    volatile int32_t* s_fail = reinterpret_cast<volatile int32_t*>(accb + 2) + 1;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t group = blockIdx.x;              // 8 row tiles = 128 weight rows
+    const int64_t m0 = (int64_t)blockIdx.y * BN;
+    const int kc = a.kc;
+
+    if (tid == 0) {
+        for (int s = 0; s < C::stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&aready[s], 8);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&accb[0], 1);
+        s_fail[0] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_addr((const void*)s_tmem)), "r"((uint32_t)C::tmem_cols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *s_tmem;
+    pdl_wait();
+
+    if (warp == 0) {
+        // ------------------------------------------------------- producer
+        if (lane == 0) {
+            pdl_launch_dependents();
+            prefetch_tmap(&xmap);
+            const int ntile = (int)min64(8, a.tiles - group * 8);
+            const uint32_t bytes = (uint32_t)ntile * kChunkBytes + C::xbytes;
+            for (int kb = 0; kb < kc; ++kb) {
+                const int s = kb % C::stages;
+                const uint32_t ph = (uint32_t)((kb / C::stages) & 1);
+                if (!s_fail[0] && !mbar_wait_bounded(&empty[s], ph ^ 1u, 0x301)) s_fail[0] = 1;
+                if (s_fail[0]) break;
+                uint8_t* st = smem + s * C::stage;
+                mbar_arrive_expect_tx(&full[s], bytes);
+                for (int tt = 0; tt < ntile; ++tt)
+                    bulk_g2s(st + C::xbytes + kGemmABytes + tt * kChunkBytes,
+                             a.w + ((group * 8 + tt) * (int64_t)kc + kb) * kChunkBytes, kChunkBytes, &full[s]);
+                tma_load_2d(st, &xmap, kb * 64, (int32_t)m0, &full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------- MMA issue
+        if (lane == 0) {
+            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                   ((uint32_t)(kGemmRows >> 4) << 24);
+            for (int kb = 0; kb < kc; ++kb) {
+                const int s = kb % C::stages;
+                const uint32_t ph = (uint32_t)((kb / C::stages) & 1);
+                if (!s_fail[0] && !mbar_wait_bounded(&aready[s], ph, 0x302)) s_fail[0] = 1;
+                if (s_fail[0]) break;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t xs = smem_addr(smem + s * C::stage);
+                const uint32_t as = xs + C::xbytes;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem, umma_desc_sw128(as + kk * 32), umma_desc_sw128(xs + kk * 32), idesc,
+                              (kb > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&empty[s]);
+            }
+            umma_commit(&accb[0]);
+        }
+    } else {
+        // ------------------------------------------------- dequant + epilogue
+        const int dw = warp - 2;                    // 0..7
+        const int q = warp & 3;                     // tensor-memory lane quarter of this warp
+        const int r = 32 * q + lane;                // weight row within the CTA tile
+        const int bb = dw >> 2;                     // block (0, 1) of the chunk
+        const int tt = r >> 4, i16 = r & 15, g = i16 & 7, rowsel = i16 >> 3;
+        for (int kb = 0; kb < kc; ++kb) {
+            const int s = kb % C::stages;
+            const uint32_t ph = (uint32_t)((kb / C::stages) & 1);
+            if (!s_fail[0] && !mbar_wait_bounded(&full[s], ph, 0x303)) s_fail[0] = 1;
+            uint8_t* st = smem + s * C::stage;
+            const uint8_t* rec = st + C::xbytes + kGemmABytes + tt * kChunkBytes;
+            const float d = __half2float(*reinterpret_cast<const __half*>(rec + kChunkQsBytes + 8 * g + 2 * (bb * 2 + rowsel)));
+            uint2 wv[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) wv[t] = *reinterpret_cast<const uint2*>(rec + 16 * (4 * g + t) + 8 * bb);
+            uint8_t* A = st + C::xbytes;
+#pragma unroll
+            for (int uu = 0; uu < 4; ++uu) {
+                const int half = uu >> 1, w = uu & 1;
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int t = j >> 1, elem = j & 1;
+                    const uint32_t word = w ? wv[t].y : wv[t].x;
+                    const int sh = 4 * (rowsel * 2 + half + 4 * elem);
+                    v[j] = (float)((int)((word >> sh) & 15u) - 8) * d;
+                }
+                const uint4 pk = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                *reinterpret_cast<uint4*>(A + sw128_offset((uint32_t)r, (uint32_t)(bb * 4 + uu))) = pk;
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&aready[s]);
+        }
+        // ---- epilogue
+        if (!s_fail[0] && !mbar_wait_bounded(&accb[0], 0, 0x304)) s_fail[0] = 1;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const int64_t row = group * kGemmRows + r;
+        const int c0 = (dw >> 2) * (BN / 2);
+        for (int cc = 0; cc < BN / 2; cc += 8) {
+            float v[8];
+            tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c0 + cc), v);
+            if (row < a.n) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int64_t mi = m0 + c0 + cc + j;
+                    if (mi >= a.m) break;
+                    float o = v[j];
+                    if (a.op == VOX_EP_RESIDUAL) o += a.res[mi * a.ldr + row];
+                    else if (a.op == VOX_EP_GELU) o = gelu_erf_g(o);
+                    if (a.y_bf16)
+                        static_cast<uint16_t*>(a.y)[mi * a.ldy + row] = f32_to_bf16_bits(o);
+                    else
+                        static_cast<float*>(a.y)[mi * a.ldy + row] = o;
+                }
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 1) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::tmem_cols)
+                     : "memory");
+    }
+}
+
+template <int BN>
+static vox_status launch_gemm_bn(const GemmArgs& a, const void* x, int64_t ldx, cudaStream_t s)
+{
+    using C = GemmCfg<BN>;
+    CUtensorMap xmap;
+    vox_status st = make_tmap_2d(&xmap, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.k, (uint64_t)a.m,
+                                 (uint64_t)ldx * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != VOX_OK) return st;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(q4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem);
+        if (e != cudaSuccess) {
+            set_cuda_error(e);
+            return VOX_ERR_CUDA;
+        }
+        attr = true;
+    }
+    dim3 grid((unsigned)ceil_div(a.tiles, 8), (unsigned)ceil_div(a.m, BN));
+    return launch_pdl(q4_gemm_kernel<BN>, grid, dim3(kGemmThreads), (size_t)C::smem, s, xmap, a);
+}
+
+static int pick_bn(int64_t tiles, int64_t m)
+{
+    const char* e = getenv("VOX_GEMM_BN");
+    if (e) {
+        int v = atoi(e);
+        if (v == 32 || v == 64 || v == 128 || v == 256) return v;
+    }
+    const int64_t groups = ceil_div(tiles, 8);
+    const int64_t sms = device_sm_count();
+    int best = 256;
+    int64_t best_cost = INT64_MAX;
+    for (int bn = 256; bn >= 32; bn >>= 1) {
+        if (bn > 32 && (bn >> 1) >= m) continue;            // a smaller tile already covers every row
+        const int64_t ctas = groups * ceil_div(m, bn);
+        const int64_t waves = ceil_div(ctas, sms);
+        const int64_t cost = waves * (bn > 64 ? bn : 64);    // per-stage time ~ max(MMA, dequant)
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+vox_status launch_q4_gemm(const uint8_t* w, int64_t n, int64_t k, const void* x, int64_t m, int64_t ldx, void* y,
+                          int y_dtype, int64_t ldy, const vox_epilogue* ep, cudaStream_t s)
+{
+    GemmArgs a = {};
+    a.w = w;
+    a.n = n;
+    a.k = k;
+    a.tiles = (int32_t)ceil_div(n, 16);
+    a.kc = (int32_t)(k / 64);
+    a.m = m;
+    a.y = y;
+    a.y_bf16 = y_dtype == VOX_BF16;
+    a.ldy = ldy;
+    a.op = ep ? ep->op : VOX_EP_NONE;
+    a.res = ep ? ep->residual : nullptr;
+    a.ldr = ep ? ep->ldr : 0;
+    switch (pick_bn(a.tiles, m)) {
+    case 32: return launch_gemm_bn<32>(a, x, ldx, s);
+    case 64: return launch_gemm_bn<64>(a, x, ldx, s);
+    case 128: return launch_gemm_bn<128>(a, x, ldx, s);
+    default: return launch_gemm_bn<256>(a, x, ldx, s);
+    }
+}
+
+}  // namespace vox

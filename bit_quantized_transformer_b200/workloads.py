@@ -1,0 +1,242 @@
+"""Device-side state of the synthetic workloads, built through libvox.
+
+Weights are drawn by :mod:`synth` (GGUF Q4_0 blocks), copied to the GPU and
+repacked there by ``vox_q4_pack``; caches, activations and workspaces are
+plain torch allocations.  The objects keep every tensor alive and expose the
+``vox_decoder`` / ``vox_encoder`` descriptors of include/vox.h.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+import synth
+
+from . import vox as V
+
+
+def to_dev(a: np.ndarray, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def bf16_dev(bits: np.ndarray, device) -> torch.Tensor:
+    """bf16 bit patterns (uint16) -> device bfloat16 tensor with the same bits."""
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def pack_q4(qs: np.ndarray, d: np.ndarray, device, flags: int = V.VOX_PACK_PLAIN):
+    """GGUF (qs, d) -> packed device weight; returns (tensor, vox_q4_weight)."""
+    n, nb, _ = qs.shape
+    k = nb * 32
+    g = to_dev(synth.gguf_bytes(qs, d).reshape(-1), device)
+    packed = torch.empty(V.vox_q4_packed_bytes(n, k), dtype=torch.uint8, device=device)
+    V.vox_q4_pack(g, n, k, flags, packed)
+    del g
+    return packed, V.weight(packed, n, k)
+
+
+def stack_rows(*parts):
+    return (np.concatenate([p[0] for p in parts], axis=0), np.concatenate([p[1] for p in parts], axis=0))
+
+
+class DecoderModel:
+    """26-layer synthetic decoder (or fewer layers) with rolling caches.
+
+    ``filled`` positions 0..filled-1 are taken as already present in the
+    caches (their contents are the seeded N(0,1) bf16 draws); the next step
+    writes position ``filled``.
+    """
+
+    def __init__(self, shape: synth.DecoderShape, seed: int = 0, device="cuda", n_layers=None,
+                 filled: int = 0, token: int = 0, eps: float = 1e-5, window=None):
+        self.shape = shape
+        self.seed = seed
+        self.device = device
+        self.L = shape.n_layers if n_layers is None else n_layers
+        self.W = shape.window if window is None else window
+        self.eps = eps
+        D, F = shape.dim, shape.ffn
+        QD, KVD = shape.q_dim, shape.kv_dim
+        keep = []
+        wqkv, wo, w13, w2, kc, vc = [], [], [], [], [], []
+        for l in range(self.L):
+            w = synth.decoder_layer_weights(shape, l, seed)
+            t, desc = pack_q4(*stack_rows(w["wq"], w["wk"], w["wv"]), device)
+            keep.append(t); wqkv.append(desc)
+            t, desc = pack_q4(*w["wo"], device)
+            keep.append(t); wo.append(desc)
+            t, desc = pack_q4(*stack_rows(w["w1"], w["w3"]), device, V.VOX_PACK_GATE_UP)
+            keep.append(t); w13.append(desc)
+            t, desc = pack_q4(*w["w2"], device)
+            keep.append(t); w2.append(desc)
+            kb, vb = synth.decoder_layer_cache(shape, l, seed, self.W)
+            kt, vt = bf16_dev(kb, device), bf16_dev(vb, device)
+            keep += [kt, vt]
+            kc.append(kt.data_ptr()); vc.append(vt.data_ptr())
+        self.emb_t, emb = pack_q4(*synth.q4_blocks(shape.vocab, D, seed, synth.EMB_ID), device)
+        self.lm_t, lm = pack_q4(*synth.q4_blocks(shape.vocab, D, seed, synth.LM_HEAD_ID), device)
+        self._keep = keep
+        self.wqkv, self.wo, self.w13, self.w2 = wqkv, wo, w13, w2
+        self.k_cache = [keep[6 * l + 4] for l in range(self.L)]
+        self.v_cache = [keep[6 * l + 5] for l in range(self.L)]
+
+        f32 = dict(dtype=torch.float32, device=device)
+        self.token = torch.tensor([token], dtype=torch.int32, device=device)
+        self.pos = torch.tensor([filled], dtype=torch.int64, device=device)
+        self.x = torch.zeros(D, **f32)
+        self.h = torch.zeros(D, **f32)
+        self.qkv = torch.zeros(QD + 2 * KVD, **f32)
+        self.attn = torch.zeros(QD, **f32)
+        self.act = torch.zeros(F, **f32)
+        self.logits = torch.zeros(shape.vocab, **f32)
+
+        Arr = V.vox_q4_weight * self.L
+        Ptr = ctypes.c_void_p * self.L
+        self._arrs = [Arr(*wqkv), Arr(*wo), Arr(*w13), Arr(*w2), Ptr(*kc), Ptr(*vc)]
+        dec = V.vox_decoder()
+        dec.n_layers, dec.dim, dec.n_q_heads, dec.n_kv_heads = self.L, D, shape.n_q_heads, shape.n_kv_heads
+        dec.head_dim, dec.ffn, dec.vocab, dec.window, dec.eps = shape.head_dim, F, shape.vocab, self.W, eps
+        dec.wqkv, dec.wo, dec.w13, dec.w2 = [ctypes.cast(a, ctypes.POINTER(V.vox_q4_weight)) for a in self._arrs[:4]]
+        dec.embedding, dec.lm_head = emb, lm
+        dec.k_cache = ctypes.cast(self._arrs[4], ctypes.POINTER(ctypes.c_void_p))
+        dec.v_cache = ctypes.cast(self._arrs[5], ctypes.POINTER(ctypes.c_void_p))
+        for name in ("token", "pos", "x", "h", "qkv", "attn", "act", "logits"):
+            setattr(dec, name, getattr(self, name).data_ptr())
+        ws = V.vox_decoder_workspace(dec)
+        self.workspace = torch.zeros(ws, dtype=torch.uint8, device=device)
+        dec.workspace, dec.ws_bytes = self.workspace.data_ptr(), ws
+        self.dec = dec
+        self.emb, self.lm = emb, lm
+
+    def step(self, stream=None):
+        V.vox_decoder_step(self.dec, stream)
+
+    # ----------------------------------------------------------- graphs
+    def capture(self, fn=None):
+        """Capture `fn` (default: one decoder step) into a CUDA graph.  One
+        eager run on a side stream first, as torch requires before capture."""
+        fn = self.step if fn is None else fn
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    def gemv_chain(self):
+        """The step's projections alone (same launches, weights and epilogues
+        as vox_decoder_step, without attention): used to time the GEMV."""
+        QD, KVD, D, F = self.shape.q_dim, self.shape.kv_dim, self.shape.dim, self.shape.ffn
+        ws = self.workspace
+        for l in range(self.L):
+            e = V.vox_epilogue(op=V.VOX_EP_KV_APPEND, rmsnorm=1, eps=self.eps, k_cache=self.k_cache[l].data_ptr(),
+                               v_cache=self.v_cache[l].data_ptr(), n_kv_heads=self.shape.n_kv_heads,
+                               head_dim=self.shape.head_dim, window=self.W, q_rows=QD, pos_dev=self.pos.data_ptr())
+            V.vox_q4_gemv(self.wqkv[l], self.x, 1, D, self.qkv, QD + 2 * KVD, e, ws, ws.numel())
+            r = V.vox_epilogue(op=V.VOX_EP_RESIDUAL, residual=self.x.data_ptr(), ldr=D)
+            V.vox_q4_gemv(self.wo[l], self.attn, 1, QD, self.h, D, r, ws, ws.numel())
+            f = V.vox_epilogue(op=V.VOX_EP_SILU_MUL, rmsnorm=1, eps=self.eps)
+            V.vox_q4_gemv(self.w13[l], self.h, 1, D, self.act, F, f, ws, ws.numel())
+            r2 = V.vox_epilogue(op=V.VOX_EP_RESIDUAL, residual=self.h.data_ptr(), ldr=D)
+            V.vox_q4_gemv(self.w2[l], self.act, 1, F, self.x, D, r2, ws, ws.numel())
+        am = V.vox_epilogue(op=V.VOX_EP_ARGMAX, rmsnorm=1, eps=self.eps, argmax=self.token.data_ptr())
+        V.vox_q4_gemv(self.lm, self.x, 1, D, self.logits, self.shape.vocab, am, ws, ws.numel())
+
+    def gemv_chain_launches(self) -> int:
+        return 4 * self.L + 1
+
+    def gemv_chain_bytes(self) -> int:
+        return sum(w.n * w.k * 18 // 32 for w in self.wqkv + self.wo + self.w13 + self.w2) + \
+            self.shape.vocab * self.shape.dim * 18 // 32
+
+    def attn_chain(self, pos: int):
+        """The step's attention launches alone (per layer: split-KV + combine),
+        at a host-given position."""
+        wsb = V.vox_gqa_decode_attn_workspace(self.shape.n_q_heads, self.shape.n_kv_heads, self.shape.head_dim,
+                                              self.W)
+        ws = self.workspace[self.workspace.numel() - wsb:]
+        for l in range(self.L):
+            V.vox_gqa_decode_attn(self.qkv, self.k_cache[l], self.v_cache[l], self.attn, self.shape.n_q_heads,
+                                  self.shape.n_kv_heads, self.shape.head_dim, self.W, pos,
+                                  1.0 / self.shape.head_dim ** 0.5, ws, wsb)
+
+    def step_launches(self) -> int:
+        """Kernels one vox_decoder_step launches."""
+        return 1 + self.L * 6 + 1 + 1
+
+    def weight_bytes(self) -> int:
+        """Packed Q4 bytes streamed per step (all layers + LM head + one embedding row)."""
+        tot = sum(w.n * w.k * 18 // 32 for w in self.wqkv + self.wo + self.w13 + self.w2)
+        return tot + self.shape.vocab * self.shape.dim * 18 // 32 + self.shape.dim * 18 // 32
+
+    def kv_bytes(self, pos: int) -> int:
+        """bf16 K and V bytes the attention reads after position ``pos`` was written."""
+        nv = min(pos + 1, self.W)
+        return self.L * 2 * self.shape.n_kv_heads * nv * self.shape.head_dim * 2
+
+
+class EncoderModel:
+    """Synthetic encoder chunk: rows x dim input, per-layer history caches, adapter."""
+
+    def __init__(self, shape: synth.EncoderShape, seed: int = 0, device="cuda", n_layers=None, eps: float = 1e-5):
+        self.shape = shape
+        self.L = shape.n_layers if n_layers is None else n_layers
+        D, F, R = shape.dim, shape.ffn, shape.rows
+        keep = []
+        wqkv, wo, wup, wdown, kh, vh = [], [], [], [], [], []
+        for l in range(self.L):
+            w = synth.encoder_layer_weights(shape, l, seed)
+            for key, lst in (("wqkv", wqkv), ("wo", wo), ("wup", wup), ("wdown", wdown)):
+                t, desc = pack_q4(*w[key], device)
+                keep.append(t); lst.append(desc)
+            kb, vb = synth.encoder_layer_history(shape, l, seed)
+            kt, vt = bf16_dev(kb, device), bf16_dev(vb, device)
+            keep += [kt, vt]
+            kh.append(kt.data_ptr()); vh.append(vt.data_ptr())
+        self.ad_t, ad = pack_q4(*synth.q4_blocks(shape.adapter_out, shape.downsample * D, seed, synth.ADAPTER_ID),
+                                device)
+        self._keep = keep
+        self.wqkv, self.wo, self.wup, self.wdown = wqkv, wo, wup, wdown
+        self.k_hist = [keep[6 * l + 4] for l in range(self.L)]
+        self.v_hist = [keep[6 * l + 5] for l in range(self.L)]
+        self.x0 = to_dev(synth.activations(R, D, seed, synth.ENC_X_ID), device)
+        self.x = self.x0.clone()
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.xn = torch.zeros(R, D, **bf)
+        self.qkv = torch.zeros(R, 3 * D, **bf)
+        self.att = torch.zeros(R, D, **bf)
+        self.up = torch.zeros(R, F, **bf)
+        self.out = torch.zeros(R // shape.downsample, shape.adapter_out, dtype=torch.float32, device=device)
+        Arr = V.vox_q4_weight * self.L
+        Ptr = ctypes.c_void_p * self.L
+        self._arrs = [Arr(*wqkv), Arr(*wo), Arr(*wup), Arr(*wdown), Ptr(*kh), Ptr(*vh)]
+        e = V.vox_encoder()
+        e.n_layers, e.dim, e.n_heads, e.head_dim = self.L, D, shape.n_heads, shape.head_dim
+        e.ffn, e.window, e.rows, e.adapter_out, e.eps = F, shape.window, R, shape.adapter_out, eps
+        e.wqkv, e.wo, e.wup, e.wdown = [ctypes.cast(a, ctypes.POINTER(V.vox_q4_weight)) for a in self._arrs[:4]]
+        e.adapter = ad
+        e.k_hist = ctypes.cast(self._arrs[4], ctypes.POINTER(ctypes.c_void_p))
+        e.v_hist = ctypes.cast(self._arrs[5], ctypes.POINTER(ctypes.c_void_p))
+        for name in ("x", "xn", "qkv", "att", "up"):
+            setattr(e, name, getattr(self, name).data_ptr())
+        e.adapter_out_buf = self.out.data_ptr()
+        self.enc = e
+        self.adapter = ad
+
+    def reset(self):
+        self.x.copy_(self.x0)
+
+    def run(self, stream=None):
+        V.vox_encoder_chunk(self.enc, stream)
+
+    def gemm_flops(self) -> int:
+        s = self.shape
+        R, D, F = s.rows, s.dim, s.ffn
+        per_layer = 2 * R * D * (3 * D + D + F) + 2 * R * F * D
+        return self.L * per_layer + 2 * (R // s.downsample) * (s.downsample * D) * s.adapter_out

@@ -1,0 +1,302 @@
+/*
+ * vox.h -- C ABI of the B200 (sm_100a) Q4_0 decode/encode hot path of
+ * Voxtral Mini 4B Realtime.
+ *
+ * Plain C: every pointer is a raw address, every size an integer, and the
+ * stream is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ * "device" pointers are CUDA device memory owned by the caller; the library
+ * never allocates, never frees and never synchronises.  All calls are
+ * asynchronous on the given stream.  Arguments are validated on the host
+ * before anything is launched; a call that returns an error has launched
+ * nothing (except VOX_ERR_CUDA, which reports a failed launch).
+ *
+ * Sources of the operations (page titles and sections as on the pages):
+ *  [Q4]   "Voxtral Mini 4B Realtime (Rust)", page 5, "Arquitetura": the Q4
+ *         GGUF path quantises with GGUF Q4_0 and runs custom shaders.
+ *         Q4_0 block: fp16 scale d + 16 bytes holding 32 4-bit codes q,
+ *         weight w = (q - 8) * d; element j < 16 is the low nibble of byte j,
+ *         element j + 16 the high nibble (GGUF order).
+ *  [FUSE] "브라우저에서 도는 4B 음성인식: Voxtral Rust+WASM 구현 해부", section
+ *         "F32(9GB) vs Q4 GGUF(2.5GB)": dequantisation fused into the matmul.
+ *  [EMB]  same page, and "Voxtral Mini 4B Realtime (Rust)" page 5 "Soluções
+ *         técnicas": the 1.5 GiB embedding table kept as Q4 on the GPU with
+ *         single-row lookups.
+ *  [ARCH] "Mistral Voxtral Realtime 4B ... 순수 C 기반 CPU 전용 추론 구현",
+ *         "모델 아키텍처": decoder 26 layers, dim 3072, GQA 32 query / 8 KV
+ *         heads; encoder 32 causal layers, dim 1280, 32 heads, window 750;
+ *         adapter Linear(5120->3072) -> GELU -> Linear; vocabulary 131072.
+ *  [ROLL] same page, "주요 기능": rolling KV cache, an 8192-position sliding
+ *         window that keeps memory constant for unbounded audio.
+ *  [BATCH] same page, "주요 기능": fused GPU ops and batched attention; and
+ *         "성능 벤치마크": the decoder runs a whole token step as one GPU
+ *         submission.
+ */
+#ifndef VOX_H
+#define VOX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------ status codes */
+typedef int32_t vox_status;
+enum {
+    VOX_OK = 0,
+    VOX_ERR_NULL = 1,       /* a required pointer is NULL                          */
+    VOX_ERR_SHAPE = 2,      /* a size is out of the supported set (k % 32 != 0 ...) */
+    VOX_ERR_ALIGN = 3,      /* a pointer or leading dimension breaks an alignment rule */
+    VOX_ERR_DTYPE = 4,      /* unsupported element type for this argument          */
+    VOX_ERR_RANGE = 5,      /* pos < 0, window <= 0, n_q % n_kv != 0, row out of range */
+    VOX_ERR_WORKSPACE = 6,  /* workspace NULL or smaller than the query call says   */
+    VOX_ERR_TIMEOUT = 7,    /* reserved: a bounded device-side wait gave up         */
+    VOX_ERR_CUDA = 8        /* a CUDA launch or query failed; see vox_last_error()   */
+};
+
+/* element types */
+enum { VOX_F32 = 0, VOX_BF16 = 1, VOX_F16 = 2 };
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *vox_status_str(vox_status s);
+/* Text of the last CUDA error seen by this thread in a vox_* call ("" if none). */
+const char *vox_last_error(void);
+/* Device status word of the calling thread's current device: 0 when every
+ * bounded device-side wait completed, else a code naming the wait that gave
+ * up (the kernel then returned early and its outputs are not valid).  This
+ * call synchronises the device; clear != 0 resets the word.  -1 if the word
+ * cannot be read. */
+int32_t vox_device_status(int32_t clear);
+
+/* ------------------------------------------------------- packed Q4_0 weight
+ * The GGUF blocks of an n x k matrix are repacked once ([Q4]: "repacked once
+ * for 16-byte vector loads") into a tiled layout of the same total size up to
+ * padding: rows are grouped in tiles of 16, columns in chunks of 64 (two
+ * blocks); each (tile, chunk) is 576 contiguous bytes -- 512 bytes of codes
+ * arranged so that one 16-byte load per lane feeds that lane's tensor-core
+ * fragments, then 64 bytes of the 32 fp16 scales.  Tiles are stored
+ * row-tile-major, chunks in k order.  Rows past n and columns past k are
+ * padding with d = 0 and q = 8 (weight 0).  The layout is internal: only the
+ * vox_* calls read it, and vox_q4_dequant returns the logical weights. */
+typedef struct {
+    const void *data;   /* device, vox_q4_packed_bytes(n, k) bytes, 16-byte aligned */
+    int64_t n;          /* output rows (logical)                                     */
+    int64_t k;          /* input columns, a multiple of 32                           */
+} vox_q4_weight;
+
+/* Bytes of the packed layout: ceil(n/16)*16 * ceil(k/64)*64 * 18/32.  -1 if
+ * n < 1 or k < 32 or k % 32 != 0. */
+int64_t vox_q4_packed_bytes(int64_t n, int64_t k);
+
+/* pack flags */
+enum {
+    VOX_PACK_PLAIN = 0,
+    /* The input holds [W1; W3] (n = 2F rows: F gate rows then F up rows, F a
+     * multiple of 8).  Packed row order interleaves groups of 8: packed rows
+     * 16j..16j+7 are W1 rows 8j..8j+7 and packed rows 16j+8..16j+15 are W3
+     * rows 8j..8j+7, which is what the VOX_EP_SILU_MUL epilogue expects. */
+    VOX_PACK_GATE_UP = 1
+};
+
+/* vox_q4_pack -- [Q4].  gguf: device, n * k/32 blocks of 18 bytes in GGUF
+ * order (row-major: block b of row r at byte (r*k/32 + b)*18; bytes 0-1 the
+ * little-endian fp16 d, bytes 2-17 the codes).  packed: device,
+ * vox_q4_packed_bytes(n, k) bytes, 16-byte aligned, fully written (padding
+ * included).  Errors: NULL pointers -> VOX_ERR_NULL; k % 32, n < 1 or a
+ * GATE_UP n that is not 2F with F % 8 == 0 -> VOX_ERR_SHAPE; packed not 16-byte
+ * aligned -> VOX_ERR_ALIGN; unknown flags -> VOX_ERR_RANGE. */
+vox_status vox_q4_pack(const void *gguf, int64_t n, int64_t k, int32_t flags, void *packed,
+                       void *stream);
+
+/* vox_q4_dequant -- [Q4], [EMB].  Writes w[r][c] = (q - 8) * d for packed
+ * rows r in [row0, row0 + nrows) and all k columns to out (device, row-major
+ * with leading dimension ldo >= k elements).  out_dtype VOX_F32 gives the
+ * exact product (it always fits fp32); VOX_BF16 rounds it to nearest-even
+ * (NaN -> 0x7FC0).  Row numbers are packed rows (for VOX_PACK_GATE_UP weights
+ * that is the interleaved order).  Errors: NULL -> VOX_ERR_NULL; rows outside
+ * [0, n) -> VOX_ERR_RANGE; ldo < k -> VOX_ERR_SHAPE; other dtypes ->
+ * VOX_ERR_DTYPE. */
+vox_status vox_q4_dequant(const vox_q4_weight *w, int64_t row0, int64_t nrows, void *out,
+                          int32_t out_dtype, int64_t ldo, void *stream);
+
+/* --------------------------------------------------------------- epilogues
+ * A small POD that fuses the work around a projection into the projection's
+ * kernel: an optional RMSNorm of each input row before the product (reading:
+ * x / sqrt(mean(x^2) + eps) * g, pre-norm), and one output operation. */
+enum {
+    VOX_EP_NONE = 0,      /* y = W x                                                  */
+    VOX_EP_RESIDUAL = 1,  /* y = residual + W x (residual may alias y)                 */
+    VOX_EP_SILU_MUL = 2,  /* W packed with VOX_PACK_GATE_UP: y[j] = silu(g_j) * u_j,
+                             y has n/2 columns; silu(a) = a / (1 + exp(-a))            */
+    VOX_EP_GELU = 3,      /* y = gelu(W x), exact erf form                             */
+    VOX_EP_KV_APPEND = 4, /* rows [0, q_rows) -> y as usual; rows [q_rows, q_rows+kv)
+                             are k and [q_rows+kv, q_rows+2kv) are v (kv =
+                             n_kv_heads*head_dim): they are also written to y and,
+                             rounded to bf16, into slot (pos + i) mod window of the
+                             caches for token i ([ROLL])                               */
+    VOX_EP_ARGMAX = 5     /* y = W x, and argmax[i] = index of the largest y[i][:],
+                             lowest index on ties, a NaN wins over numbers             */
+};
+
+typedef struct {
+    int32_t op;                /* VOX_EP_*                                            */
+    int32_t rmsnorm;           /* 1: normalise each input row first                    */
+    float eps;                 /* RMSNorm epsilon (1e-5 in this library's model)       */
+    const float *norm_weight;  /* device [k] gain g, or NULL for g = 1                 */
+    const float *residual;     /* RESIDUAL: device [m][ldr] fp32                       */
+    int64_t ldr;
+    void *k_cache;             /* KV_APPEND: device bf16 [n_kv_heads][window][head_dim] */
+    void *v_cache;
+    int32_t n_kv_heads, head_dim, window, q_rows;
+    int64_t pos;               /* KV_APPEND: position of input row 0                   */
+    const int64_t *pos_dev;    /* if not NULL, the position is read from device memory  */
+    int32_t *argmax;           /* ARGMAX: device int32 [m]                              */
+} vox_epilogue;
+
+/* ----------------------------------------------------------- Q4_0 GEMV (M<=8)
+ * vox_q4_gemv -- [Q4], [FUSE].  y[i][j] = sum_c w[j][c] * x[i][c] for
+ * i < m (1 <= m <= 8) and packed rows j < n, dequantising in registers with no
+ * separate pass, then the epilogue.  x: device fp32 [m][ldx]; y: device fp32
+ * [m][ldy] (n columns, or n/2 for SILU_MUL).  The product runs on the tensor
+ * cores with the activations rounded to fp16 after an exact per-row
+ * power-of-two scaling and fp32 accumulation; the result is within 2e-3 of
+ * the fp64 product, normalised by |x_i| |w_j|.  workspace: device scratch of
+ * vox_q4_gemv_workspace() bytes, 16-byte aligned: per-tile arrival counters
+ * (for tiles split between CTAs), partial tiles and argmax candidates.  Zero
+ * it once before its first use; every call leaves the counters at zero
+ * again.  Calls that share a workspace must not overlap on the GPU.  Limits: m * ceil(k/64)*64 <= 81920.
+ * Errors: NULL -> VOX_ERR_NULL; m outside 1..8, k % 32, ldx < k, ldy too small,
+ * SILU_MUL with n % 16, KV_APPEND rows that do not fit n, or the size limit ->
+ * VOX_ERR_SHAPE; weight data not 16-byte aligned -> VOX_ERR_ALIGN; bad
+ * epilogue fields -> VOX_ERR_RANGE; short workspace -> VOX_ERR_WORKSPACE. */
+vox_status vox_q4_gemv(const vox_q4_weight *w, const float *x, int64_t m, int64_t ldx,
+                       float *y, int64_t ldy, const vox_epilogue *ep,
+                       void *workspace, size_t ws_bytes, void *stream);
+size_t vox_q4_gemv_workspace(const vox_q4_weight *w, int64_t m, const vox_epilogue *ep);
+
+/* ------------------------------------------------------ Q4_0 GEMM (M >= 16)
+ * vox_q4_gemm -- [Q4], [FUSE], encoder chunks and batched rows.
+ * Y = X W^T: y[i][j] = sum_c x[i][c] w[j][c] for i < m, j < n.  x: device bf16
+ * [m][ldx] (ldx a multiple of 8, x 16-byte aligned).  The packed weights are
+ * staged by TMA into shared memory, dequantised there to bf16 and fed to the
+ * tcgen05 tensor cores with fp32 accumulation in tensor memory.  y: device
+ * [m][ldy] of y_dtype VOX_F32 or VOX_BF16.  Epilogues: NONE, RESIDUAL
+ * (fp32 y only), GELU; no RMSNorm prologue (use vox_rmsnorm first).  Errors as
+ * for vox_q4_gemv; m < 1 or k % 64 -> VOX_ERR_SHAPE. */
+vox_status vox_q4_gemm(const vox_q4_weight *w, const void *x, int32_t x_dtype, int64_t m,
+                       int64_t ldx, void *y, int32_t y_dtype, int64_t ldy,
+                       const vox_epilogue *ep, void *stream);
+
+/* ------------------------------------------------------------ rolling cache
+ * vox_kv_append_rolling -- [ROLL].  Stores one position: k_new and v_new
+ * (device [n_kv_heads][head_dim] of new_dtype VOX_F32 or VOX_BF16) are
+ * rounded to bf16 (nearest-even) and written to slot pos mod window of
+ * k_cache / v_cache (device bf16 [n_kv_heads][window][head_dim]).  After the
+ * call the valid slots are the first min(pos + 1, window).  Errors: NULL ->
+ * VOX_ERR_NULL; pos < 0 or window <= 0 -> VOX_ERR_RANGE; head_dim outside
+ * 1..1024 or n_kv_heads < 1 -> VOX_ERR_SHAPE. */
+vox_status vox_kv_append_rolling(void *k_cache, void *v_cache, const void *k_new, const void *v_new,
+                                 int32_t new_dtype, int32_t n_kv_heads, int32_t head_dim,
+                                 int32_t window, int64_t pos, void *stream);
+
+/* vox_gqa_decode_attn -- [ARCH] GQA, [ROLL], [BATCH].  One decode query per
+ * head over the rolling cache after position pos was written: query head h
+ * reads kv head h / (n_q_heads / n_kv_heads); s_j = scale * q_h . k_j over the
+ * valid slots j < min(pos + 1, window); out_h = softmax(s) . V.  q: device fp32
+ * [n_q_heads][head_dim]; caches: device bf16 [n_kv_heads][window][head_dim],
+ * 16-byte aligned; out: device fp32 [n_q_heads][head_dim].  Split-KV: slot
+ * ranges are reduced independently into the workspace (device, at least
+ * vox_gqa_decode_attn_workspace() bytes, 16-byte aligned, no initial contents
+ * needed) and merged by a log-sum-exp combine.  Calls sharing a workspace
+ * must not overlap on the GPU.  head_dim must be 128 (the decoder's).
+ * Errors: NULL -> VOX_ERR_NULL; pos < 0, window <= 0, n_q % n_kv != 0, a
+ * group above 8 or more than 512 kv heads -> VOX_ERR_RANGE; other head_dim
+ * -> VOX_ERR_SHAPE; short workspace -> VOX_ERR_WORKSPACE; caches or workspace
+ * not 16-byte aligned -> VOX_ERR_ALIGN. */
+vox_status vox_gqa_decode_attn(const float *q, const void *k_cache, const void *v_cache, float *out,
+                               int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                               int32_t window, int64_t pos, float scale,
+                               void *workspace, size_t ws_bytes, void *stream);
+size_t vox_gqa_decode_attn_workspace(int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                     int32_t window);
+
+/* vox_window_attn -- [ARCH] encoder: causal sliding-window multi-head
+ * attention for a chunk of n_q query rows.  Query row i sits at absolute
+ * position n_hist + i and sees key position p iff pos_i - window < p <= pos_i.
+ * Keys/values at positions < n_hist come from k_hist/v_hist rows (device bf16
+ * [n_hist][ld_hist]); positions n_hist + i from k_new/v_new rows (device bf16
+ * [n_q][ld_new]).  Head h uses columns [h*head_dim, (h+1)*head_dim).  q: device
+ * bf16 [n_q][ldq]; out: device [n_q][ldo] of out_dtype VOX_F32 or VOX_BF16.
+ * Errors: NULL -> VOX_ERR_NULL; window <= 0 -> VOX_ERR_RANGE; head_dim not in
+ * 1..64 or leading dimensions too small -> VOX_ERR_SHAPE. */
+vox_status vox_window_attn(const void *q, int64_t ldq, const void *k_hist, const void *v_hist,
+                           int64_t ld_hist, int64_t n_hist, const void *k_new, const void *v_new,
+                           int64_t ld_new, int64_t n_q, void *out, int32_t out_dtype, int64_t ldo,
+                           int32_t n_heads, int32_t head_dim, int32_t window, float scale,
+                           void *stream);
+
+/* ---------------------------------------------------------------- glue ops
+ * vox_rmsnorm -- pre-norm of the decoder and encoder layers (reading: eps
+ * inside the square root, gain g or 1).  x: device fp32 [m][ldx]; out: device
+ * [m][ldo] of out_dtype VOX_F32 or VOX_BF16. */
+vox_status vox_rmsnorm(const float *x, int64_t m, int64_t n, int64_t ldx, float eps,
+                       const float *g, void *out, int32_t out_dtype, int64_t ldo, void *stream);
+
+/* ------------------------------------------------------------ composed path
+ * The decoder token step and the encoder chunk, built from the calls above
+ * and launched back to back on one stream (the pages' "one submission per
+ * token step"; the caller may capture the call in a CUDA graph). */
+typedef struct {
+    int32_t n_layers, dim, n_q_heads, n_kv_heads, head_dim, ffn, vocab, window;
+    float eps;
+    const vox_q4_weight *wqkv;   /* host array [n_layers]: [Wq; Wk; Wv], (q+2kv) x dim */
+    const vox_q4_weight *wo;     /* host array [n_layers]: dim x q_dim                  */
+    const vox_q4_weight *w13;    /* host array [n_layers]: VOX_PACK_GATE_UP, 2ffn x dim */
+    const vox_q4_weight *w2;     /* host array [n_layers]: dim x ffn                    */
+    vox_q4_weight embedding;     /* vocab x dim                                         */
+    vox_q4_weight lm_head;       /* vocab x dim                                         */
+    void *const *k_cache;        /* host array [n_layers] of device bf16 caches         */
+    void *const *v_cache;
+    int32_t *token;              /* device [1]: input token; receives the argmax          */
+    int64_t *pos;                /* device [1]: this step's position; incremented at end   */
+    float *x, *h, *qkv, *attn, *act, *logits;  /* device activations: dim, dim,
+                                    q+2kv, q_dim, ffn, vocab floats                     */
+    void *workspace;             /* device, vox_decoder_workspace() bytes, zero-filled once */
+    size_t ws_bytes;
+} vox_decoder;
+
+size_t vox_decoder_workspace(const vox_decoder *dec);
+/* One greedy decode step: x = embedding[token]; 26 x {RMSNorm + QKV GEMV with
+ * rolling append, GQA attention, Wo GEMV + residual, RMSNorm + W1||W3 GEMV +
+ * SiLU*mul, W2 GEMV + residual}; RMSNorm + LM head GEMV + argmax -> token;
+ * pos += 1. */
+vox_status vox_decoder_step(const vox_decoder *dec, void *stream);
+
+typedef struct {
+    int32_t n_layers, dim, n_heads, head_dim, ffn, window, rows, adapter_out;
+    float eps;
+    const vox_q4_weight *wqkv;   /* host array [n_layers]: 3dim x dim                   */
+    const vox_q4_weight *wo;     /* dim x dim                                           */
+    const vox_q4_weight *wup;    /* ffn x dim                                           */
+    const vox_q4_weight *wdown;  /* dim x ffn                                           */
+    vox_q4_weight adapter;       /* adapter_out x 4dim                                   */
+    const void *const *k_hist;   /* host array [n_layers] of device bf16 [window][dim]  */
+    const void *const *v_hist;
+    float *x;                    /* device fp32 [rows][dim]: chunk input, updated in place */
+    void *xn;                    /* device bf16 [rows][dim] scratch                     */
+    void *qkv;                   /* device bf16 [rows][3dim] scratch                    */
+    void *att;                   /* device bf16 [rows][dim] scratch                     */
+    void *up;                    /* device bf16 [rows][ffn] scratch                     */
+    float *adapter_out_buf;      /* device fp32 [rows/4][adapter_out]                   */
+} vox_encoder;
+
+/* One encoder chunk: 32 x {RMSNorm, QKV GEMM, window attention, O GEMM +
+ * residual, RMSNorm, up GEMM + GELU, down GEMM + residual}, then the 4x
+ * downsample (rows 4r..4r+3 concatenated) and the adapter's first GEMM. */
+vox_status vox_encoder_chunk(const vox_encoder *enc, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VOX_H */

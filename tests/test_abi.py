@@ -1,0 +1,197 @@
+"""The C ABI: libvox.so loads without a GPU, exports every entry point that
+include/vox.h declares, and rejects bad arguments on the host with the
+documented status codes before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vox.h")
+
+
+@pytest.fixture(scope="module")
+def V():
+    from bit_quantized_transformer_b200 import build
+
+    build.build()
+    from bit_quantized_transformer_b200 import vox
+
+    return vox
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(vox_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("vox_q4_dequant", "vox_q4_gemv", "vox_q4_gemm", "vox_kv_append_rolling", "vox_gqa_decode_attn",
+                 "vox_q4_pack", "vox_decoder_step", "vox_encoder_chunk"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(V):
+    missing = [n for n in declared_functions() if not hasattr(V.lib, n)]
+    assert not missing, missing
+
+
+def test_library_exports_nothing_undeclared(V):
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", V.LIB_PATH], capture_output=True, text=True).stdout
+    exported = sorted({l.split()[-1] for l in out.splitlines() if " T vox_" in l})
+    assert exported == declared_functions()
+
+
+def test_status_strings(V):
+    assert V.lib.vox_status_str(0) == b"VOX_OK"
+    assert V.lib.vox_status_str(V.VOX_ERR_WORKSPACE) == b"VOX_ERR_WORKSPACE"
+    assert V.lib.vox_status_str(99) == b"VOX_ERR_UNKNOWN"
+
+
+def test_packed_bytes(V):
+    assert V.vox_q4_packed_bytes(4096, 3072) == 4096 * 3072 * 18 // 32
+    assert V.vox_q4_packed_bytes(17, 32) == 32 * 64 * 18 // 32        # padded to 2 tiles x 1 chunk
+    assert V.vox_q4_packed_bytes(16, 48) == -1
+    assert V.vox_q4_packed_bytes(0, 64) == -1
+
+
+FAKE = 0x10000          # a 16-byte aligned address; never dereferenced: validation fails first
+
+
+def test_pack_validation(V):
+    L = V.lib
+    assert L.vox_q4_pack(None, 16, 64, 0, FAKE, None) == V.VOX_ERR_NULL
+    assert L.vox_q4_pack(FAKE, 16, 48, 0, FAKE, None) == V.VOX_ERR_SHAPE
+    assert L.vox_q4_pack(FAKE, 0, 64, 0, FAKE, None) == V.VOX_ERR_SHAPE
+    assert L.vox_q4_pack(FAKE, 16, 64, 7, FAKE, None) == V.VOX_ERR_RANGE
+    assert L.vox_q4_pack(FAKE, 24, 64, V.VOX_PACK_GATE_UP, FAKE, None) == V.VOX_ERR_SHAPE
+    assert L.vox_q4_pack(FAKE, 16, 64, 0, FAKE + 4, None) == V.VOX_ERR_ALIGN
+
+
+def test_dequant_validation(V):
+    L = V.lib
+    w = V.vox_q4_weight(FAKE, 32, 64)
+    assert L.vox_q4_dequant(ctypes.byref(w), 0, 1, None, V.VOX_F32, 64, None) == V.VOX_ERR_NULL
+    assert L.vox_q4_dequant(ctypes.byref(w), 0, 1, FAKE, V.VOX_F16, 64, None) == V.VOX_ERR_DTYPE
+    assert L.vox_q4_dequant(ctypes.byref(w), 31, 2, FAKE, V.VOX_F32, 64, None) == V.VOX_ERR_RANGE
+    assert L.vox_q4_dequant(ctypes.byref(w), -1, 1, FAKE, V.VOX_F32, 64, None) == V.VOX_ERR_RANGE
+    assert L.vox_q4_dequant(ctypes.byref(w), 0, 1, FAKE, V.VOX_F32, 63, None) == V.VOX_ERR_SHAPE
+    bad = V.vox_q4_weight(FAKE + 8, 32, 64)
+    assert L.vox_q4_dequant(ctypes.byref(bad), 0, 1, FAKE, V.VOX_F32, 64, None) == V.VOX_ERR_ALIGN
+    assert L.vox_q4_dequant(None, 0, 1, FAKE, V.VOX_F32, 64, None) == V.VOX_ERR_NULL
+
+
+def test_gemv_validation(V):
+    L = V.lib
+    w = V.vox_q4_weight(FAKE, 64, 96)
+    ws = V.vox_q4_gemv_workspace(w, 1, None)
+    assert ws > 0
+    g = lambda m=1, ldx=96, ldy=64, ep=None, wsp=FAKE, wsb=ws, x=FAKE, y=FAKE: L.vox_q4_gemv(
+        ctypes.byref(w), x, m, ldx, y, ldy, ctypes.byref(ep) if ep else None, wsp, wsb, None)
+    assert g(x=None) == V.VOX_ERR_NULL
+    assert g(m=0) == V.VOX_ERR_SHAPE
+    assert g(m=9) == V.VOX_ERR_SHAPE
+    assert g(ldx=95) == V.VOX_ERR_SHAPE
+    assert g(ldy=63) == V.VOX_ERR_SHAPE
+    assert g(wsp=None) == V.VOX_ERR_WORKSPACE
+    assert g(wsb=ws - 1) == V.VOX_ERR_WORKSPACE
+    ep = V.vox_epilogue(op=V.VOX_EP_RESIDUAL, residual=None, ldr=64)
+    assert g(ep=ep) == V.VOX_ERR_NULL
+    ep = V.vox_epilogue(op=9)
+    assert g(ep=ep) == V.VOX_ERR_RANGE
+    ep = V.vox_epilogue(op=V.VOX_EP_KV_APPEND, k_cache=FAKE, v_cache=FAKE, n_kv_heads=1, head_dim=32, window=4,
+                        q_rows=8, pos=0)
+    assert g(ep=ep) == V.VOX_ERR_SHAPE            # 8 + 2*32 rows > 64
+    ep = V.vox_epilogue(op=V.VOX_EP_KV_APPEND, k_cache=FAKE, v_cache=FAKE, n_kv_heads=1, head_dim=16, window=4,
+                        q_rows=8, pos=-1)
+    assert g(ep=ep) == V.VOX_ERR_RANGE
+    ep = V.vox_epilogue(op=V.VOX_EP_ARGMAX, argmax=None)
+    assert g(ep=ep) == V.VOX_ERR_NULL
+    wide = V.vox_q4_weight(FAKE, 64, 16384)
+    assert L.vox_q4_gemv(ctypes.byref(wide), FAKE, 8, 16384, FAKE, 64, None, FAKE, 1 << 30, None) == V.VOX_ERR_SHAPE
+    ep = V.vox_epilogue(op=V.VOX_EP_SILU_MUL)
+    w24 = V.vox_q4_weight(FAKE, 24, 96)
+    assert L.vox_q4_gemv(ctypes.byref(w24), FAKE, 1, 96, FAKE, 24, ctypes.byref(ep), FAKE, 1 << 30,
+                         None) == V.VOX_ERR_SHAPE
+
+
+def test_gemm_validation(V):
+    L = V.lib
+    w = V.vox_q4_weight(FAKE, 128, 128)
+    g = lambda xd=V.VOX_BF16, m=16, ldx=128, yd=V.VOX_F32, ldy=128, ep=None, x=FAKE: L.vox_q4_gemm(
+        ctypes.byref(w), x, xd, m, ldx, FAKE, yd, ldy, ctypes.byref(ep) if ep else None, None)
+    assert g(x=None) == V.VOX_ERR_NULL
+    assert g(xd=V.VOX_F32) == V.VOX_ERR_DTYPE
+    assert g(yd=V.VOX_F16) == V.VOX_ERR_DTYPE
+    assert g(m=0) == V.VOX_ERR_SHAPE
+    assert g(ldx=130) == V.VOX_ERR_SHAPE
+    assert g(x=FAKE + 2) == V.VOX_ERR_ALIGN
+    assert g(ep=V.vox_epilogue(op=V.VOX_EP_ARGMAX, argmax=FAKE)) == V.VOX_ERR_RANGE
+    assert g(ep=V.vox_epilogue(op=V.VOX_EP_RESIDUAL, residual=FAKE, ldr=128), yd=V.VOX_BF16) == V.VOX_ERR_DTYPE
+    w96 = V.vox_q4_weight(FAKE, 128, 96)
+    assert L.vox_q4_gemm(ctypes.byref(w96), FAKE, V.VOX_BF16, 16, 96, FAKE, V.VOX_F32, 128, None,
+                         None) == V.VOX_ERR_SHAPE
+
+
+def test_kv_and_attention_validation(V):
+    L = V.lib
+    assert L.vox_kv_append_rolling(None, FAKE, FAKE, FAKE, 0, 8, 128, 16, 0, None) == V.VOX_ERR_NULL
+    assert L.vox_kv_append_rolling(FAKE, FAKE, FAKE, FAKE, 0, 8, 128, 16, -1, None) == V.VOX_ERR_RANGE
+    assert L.vox_kv_append_rolling(FAKE, FAKE, FAKE, FAKE, 0, 8, 128, 0, 0, None) == V.VOX_ERR_RANGE
+    assert L.vox_kv_append_rolling(FAKE, FAKE, FAKE, FAKE, 2, 8, 128, 16, 0, None) == V.VOX_ERR_DTYPE
+    ws = V.vox_gqa_decode_attn_workspace(32, 8, 128, 8192)
+    assert ws > 0
+    a = lambda nq=32, nkv=8, hd=128, W=8192, pos=0, wsp=FAKE, wsb=ws, kc=FAKE: L.vox_gqa_decode_attn(
+        FAKE, kc, FAKE, FAKE, nq, nkv, hd, W, pos, 0.088, wsp, wsb, None)
+    assert a(kc=None) == V.VOX_ERR_NULL
+    assert a(nq=30) == V.VOX_ERR_RANGE
+    assert a(nq=80, nkv=8) == V.VOX_ERR_RANGE     # group of 10 > 8
+    assert a(pos=-1) == V.VOX_ERR_RANGE
+    assert a(W=0) == V.VOX_ERR_RANGE
+    assert a(hd=64) == V.VOX_ERR_SHAPE
+    assert a(wsp=None) == V.VOX_ERR_WORKSPACE
+    assert a(wsb=ws - 16) == V.VOX_ERR_WORKSPACE
+    assert a(kc=FAKE + 2) == V.VOX_ERR_ALIGN
+
+
+def test_window_attn_and_rmsnorm_validation(V):
+    L = V.lib
+    w = lambda hd=40, W=750, nq=256, ldq=3840, od=V.VOX_BF16, q=FAKE: L.vox_window_attn(
+        q, ldq, FAKE, FAKE, 1280, 750, FAKE, FAKE, 3840, nq, FAKE, od, 1280, 32, hd, W, 0.158, None)
+    assert w(q=None) == V.VOX_ERR_NULL
+    assert w(W=0) == V.VOX_ERR_RANGE
+    assert w(hd=65) == V.VOX_ERR_SHAPE
+    assert w(ldq=1000) == V.VOX_ERR_SHAPE
+    assert w(od=V.VOX_F16) == V.VOX_ERR_DTYPE
+    r = L.vox_rmsnorm
+    assert r(None, 1, 64, 64, 1e-5, None, FAKE, V.VOX_F32, 64, None) == V.VOX_ERR_NULL
+    assert r(FAKE, 1, 64, 63, 1e-5, None, FAKE, V.VOX_F32, 64, None) == V.VOX_ERR_SHAPE
+    assert r(FAKE, 1, 64, 64, -1.0, None, FAKE, V.VOX_F32, 64, None) == V.VOX_ERR_RANGE
+
+
+def test_composed_validation(V):
+    L = V.lib
+    d = V.vox_decoder()
+    assert L.vox_decoder_step(None, None) == V.VOX_ERR_NULL
+    assert L.vox_decoder_step(ctypes.byref(d), None) == V.VOX_ERR_NULL
+    e = V.vox_encoder()
+    assert L.vox_encoder_chunk(ctypes.byref(e), None) == V.VOX_ERR_NULL
+
+
+def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
+    """The binding refuses to import when libvox.so is absent (no fallback)."""
+    import importlib.util
+    import shutil
+
+    pkg = tmp_path / "pkgcopy"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "bit_quantized_transformer_b200", "vox.py"), pkg / "vox.py")
+    spec = importlib.util.spec_from_file_location("vox_copy", pkg / "vox.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

@@ -1,0 +1,237 @@
+"""Parity of the composed paths (vox_decoder_step, vox_encoder_chunk) with the
+oracle, kernel by kernel on the GPU's own inputs to each kernel (teacher
+forcing, so errors do not compound), at the benchmark's full sizes.
+
+* one decoder layer, KV length 1024 (every kernel of the layer checked);
+* the full 26-layer step with the cache filled to 8192 + 300 (wrapped): the
+  last layer's attention, FFN and residual, the LM head on sampled rows and
+  the argmax;
+* one encoder layer + the adapter GEMM at M = 256.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import ref
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def env():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from bit_quantized_transformer_b200 import build
+
+    build.build()
+    from bit_quantized_transformer_b200 import vox as V
+    from bit_quantized_transformer_b200 import workloads as WL
+
+    return torch, V, WL
+
+
+def np_of(t):
+    return t.detach().cpu().numpy()
+
+
+def bits(t):
+    import torch
+
+    return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def gemv_err(y, x, qs, d, extra=None):
+    W = ref.q4_weights(qs, d)
+    want = np.atleast_2d(x).astype(np.float64) @ W.T
+    if extra is not None:
+        want = want + extra
+    return ref.gemv_error(np.atleast_2d(y), want, x, W)
+
+
+def check_layer_tail(shape, layer, dm, seed, pos_written):
+    """Attention, FFN and the final residual of `layer` from the GPU buffers."""
+    D, QD, KVD, F = shape.dim, shape.q_dim, shape.kv_dim, shape.ffn
+    w = synth.decoder_layer_weights(shape, layer, seed)
+    qkv = np_of(dm.qkv)
+    kc, vc = bits(dm.k_cache[layer]), bits(dm.v_cache[layer])
+    # the rolling append wrote bf16 of this step's k and v at slot pos mod W
+    slot = pos_written % dm.W
+    assert np.array_equal(kc[:, slot], ref.f32_to_bf16(qkv[QD:QD + KVD]).reshape(shape.n_kv_heads, -1))
+    assert np.array_equal(vc[:, slot], ref.f32_to_bf16(qkv[QD + KVD:]).reshape(shape.n_kv_heads, -1))
+    k0, v0 = synth.decoder_layer_cache(shape, layer, seed, dm.W)
+    others = np.ones(dm.W, bool)
+    others[slot] = False
+    assert np.array_equal(kc[:, others], k0[:, others]) and np.array_equal(vc[:, others], v0[:, others])
+    # attention on the GPU's q and caches
+    q = qkv[:QD].reshape(shape.n_q_heads, shape.head_dim)
+    o = np_of(dm.attn).reshape(shape.n_q_heads, shape.head_dim)
+    o_ref = ref.c_gqa_attn(q, kc, vc, pos_written)
+    nv = min(pos_written + 1, dm.W)
+    err_attn = ref.attn_error(o, o_ref, ref.attn_probs(q, kc, pos_written), ref.bf16_to_f64(vc[:, :nv]),
+                              shape.n_q_heads // shape.n_kv_heads)
+    assert err_attn <= TOL, err_attn
+    # FFN on the GPU's h: a = silu(W1 n2) * (W3 n2)
+    h = np_of(dm.h)
+    n2 = ref.rmsnorm(h)
+    g = n2 @ ref.q4_weights(*w["w1"]).T
+    u = n2 @ ref.q4_weights(*w["w3"]).T
+    a = np_of(dm.act)
+    w1n = np.linalg.norm(ref.q4_weights(*w["w1"]), axis=1)
+    w3n = np.linalg.norm(ref.q4_weights(*w["w3"]), axis=1)
+    bound = 1.1 * np.abs(u) * np.linalg.norm(n2) * w1n + np.abs(ref.silu(g)) * np.linalg.norm(n2) * w3n
+    assert np.all(np.abs(a - ref.silu(g) * u) <= TOL * bound)
+    # x_out = h + W2 a
+    x_out = np_of(dm.x)
+    err_w2 = gemv_err((x_out - h)[None], a[None], *w["w2"])
+    assert err_w2 <= TOL, err_w2
+    return w, o
+
+
+def test_decoder_layer_kv1024(env):
+    torch, V, WL = env
+    shape = synth.DecoderShape()
+    tok = 4242
+    dm = WL.DecoderModel(shape, seed=0, n_layers=1, filled=1024, token=tok)
+    dm.step()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    assert int(dm.pos.item()) == 1025
+    D, QD, KVD = shape.dim, shape.q_dim, shape.kv_dim
+    # x0 = embedding row, exact
+    eq, ed = synth.q4_blocks(shape.vocab, D, 0, synth.EMB_ID)
+    x0 = ref.c_dequant_f32(eq, ed, row0=tok, nrows=1)[0]
+    # QKV on the GPU's (exact) x0 with the RMSNorm prologue
+    w = synth.decoder_layer_weights(shape, 0, 0)
+    qs = np.concatenate([w["wq"][0], w["wk"][0], w["wv"][0]])
+    ds = np.concatenate([w["wq"][1], w["wk"][1], w["wv"][1]])
+    n0 = ref.rmsnorm(x0)
+    err_qkv = gemv_err(np_of(dm.qkv)[None], n0[None], qs, ds)
+    assert err_qkv <= TOL, err_qkv
+    w, o = check_layer_tail(shape, 0, dm, 0, 1024)
+    # Wo + residual on the GPU's attention output
+    err_wo = gemv_err((np_of(dm.h) - x0)[None], np_of(dm.attn)[None], *w["wo"])
+    assert err_wo <= TOL, err_wo
+    # LM head on sampled rows + greedy argmax of the GPU's logits
+    lq, ld = synth.q4_blocks(shape.vocab, D, 0, synth.LM_HEAD_ID)
+    logits = np_of(dm.logits)
+    xf = ref.rmsnorm(np_of(dm.x))
+    rows = np.unique(np.concatenate([np.random.default_rng(1).integers(0, shape.vocab, 256),
+                                     [int(np.argmax(logits))]]))
+    err_lm = gemv_err(logits[rows][None], xf[None], lq[rows], ld[rows])
+    assert err_lm <= TOL, err_lm
+    assert int(dm.token.item()) == int(np.argmax(logits))
+    # end to end (reported, not gated): the oracle's own fp64 layer from x0
+    Wd = {k: ref.q4_weights(*v) for k, v in w.items()}
+    k0, v0 = synth.decoder_layer_cache(shape, 0, 0, dm.W)
+    st = ref.decoder_layer(x0, Wd, k0.copy(), v0.copy(), 1024, shape.n_q_heads, shape.n_kv_heads)
+    e2e = np.max(np.abs(np_of(dm.x) - st["out"])) / np.max(np.abs(st["out"]))
+    print(f"decoder layer end-to-end max rel error {e2e:.3e}")
+
+
+def test_decoder_step_full_wrapped(env):
+    torch, V, WL = env
+    shape = synth.DecoderShape()
+    filled = 8192 + 300
+    dm = WL.DecoderModel(shape, seed=0, filled=filled, token=17)
+    dm.step()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    assert int(dm.pos.item()) == filled + 1
+    check_layer_tail(shape, shape.n_layers - 1, dm, 0, filled)
+    lq, ld = synth.q4_blocks(shape.vocab, shape.dim, 0, synth.LM_HEAD_ID)
+    logits = np_of(dm.logits)
+    xf = ref.rmsnorm(np_of(dm.x))
+    rows = np.unique(np.concatenate([np.random.default_rng(2).integers(0, shape.vocab, 512),
+                                     [int(np.argmax(logits))]]))
+    err_lm = gemv_err(logits[rows][None], xf[None], lq[rows], ld[rows])
+    assert err_lm <= TOL, err_lm
+    assert int(dm.token.item()) == int(np.argmax(logits))
+    # a second step advances the ring by one slot and reads the new token
+    dm.step()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    assert int(dm.pos.item()) == filled + 2
+    assert int(dm.token.item()) == int(np.argmax(np_of(dm.logits)))
+
+
+def test_decoder_step_graph_replay_matches_eager(env):
+    """The captured step replays exactly what the eager step computes."""
+    torch, V, WL = env
+    shape = synth.DecoderShape(n_layers=2)
+    a = WL.DecoderModel(shape, seed=3, filled=500, token=9)
+    b = WL.DecoderModel(shape, seed=3, filled=500, token=9)
+    for _ in range(3):
+        a.step()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        b.step(s)                                        # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        b.step()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert int(a.pos.item()) == int(b.pos.item()) == 503
+    assert int(a.token.item()) == int(b.token.item())
+    assert torch.equal(a.logits, b.logits)
+    for l in range(2):
+        assert torch.equal(a.k_cache[l].view(torch.int16), b.k_cache[l].view(torch.int16))
+
+
+def test_encoder_layer_and_adapter(env):
+    torch, V, WL = env
+    shape = synth.EncoderShape()
+    em = WL.EncoderModel(shape, seed=0, n_layers=1)
+    em.run()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    D, F, R, nh, hd = shape.dim, shape.ffn, shape.rows, shape.n_heads, shape.head_dim
+    w = synth.encoder_layer_weights(shape, 0, 0)
+    x0 = synth.activations(R, D, 0, synth.ENC_X_ID)
+    qkv_b = bits(em.qkv)
+    # QKV GEMM on bf16(RMSNorm(x0))
+    xn = ref.bf16_to_f64(ref.f32_to_bf16(ref.rmsnorm(x0).astype(np.float32)))
+    err = gemv_err(ref.bf16_to_f64(qkv_b), xn, *w["wqkv"])
+    assert err <= TOL, err
+    # window attention on the GPU's q, k, v and the history
+    kh, vh = synth.encoder_layer_history(shape, 0, 0)
+    Q = ref.bf16_to_f64(qkv_b[:, :D])
+    K = np.concatenate([ref.bf16_to_f64(kh), ref.bf16_to_f64(qkv_b[:, D:2 * D])])
+    Vv = np.concatenate([ref.bf16_to_f64(vh), ref.bf16_to_f64(qkv_b[:, 2 * D:])])
+    rows = list(range(0, R, 15)) + [R - 1]
+    att_ref = np.concatenate([ref.window_attn(Q[i:i + 1], K, Vv, shape.window + i, shape.window, nh, hd)
+                              for i in rows])
+    att = ref.bf16_to_f64(bits(em.att))
+    for ii, i in enumerate(rows):
+        p = shape.window + i
+        lo = p - shape.window + 1
+        for h in range(nh):
+            sl = slice(h * hd, (h + 1) * hd)
+            s = (K[lo:p + 1, sl] @ Q[i, sl]) / math.sqrt(hd)
+            pr = np.exp(s - s.max()); pr /= pr.sum()
+            den = np.linalg.norm(pr) * np.linalg.norm(Vv[lo:p + 1, sl], axis=0)
+            assert np.max(np.abs(att[i, sl] - att_ref[ii, sl]) / den) <= TOL
+    # h = x0 + Wo att and x1 = h + Wdown up, checked through h = x1 - Wdown up
+    up = ref.bf16_to_f64(bits(em.up))
+    x1 = np_of(em.x).astype(np.float64)
+    h_est = x1 - up @ ref.q4_weights(*w["wdown"]).T
+    err_o = gemv_err(h_est - x0, att, *w["wo"])
+    err_dn = ref.gemv_error(x1 - h_est, up @ ref.q4_weights(*w["wdown"]).T, up, ref.q4_weights(*w["wdown"]))
+    assert err_o <= 2 * TOL, err_o
+    assert err_dn <= TOL
+    n2 = ref.bf16_to_f64(ref.f32_to_bf16(ref.rmsnorm(h_est).astype(np.float32)))
+    Wup = ref.q4_weights(*w["wup"])
+    assert ref.gemv_error(up, ref.gelu(n2 @ Wup.T), n2, Wup) <= 2 * TOL
+    # adapter on the downsampled bf16 rows of x1
+    aq, ad = synth.q4_blocks(shape.adapter_out, 4 * D, 0, synth.ADAPTER_ID)
+    xd = ref.downsample_rows(ref.bf16_to_f64(ref.f32_to_bf16(x1.astype(np.float32))), 4)
+    err_ad = gemv_err(np_of(em.out), xd, aq, ad)
+    assert err_ad <= TOL, err_ad
