@@ -6,35 +6,55 @@
 // 4B 음성인식: Voxtral Rust+WASM 구현 해부", section "F32(9GB) vs Q4 GGUF").
 //
 // Design (B200, HBM-bound at M <= 8):
-//  * Work split: "stream-K" at warp granularity over the (16-row tile,
-//    64-column chunk) records of the packed weight: every warp of the grid
-//    owns one contiguous range of records, so every warp streams the same
-//    number of bytes whatever n and k are, and no warp waits for another
-//    while streaming.  Tiles a warp covers completely are finished from its
-//    registers; the few tiles cut at range ends are summed once at the end,
-//    in warp order through shared memory and, for tiles cut between CTAs, in
-//    CTA order through the workspace by whichever CTA arrives last (atomic
-//    count per tile): deterministic, and no CTA ever waits for another.
-//  * Data movement: each lane's share of a record is exactly one 16-byte
-//    load of codes and one 8-byte load of scales, straight into registers,
-//    software-pipelined four records deep.  The first loads are issued before
-//    griddepcontrol.wait, as weights never depend on upstream kernels.
+//  * Work split: every CTA owns a contiguous run of whole 16-row tiles, and
+//    inside it every warp owns one contiguous, equal range of the run's
+//    (tile, 64-column chunk) records ("stream-K" at warp granularity).  A
+//    tile a warp covers completely is finished from its registers; a tile cut
+//    between warps is finished by the warp that started it, which adds the
+//    pieces of the following warps in warp order from shared memory:
+//    deterministic, and no CTA ever waits for another.
+//  * Data movement: each warp streams its range through its own ring of
+//    shared-memory stages, one bulk (TMA) copy of two 576-byte records per
+//    stage, completing on a per-stage mbarrier.  The first stages are issued
+//    before griddepcontrol.wait, as weights never depend on upstream kernels;
+//    bytes in flight cost no registers.
 //  * Dequantisation: each 32-bit word of codes gives four half2 A-fragment
 //    registers with one LOP3 each (OR the nibble into the fraction of 1024.0
 //    or 64.0, whose ulp is 1 at that nibble position: exact 1024+q / 64+q).
-//    The constant offsets are removed through the MMA's C input, which is
-//    preloaded with -(1032 * sum x_lo + 72 * sum x_hi) per block.
-//  * Tensor cores: mma.sync m16n8k16 fp16 x fp16 -> fp32.  The activations
-//    are scaled per row by an exact power of two into fp16 range first, and
-//    the per-block scale d is applied in fp32 after each block's two MMAs.
+//    The constant offsets are removed through the MMAs' C inputs, preloaded
+//    with -1032 * sum x_lo and -72 * sum x_hi per block.
+//  * Tensor cores: mma.sync m16n8k16 fp16 x fp16 -> fp32, the low- and
+//    high-nibble halves of a block as two independent MMAs, and the two
+//    records of a stage issued back to back, so the MMA latency overlaps.
+//  * Activations: each 32-column block of x (times the RMSNorm weight) is
+//    scaled by its own exact power of two into [2^13, 2^14) before the fp16
+//    conversion, and the block's inverse scale is folded into its d in fp32.
+//    No row statistic is needed before the main loop: the RMSNorm factor
+//    multiplies the finished dot products in the epilogue.  The prologue is
+//    one round of loads and one CTA barrier.
 #include "vox_internal.cuh"
+
+#include <stdlib.h>
 
 namespace vox {
 
-constexpr int kGemvWarps = 8;
-constexpr int kGemvThreads = 32 * kGemvWarps;                 // 256
-constexpr int kGemvPrefetch = 4;                              // records in flight per lane
-constexpr int kGemvMaxCtas = 1024;
+#ifndef VOX_GEMV_WARPS
+#define VOX_GEMV_WARPS 8
+#endif
+constexpr int kGemvWarps = VOX_GEMV_WARPS;
+constexpr int kGemvThreads = 32 * kGemvWarps;
+constexpr int kGemvRecs = 4;                                  // records per ring stage
+constexpr int kGemvStageBytes = kGemvRecs * kChunkBytes;      // 2304
+static_assert(kGemvRecs == 4, "the record loop's fast path adds four records");
+constexpr int kGemvMaxStages = 8;
+constexpr int kGemvDefaultStages = 3;
+#ifndef VOX_GEMV_MIN_CTAS
+#define VOX_GEMV_MIN_CTAS 2
+#endif
+#ifndef VOX_GEMV_BATCH
+#define VOX_GEMV_BATCH 9
+#endif
+constexpr int kGemvBatch = VOX_GEMV_BATCH;                    // prologue float4 loads in flight per thread
 
 struct GemvArgs {
     const uint8_t* w;
@@ -42,7 +62,7 @@ struct GemvArgs {
     int32_t tiles, kc;
     const float* x;
     int64_t ldx;
-    int32_t m;
+    int32_t m, vec4;
     float* y;
     int64_t ldy;
     int32_t op, rmsnorm;
@@ -57,69 +77,42 @@ struct GemvArgs {
     const int64_t* pos_dev;
     int32_t* argmax;
     uint8_t* ws;
+    int32_t stages;
 };
 
 // Shared-memory carve-up, computed identically on host and device.
 struct GemvSmem {
-    uint32_t bs, bias, part, part_tile, smul, inv, stats, best_v, best_i, flags, total;
+    uint32_t ring, bars, bs, cb, part, ptile, sq, best_v, best_i, total;
 };
 
-__host__ __device__ inline GemvSmem gemv_smem_layout(int kc, int m)
+__host__ __device__ inline GemvSmem gemv_smem_layout(int kc, int m, int stages)
 {
     GemvSmem L;
     uint32_t off = 0;
-    L.bs = off;        off += (uint32_t)kc * (uint32_t)m * 128u;
-    L.bias = off;      off += ((uint32_t)kc * (uint32_t)m * 8u + 15u) & ~15u;
-    L.part = off;      off += kGemvWarps * 2 * 32 * 4 * 4;
-    L.part_tile = off; off += kGemvWarps * 2 * 8;
-    L.smul = off;      off += 8 * 4;
-    L.inv = off;       off += 8 * 4;
-    L.stats = off;     off += 2 * kGemvWarps * 8 * 4;
-    L.best_v = off;    off += kGemvWarps * 8 * 4;
-    L.best_i = off;    off += kGemvWarps * 8 * 4;
-    L.flags = off;     off += 16;
+    L.ring = off;    off += (uint32_t)kGemvWarps * (uint32_t)stages * kGemvStageBytes;
+    L.bars = off;    off += (uint32_t)kGemvWarps * (uint32_t)stages * 8u;
+    off = (off + 15u) & ~15u;
+    L.bs = off;      off += (uint32_t)kc * (uint32_t)m * 128u;     // fp16 B fragments
+    L.cb = off;      off += (uint32_t)kc * (uint32_t)m * 16u;      // per (token, block): offset constant, 1/scale
+    L.part = off;    off += kGemvWarps * 32 * 16;
+    L.ptile = off;   off += kGemvWarps * 4;
+    L.sq = off;      off += kGemvWarps * 8 * 4;
+    L.best_v = off;  off += kGemvWarps * 8 * 4;
+    L.best_i = off;  off += kGemvWarps * 8 * 4;
     L.total = off;
     return L;
 }
 
-// Workspace: two partial tiles per CTA, the per-CTA argmax candidates with
-// one global arrival counter, then the per-tile arrival counters.  The
-// fixed-size regions come first so that calls on matrices with different tile
-// counts sharing one workspace only ever overlap counter with counter (all
-// counters are back at zero when a call ends).
-struct GemvWs {
-    size_t partials, best_v, best_i, gcount, counters, total;
-};
-
-__host__ __device__ inline GemvWs gemv_ws_layout(int64_t tiles, int with_argmax)
-{
-    (void)with_argmax;
-    GemvWs L;
-    size_t off = 0;
-    L.partials = off;  off += (size_t)kGemvMaxCtas * 2 * 16 * 8 * 4;
-    L.best_v = off;    off += (size_t)kGemvMaxCtas * 8 * 4;
-    L.best_i = off;    off += (size_t)kGemvMaxCtas * 8 * 4;
-    L.gcount = off;    off += 256;
-    L.counters = off;  off += (size_t)tiles * 4;
-    L.total = (off + 255) & ~(size_t)255;
-    return L;
-}
+// Workspace: one 64-bit argmax key per token and the CTA arrival counter of
+// the argmax epilogue.  Both are zero between calls.
+constexpr size_t kGemvWsKeys = 0, kGemvWsCount = 64, kGemvWsBytes = 256;
 
 size_t gemv_workspace_bytes(int64_t n, int64_t k, int op)
 {
+    (void)n;
     (void)k;
-    return gemv_ws_layout(ceil_div(n, 16), op == VOX_EP_ARGMAX).total;
-}
-
-__host__ __device__ __forceinline__ int64_t sk_begin(int64_t b, int64_t total, int64_t G)
-{
-    return b * total / G;
-}
-
-// Owner (CTA or warp) of the contiguous range containing record c.
-__host__ __device__ __forceinline__ int64_t sk_owner(int64_t c, int64_t total, int64_t G)
-{
-    return ((c + 1) * G - 1) / total;
+    (void)op;
+    return kGemvWsBytes;
 }
 
 // "a beats b" for greedy argmax: NaN wins, then larger value, then lower index.
@@ -129,6 +122,35 @@ __device__ __forceinline__ bool argmax_better(float va, int32_t ia, float vb, in
     if (na != nb) return na;
     if (!na && va != vb) return va > vb;
     return ia < ib;
+}
+
+// A 64-bit key whose unsigned order is the argmax order above: NaN above
+// every number, numbers by value (-0 == +0), then the lower index.  0 is
+// below every key, so a zeroed slot is an empty candidate.
+__device__ __forceinline__ unsigned long long argmax_key(float v, int32_t i)
+{
+    uint32_t u = __float_as_uint(v), ku;
+    if (isnan(v)) {
+        ku = 0xFFFFFFFFu;
+    } else {
+        if (u == 0x80000000u) u = 0u;
+        ku = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    }
+    return ((unsigned long long)ku << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)i);
+}
+
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ float4 lds128f(uint32_t addr)
+{
+    float4 v;
+    asm("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
 }
 
 __device__ __forceinline__ float gelu_erf(float v)
@@ -141,65 +163,94 @@ __device__ __forceinline__ float silu_f(float v)
     return v / (1.0f + expf(-v));
 }
 
-// One record's math for one warp: two Q4_0 blocks, each two m16n8k16 MMAs
-// (low / high nibbles) started from the block's offset correction, then
-// scaled by the block's d in fp32.  q, dd: this lane's code and scale words.
+// Four consecutive floats p[4f .. 4f+3]; one 16-byte load when aligned.
+__device__ __forceinline__ float4 ld_f4(const float* p, int f, int vec)
+{
+    if (vec) return *(reinterpret_cast<const float4*>(p) + f);
+    return make_float4(p[4 * f], p[4 * f + 1], p[4 * f + 2], p[4 * f + 3]);
+}
+
+// Issue ring batch j of a warp's range [wb, we): up to kGemvRecs records
+// in one bulk copy, completing on `bar`.
+__device__ __forceinline__ void gemv_issue(const uint8_t* w, int64_t wb, int64_t we, int j, uint8_t* dst,
+                                           uint64_t* bar)
+{
+    const int64_t r0 = wb + (int64_t)j * kGemvRecs;
+    const uint32_t bytes = (uint32_t)min64(kGemvRecs, we - r0) * kChunkBytes;
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_g2s(dst, w + r0 * kChunkBytes, bytes, bar);
+}
+
+// One record's math for one warp: two Q4_0 blocks, each as two chained
+// m16n8k16 MMAs (low / high nibbles) from zero, then corrected by the
+// block's offset constant and scaled by d / (activation scale) in fp32.
+// q, dd: this lane's code and scale words.  p[2h + e] += row g + 8h, token 2t + e.
 template <int MT>
-__device__ __forceinline__ void gemv_record(uint4 q, uint2 dd, uint32_t bs, uint32_t bias, int nblk, int chunk,
-                                            int m, int tok, int t, float (&acc)[4])
+__device__ __forceinline__ void gemv_record(uint4 q, uint2 dd, uint32_t bs, uint32_t cb, int nblk, int chunk,
+                                            int m, int tok, int t, float (&p)[4])
 {
     const uint32_t M_P = 0x000F000Fu, M_Q = 0x00F000F0u, C_P = 0x64006400u, C_Q = 0x54005400u;
     const float2 d0 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
     const float2 d1 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
     const int blk0 = chunk * 2;
-    float2 bias0, bias1;
-    if (MT == 1) {
-        const float2 bb = lds64f(bias + 4u * blk0);
-        bias0 = make_float2(bb.x, 0.f);
-        bias1 = make_float2(bb.y, 0.f);
-    } else {
-        const int t0 = 2 * t, t1 = 2 * t + 1;
-        bias0 = make_float2(t0 < m ? lds32f(bias + 4u * (t0 * nblk + blk0)) : 0.f,
-                            t1 < m ? lds32f(bias + 4u * (t1 * nblk + blk0)) : 0.f);
-        bias1 = make_float2(t0 < m ? lds32f(bias + 4u * (t0 * nblk + blk0 + 1)) : 0.f,
-                            t1 < m ? lds32f(bias + 4u * (t1 * nblk + blk0 + 1)) : 0.f);
-    }
-    const uint32_t bsb = bs + 4u * ((blk0 * (MT == 1 ? 1 : m) + tok) * 16 + t * 4);
+    const int ms = MT == 1 ? 1 : m;
+    const uint32_t bsb = bs + 4u * ((blk0 * ms + tok) * 16 + t * 4);
+    float4 cm = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (MT == 1) cm = lds128f(cb + 8u * blk0);                   // (constant, 1/scale) of both blocks
 #pragma unroll
     for (int bb = 0; bb < 2; ++bb) {
-        const uint4 B = lds128(bsb + 4u * bb * (MT == 1 ? 1 : m) * 16);
-        const float2 bi = bb ? bias1 : bias0;
+        const uint4 B = lds128(bsb + 4u * bb * ms * 16);
+        float2 c0, c1;                                           // tokens 2t, 2t + 1
+        if (MT == 1) {
+            c0 = bb ? make_float2(cm.z, cm.w) : make_float2(cm.x, cm.y);
+            c1 = c0;
+        } else {
+            const int t0 = 2 * t, t1 = 2 * t + 1;
+            c0 = t0 < m ? lds64f(cb + 8u * (t0 * nblk + blk0 + bb)) : make_float2(0.f, 0.f);
+            c1 = t1 < m ? lds64f(cb + 8u * (t1 * nblk + blk0 + bb)) : make_float2(0.f, 0.f);
+        }
         const uint32_t w0 = bb ? q.z : q.x;
         const uint32_t w1 = bb ? q.w : q.y;
         const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
-        float cc[4] = {bi.x, bi.y, bi.x, bi.y};
         const uint32_t alo[4] = {lop3_and_or(w0, M_P, C_P), lop3_and_or(w0s, M_P, C_P),
                                  lop3_and_or(w1, M_P, C_P), lop3_and_or(w1s, M_P, C_P)};
-        mma_f16_16816(cc, alo, B.x, B.y, cc);
         const uint32_t ahi[4] = {lop3_and_or(w0, M_Q, C_Q), lop3_and_or(w0s, M_Q, C_Q),
                                  lop3_and_or(w1, M_Q, C_Q), lop3_and_or(w1s, M_Q, C_Q)};
+        float cc[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_f16_16816(cc, alo, B.x, B.y, cc);
         mma_f16_16816(cc, ahi, B.z, B.w, cc);
         const float dg = bb ? d1.x : d0.x, dg8 = bb ? d1.y : d0.y;
-        acc[0] = fmaf(dg, cc[0], acc[0]);
-        acc[2] = fmaf(dg8, cc[2], acc[2]);
+        p[0] = fmaf(dg * c0.y, cc[0] + c0.x, p[0]);
+        p[2] = fmaf(dg8 * c0.y, cc[2] + c0.x, p[2]);
         if (MT != 1) {
-            acc[1] = fmaf(dg, cc[1], acc[1]);
-            acc[3] = fmaf(dg8, cc[3], acc[3]);
+            p[1] = fmaf(dg * c1.y, cc[1] + c1.x, p[1]);
+            p[3] = fmaf(dg8 * c1.y, cc[3] + c1.x, p[3]);
         }
     }
 }
 
+// Running greedy-argmax candidates of one lane, for its tokens 2t and 2t + 1.
+struct GemvBest {
+    float v0, v1;
+    int32_t i0, i1;
+};
+
 // Epilogue of one finished 16-row tile from the MMA accumulator layout:
-// lane (g, t) holds acc[2h + e] = tile row g + 8h, token 2t + e.
-__device__ __forceinline__ void gemv_epilogue(const GemvArgs& a, int64_t tile, const float (&acc)[4], int g, int t,
-                                              const float* s_inv, int64_t pos, float (&best_v)[2],
-                                              int32_t (&best_i)[2])
+// lane (g, t) holds acc[2h + e] = tile row g + 8h, token 2t + e; rr[e] is the
+// RMSNorm factor of token 2t + e (1 without RMSNorm).  Not inlined: it runs
+// once per tile and keeps the record loop small.
+__device__ __noinline__ GemvBest gemv_epilogue(const GemvArgs& a, int64_t tile, float4 acc4, int g, int t, float r0,
+                                               float r1, int64_t pos, GemvBest best)
 {
+    const float acc[4] = {acc4.x, acc4.y, acc4.z, acc4.w};
+    const float rr[2] = {r0, r1};
+    float best_v[2] = {best.v0, best.v1};
+    int32_t best_i[2] = {best.i0, best.i1};
     float v[4];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) v[2 * h + e] = acc[2 * h + e] * s_inv[(2 * t + e) & 7];
+        for (int e = 0; e < 2; ++e) v[2 * h + e] = acc[2 * h + e] * rr[e];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const int mt = 2 * t + e;
@@ -228,8 +279,8 @@ __device__ __forceinline__ void gemv_epilogue(const GemvArgs& a, int64_t tile, c
                 const int64_t rel = row - a.q_rows;
                 if (rel >= 0 && rel < 2 * kvd) {
                     uint16_t* cache = rel < kvd ? a.kcache : a.vcache;
-                    const int64_t rr = rel < kvd ? rel : rel - kvd;
-                    const int64_t head = rr / a.hd, col = rr - head * a.hd;
+                    const int64_t rw = rel < kvd ? rel : rel - kvd;
+                    const int64_t head = rw / a.hd, col = rw - head * a.hd;
                     const int64_t slot_id = (pos + mt) % a.window;
                     cache[(head * a.window + slot_id) * a.hd + col] = f32_to_bf16_bits(val);
                 }
@@ -264,304 +315,274 @@ __device__ __forceinline__ void gemv_epilogue(const GemvArgs& a, int64_t tile, c
             if (argmax_better(bv, bi, best_v[e], best_i[e])) { best_v[e] = bv; best_i[e] = bi; }
         }
     }
+    return GemvBest{best_v[0], best_v[1], best_i[0], best_i[1]};
+}
+
+// Prologue for activation row i: x * g -> per-block power-of-two scale ->
+// fp16 B fragments and the block's (offset constant, 1/scale), for the float4
+// groups f = f0 + u * threads + lane (f0 warp-uniform, so the 8 float4 of one
+// 32-column block sit in 8 adjacent lanes).  Columns past k (the padding of
+// the last 64-column chunk) become zeros.  sq accumulates sum x^2.
+__device__ __forceinline__ void gemv_convert(const GemvArgs& a, const float* xr, int i, int f0, int nf, int nfp,
+                                             int lane, uint32_t* s_bs32, float2* s_cb, float& sq)
+{
+    const int m = a.m, nblk = a.kc * 2;
+    float4 v[kGemvBatch], gv[kGemvBatch];
+#pragma unroll
+    for (int u = 0; u < kGemvBatch; ++u) {
+        const int f = f0 + u * kGemvThreads + lane;
+        v[u] = f < nf ? ld_f4(xr, f, a.vec4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        gv[u] = (a.g && f < nf) ? ld_f4(a.g, f, a.vec4) : make_float4(1.f, 1.f, 1.f, 1.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kGemvBatch; ++u) {
+        const int fb = f0 + u * kGemvThreads;             // warp-uniform
+        if (fb >= nfp) break;
+        const int f = fb + lane;
+        sq = fmaf(v[u].x, v[u].x, sq);
+        sq = fmaf(v[u].y, v[u].y, sq);
+        sq = fmaf(v[u].z, v[u].z, sq);
+        sq = fmaf(v[u].w, v[u].w, sq);
+        const float4 xg = make_float4(v[u].x * gv[u].x, v[u].y * gv[u].y, v[u].z * gv[u].z, v[u].w * gv[u].w);
+        float am = fmaxf(fmaxf(fabsf(xg.x), fabsf(xg.y)), fmaxf(fabsf(xg.z), fabsf(xg.w)));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));     // max over the 32-column block
+        // am in [2^(E-127), 2^(E-126)): scale 2^(140-E) puts it in [2^13, 2^14)
+        int E = (int)((__float_as_uint(am) >> 23) & 0xFFu);
+        E = E < 14 ? 14 : E;
+        const float sc = __uint_as_float((uint32_t)(267 - E) << 23);
+        const float inv = __uint_as_float((uint32_t)(E - 13) << 23);
+        const __half2 h01 = __floats2half2_rn(xg.x * sc, xg.y * sc);
+        const __half2 h23 = __floats2half2_rn(xg.z * sc, xg.w * sc);
+        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+        float s = (f01.x + f01.y) + (f23.x + f23.y);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);        // sum over one 16-column half-block
+        const float shi = __shfl_down_sync(0xffffffffu, s, 4);
+        if (f < nfp) {
+            // columns 4q .. 4q+3 of block blk: half q>>2, fragment register (q&3)>>1, pair 2(q&1)
+            const int blk = f >> 3, q = f & 7;
+            const int word = (blk * m + i) * 16 + 2 * (q & 1) * 4 + (q >> 2) * 2 + ((q & 3) >> 1);
+            s_bs32[word] = *reinterpret_cast<const uint32_t*>(&h01);
+            s_bs32[word + 4] = *reinterpret_cast<const uint32_t*>(&h23);
+            if (q == 0) s_cb[i * nblk + blk] = make_float2(-(1032.0f * s + 72.0f * shi), inv);
+        }
+    }
 }
 
 template <int MT>
-__global__ void __launch_bounds__(kGemvThreads, 2) q4_gemv_kernel(const GemvArgs a)
+__global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kernel(const __grid_constant__ GemvArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int m = a.m;
-    const int kc = a.kc;
-    const GemvSmem L = gemv_smem_layout(kc, m);
-    volatile int32_t* s_flag = reinterpret_cast<volatile int32_t*>(smem + L.flags);
-    float* s_smul = reinterpret_cast<float*>(smem + L.smul);
-    float* s_inv = reinterpret_cast<float*>(smem + L.inv);
-    float* s_stats = reinterpret_cast<float*>(smem + L.stats);
-    float* s_bias = reinterpret_cast<float*>(smem + L.bias);
-    uint16_t* s_bs16 = reinterpret_cast<uint16_t*>(smem + L.bs);
+    const int m = a.m, kc = a.kc, stages = a.stages;
+    const GemvSmem L = gemv_smem_layout(kc, m, stages);
+    uint32_t* s_bs32 = reinterpret_cast<uint32_t*>(smem + L.bs);
+    float2* s_cb = reinterpret_cast<float2*>(smem + L.cb);
     float* s_part = reinterpret_cast<float*>(smem + L.part);
-    int64_t* s_part_tile = reinterpret_cast<int64_t*>(smem + L.part_tile);
+    int32_t* s_ptile = reinterpret_cast<int32_t*>(smem + L.ptile);
+    float* s_sq = reinterpret_cast<float*>(smem + L.sq);
     float* s_best_v = reinterpret_cast<float*>(smem + L.best_v);
     int32_t* s_best_i = reinterpret_cast<int32_t*>(smem + L.best_i);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int64_t G = gridDim.x, b = blockIdx.x;
-    const int64_t GW = G * kGemvWarps, gw = b * kGemvWarps + warp;
-    const int64_t total = (int64_t)a.tiles * kc;
-    const int64_t cb = sk_begin(b, total, G), ce = sk_begin(b + 1, total, G);            // CTA range
-    const int64_t wb = sk_begin(gw, total, GW), we = sk_begin(gw + 1, total, GW);        // warp range
+    const int64_t tile_b = b * a.tiles / G, tile_e = (b + 1) * a.tiles / G;
+    const int64_t rb = tile_b * kc, R = (tile_e - tile_b) * kc;                   // this CTA's records
+    const int64_t wb = rb + R * warp / kGemvWarps, we = rb + R * (warp + 1) / kGemvWarps;
+    const int nbatch = (int)((we - wb + kGemvRecs - 1) / kGemvRecs);
 
-    // first records of this warp, issued before the upstream kernels finish
-    const uint8_t* wsrc = a.w + 16 * lane;
-    const uint8_t* dsrc = a.w + kChunkQsBytes + 8 * g;
-    uint4 rq[kGemvPrefetch];
-    uint2 rd[kGemvPrefetch];
-#pragma unroll
-    for (int u = 0; u < kGemvPrefetch; ++u) {
-        if (wb + u < we) {
-            rq[u] = __ldg(reinterpret_cast<const uint4*>(wsrc + (wb + u) * kChunkBytes));
-            rd[u] = __ldg(reinterpret_cast<const uint2*>(dsrc + (wb + u) * kChunkBytes));
-        } else {
-            rq[u] = make_uint4(0u, 0u, 0u, 0u);
-            rd[u] = make_uint2(0u, 0u);
-        }
+    // this warp's ring; the first stages are in flight before the upstream kernels finish
+    uint8_t* ring = smem + L.ring + (uint32_t)warp * (uint32_t)stages * kGemvStageBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + warp * stages;
+    if (lane == 0) {
+        for (int s = 0; s < stages; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        for (int j = 0; j < stages && j < nbatch; ++j)
+            gemv_issue(a.w, wb, we, j, ring + j * kGemvStageBytes, &bars[j]);
+        s_ptile[warp] = -1;
     }
 
     pdl_wait();                              // x (and pos) come from upstream kernels
     pdl_launch_dependents();                 // only after our own wait: at most two kernels overlap
 
-    // ---- prologue: per-row statistics -> RMSNorm factor and fp16 scaling
-    const int64_t K = a.k;
+    // ---- prologue: fp16 B fragments and block corrections of every row; sum x^2 per row
+    const int nf = (int)(a.k >> 2), nfp = kc * 16;
     for (int i = 0; i < m; ++i) {
         const float* xr = a.x + (int64_t)i * a.ldx;
-        float ssq[4] = {0.f, 0.f, 0.f, 0.f}, amx[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int64_t kk = tid; kk < K; kk += 4 * kGemvThreads) {
-            float v[4], gg[4];
+        float sq = 0.f;
+        for (int f0 = warp * 32; f0 < nfp; f0 += kGemvBatch * kGemvThreads)
+            gemv_convert(a, xr, i, f0, nf, nfp, lane, s_bs32, s_cb, sq);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int64_t k = kk + (int64_t)u * kGemvThreads;
-                v[u] = k < K ? xr[k] : 0.f;
-                gg[u] = (a.g && k < K) ? a.g[k] : 1.f;
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                ssq[u] = fmaf(v[u], v[u], ssq[u]);
-                amx[u] = fmaxf(amx[u], fabsf(v[u] * gg[u]));
-            }
-        }
-        float sq = (ssq[0] + ssq[1]) + (ssq[2] + ssq[3]);
-        float am = fmaxf(fmaxf(amx[0], amx[1]), fmaxf(amx[2], amx[3]));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            sq += __shfl_xor_sync(0xffffffffu, sq, o);
-            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-        }
-        if (lane == 0) {
-            s_stats[warp * 8 + i] = sq;
-            s_stats[kGemvWarps * 8 + warp * 8 + i] = am;
-        }
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (lane == 0) s_sq[warp * 8 + i] = sq;
     }
-    __syncthreads();
-    if (tid < m) {
-        float ssq = 0.f, amx = 0.f;
-        for (int w = 0; w < kGemvWarps; ++w) {
-            ssq += s_stats[w * 8 + tid];
-            amx = fmaxf(amx, s_stats[kGemvWarps * 8 + w * 8 + tid]);
-        }
-        const float r = a.rmsnorm ? 1.0f / sqrtf(ssq / (float)K + a.eps) : 1.0f;
-        const float an = amx * r;
-        int e = 0;
-        float sc = 1.0f;
-        if (an > 0.f && isfinite(an)) {
-            frexpf(an, &e);                  // an < 2^e
-            sc = ldexpf(1.0f, 14 - e);       // an * sc < 2^14
-        }
-        s_smul[tid] = r * sc;
-        s_inv[tid] = 1.0f / sc;              // exact power of two
-    }
-    if (tid >= m && tid < 8) s_inv[tid] = 0.f;
     __syncthreads();
 
-    // ---- prologue: activations -> fp16 B fragments + per-block offsets; one
-    // warp per (row, block), lane e converts element e, eight loads in flight
-    const int nblk = kc * 2;
-    {
-        const int e = lane, half = e >> 4, ep = e & 15, rr = ep >> 3, tt = (ep & 7) >> 1, elem = ep & 1;
-        const int items = m * nblk;
-        for (int base = warp; base < items; base += 8 * kGemvWarps) {
-            float v[8];
+    // RMSNorm factors of this lane's tokens 2t, 2t+1 (zero for tokens past m)
+    float rr[2];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int it = base + u * kGemvWarps;
-                v[u] = 0.f;
-                if (it < items) {
-                    const int i = it / nblk, blk = it - i * nblk;
-                    const int64_t k0 = (int64_t)blk * 32 + e;
-                    if (k0 < K) {
-                        const float xv = a.x[(int64_t)i * a.ldx + k0];
-                        v[u] = a.g ? xv * a.g[k0] : xv;
-                    }
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int it = base + u * kGemvWarps;
-                if (it >= items) break;
-                const int i = it / nblk, blk = it - i * nblk;
-                const __half h = __float2half_rn(v[u] * s_smul[i]);
-                float hf = __half2float(h);
-                s_bs16[((blk * m + i) * 16 + tt * 4 + half * 2 + rr) * 2 + elem] = __half_as_ushort(h);
-#pragma unroll
-                for (int o = 8; o > 0; o >>= 1) hf += __shfl_xor_sync(0xffffffffu, hf, o);   // per 16-lane half
-                const float shi = __shfl_sync(0xffffffffu, hf, 16);
-                if (lane == 0) s_bias[i * nblk + blk] = -(1032.0f * hf + 72.0f * shi);
+    for (int e = 0; e < 2; ++e) {
+        const int tk = MT == 1 ? e : 2 * t + e;
+        float r = 0.f;
+        if (tk < m) {
+            r = 1.0f;
+            if (a.rmsnorm) {
+                float ssq = 0.f;
+                for (int w = 0; w < kGemvWarps; ++w) ssq += s_sq[w * 8 + tk];
+                r = 1.0f / sqrtf(ssq / (float)a.k + a.eps);
             }
         }
+        rr[e] = r;
     }
-    __syncthreads();
+    if (MT == 1 && t != 0) rr[0] = 0.f;      // token 2t of a lane with t > 0 does not exist at m = 1
 
     const int64_t pos = a.pos_dev ? *a.pos_dev : a.pos;
+    const int nblk = kc * 2;
     const uint32_t tk = smem_token();
-    const uint32_t bs_a = smem_addr(s_bs16) + tk, bias_a = smem_addr(s_bias) + tk;
+    const uint32_t bs_a = smem_addr(s_bs32) + tk, cb_a = smem_addr(s_cb) + tk;
+    const uint32_t ring_a = smem_addr(ring);
     const int tok = g < m ? g : 0;
-    float best_v[2] = {-INFINITY, -INFINITY};
-    int32_t best_i[2] = {0x7fffffff, 0x7fffffff};
+    GemvBest best = {-INFINITY, -INFINITY, 0x7fffffff, 0x7fffffff};
 
-    // ---- main loop: this warp's records, four in flight
-    int n_part = 0;
-    s_part_tile[warp * 2 + 0] = -1;
-    s_part_tile[warp * 2 + 1] = -1;
-    if (wb < we) {
+    // ---- main loop: this warp's records through its ring
+    float tacc[4] = {0.f, 0.f, 0.f, 0.f};    // piece of the tile this warp started and did not finish
+    int64_t tail_tile = -1;
+    if (nbatch > 0) {
         int64_t tile = wb / kc;
         int cin = (int)(wb - tile * kc);
-        bool tile_whole = (cin == 0);        // this warp saw the tile from its first record
+        bool whole = (cin == 0);             // this warp saw the tile from its first record
+        int left = (int)(we - wb);           // records still to add
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int64_t base = wb; base < we; base += kGemvPrefetch) {
-#pragma unroll
-            for (int u = 0; u < kGemvPrefetch; ++u) {
-                const int64_t i = base + u;
-                if (i >= we) break;
-                const uint4 q = rq[u];
-                const uint2 dd = rd[u];
-                const int64_t nx = i + kGemvPrefetch;
-                if (nx < we) {
-                    rq[u] = __ldg(reinterpret_cast<const uint4*>(wsrc + nx * kChunkBytes));
-                    rd[u] = __ldg(reinterpret_cast<const uint2*>(dsrc + nx * kChunkBytes));
-                }
-                gemv_record<MT>(q, dd, bs_a, bias_a, nblk, cin, m, tok, t, acc);
-                if (++cin == kc || i + 1 == we) {
-                    if (cin == kc && tile_whole) {
-                        gemv_epilogue(a, tile, acc, g, t, s_inv, pos, best_v, best_i);
-                    } else {
-                        // a tile cut at this warp's range end: keep the partial sums
-                        *reinterpret_cast<float4*>(s_part + ((warp * 2 + n_part) * 32 + lane) * 4) =
-                            make_float4(acc[0], acc[1], acc[2], acc[3]);
-                        if (lane == 0) s_part_tile[warp * 2 + n_part] = tile;
-                        ++n_part;
-                    }
-                    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-                    cin = 0;
-                    ++tile;
-                    tile_whole = true;
-                }
-            }
-        }
-    }
-    __syncthreads();
-
-    // ---- tiles cut between warps: warp 0 sums the parts in warp order
-    const GemvWs W = gemv_ws_layout(a.tiles, a.op == VOX_EP_ARGMAX);
-    if (warp == 0) {
-        float* parts = reinterpret_cast<float*>(a.ws + W.partials);
-        int32_t* counters = reinterpret_cast<int32_t*>(a.ws + W.counters);
-        int64_t cur = -1;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int e = 0; e <= 2 * kGemvWarps; ++e) {
-            const int64_t tl = e < 2 * kGemvWarps ? s_part_tile[e] : -2;
-            if (tl == -1) continue;
-            if (tl != cur && cur >= 0) {
-                // flush tile `cur`: finish here, or combine with the neighbouring CTAs
-                const int64_t b_first = sk_owner(cur * kc, total, G);
-                const int64_t b_last = sk_owner(cur * kc + kc - 1, total, G);
-                bool finish = true;
-                if (b_first != b_last) {
-                    const int my_slot = (cur == cb / kc) ? 0 : 1;
-                    *reinterpret_cast<float4*>(parts + (((size_t)b * 2 + my_slot) * 32 + lane) * 4) =
+        uint32_t phase = 0;
+        int s = 0, fail_j = -1;
+        // add one record's contribution; close the tile at its end or at the range end
+        auto step = [&](const float (&p)[4]) {
+            acc[0] += p[0]; acc[2] += p[2];
+            if (MT != 1) { acc[1] += p[1]; acc[3] += p[3]; }
+            --left;
+            if (++cin == kc || left == 0) {
+                if (!whole) {
+                    // started by an earlier warp: leave the piece for it
+                    *reinterpret_cast<float4*>(s_part + (warp * 32 + lane) * 4) =
                         make_float4(acc[0], acc[1], acc[2], acc[3]);
-                    __syncwarp();
-                    int32_t last = 0;
-                    if (lane == 0) {
-                        __threadfence();
-                        const int32_t old = atomicAdd(&counters[cur], 1);
-                        last = (old == (int32_t)(b_last - b_first)) ? 1 : 0;
-                        if (last) {
-                            __threadfence();
-                            counters[cur] = 0;
-                        }
-                    }
-                    finish = __shfl_sync(0xffffffffu, last, 0) != 0;
-                    if (finish) {
-                        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-                        for (int64_t bo = b_first; bo <= b_last; ++bo) {
-                            const int sl = (cur == sk_begin(bo, total, G) / kc) ? 0 : 1;
-                            const float4 pv = __ldcg(reinterpret_cast<const float4*>(
-                                parts + (((size_t)bo * 2 + sl) * 32 + lane) * 4));
-                            acc[0] += pv.x; acc[1] += pv.y; acc[2] += pv.z; acc[3] += pv.w;
-                        }
-                    }
+                    if (lane == 0) s_ptile[warp] = (int32_t)tile;
+                } else if (cin == kc) {
+                    best = gemv_epilogue(a, tile, make_float4(acc[0], acc[1], acc[2], acc[3]), g, t, rr[0], rr[1],
+                                         pos, best);
+                } else {
+                    tacc[0] = acc[0]; tacc[1] = acc[1]; tacc[2] = acc[2]; tacc[3] = acc[3];
+                    tail_tile = tile;
                 }
-                if (finish) gemv_epilogue(a, cur, acc, g, t, s_inv, pos, best_v, best_i);
                 acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+                cin = 0;
+                ++tile;
+                whole = true;
             }
-            if (tl < 0) break;
-            cur = tl;
-            const float4 pv = *reinterpret_cast<const float4*>(s_part + (e * 32 + lane) * 4);
-            acc[0] += pv.x; acc[1] += pv.y; acc[2] += pv.z; acc[3] += pv.w;
+        };
+        for (int j = 0; j < nbatch; ++j) {
+            if (!mbar_wait_bounded(&bars[s], (phase >> s) & 1u, 0x101)) {
+                fail_j = j;
+                break;
+            }
+            phase ^= 1u << s;
+            const uint32_t base = ring_a + (uint32_t)s * kGemvStageBytes + smem_token();
+            // every record's MMAs first; the slots past `left` of a short stage are read and discarded
+            float p[kGemvRecs][4];
+            int ch = cin;
+#pragma unroll
+            for (int r = 0; r < kGemvRecs; ++r) {
+                const uint4 q = lds128(base + r * kChunkBytes + 16 * lane);
+                const uint2 e = lds64(base + r * kChunkBytes + kChunkQsBytes + 8 * g);
+                p[r][0] = p[r][1] = p[r][2] = p[r][3] = 0.f;
+                gemv_record<MT>(q, e, bs_a, cb_a, nblk, ch, m, tok, t, p[r]);
+                ch = ch + 1 == kc ? 0 : ch + 1;
+            }
+            if (left > kGemvRecs && cin + kGemvRecs < kc) {
+                // no tile end and no range end inside this stage
+                acc[0] += (p[0][0] + p[1][0]) + (p[2][0] + p[3][0]);
+                acc[2] += (p[0][2] + p[1][2]) + (p[2][2] + p[3][2]);
+                if (MT != 1) {
+                    acc[1] += (p[0][1] + p[1][1]) + (p[2][1] + p[3][1]);
+                    acc[3] += (p[0][3] + p[1][3]) + (p[2][3] + p[3][3]);
+                }
+                cin += kGemvRecs;
+                left -= kGemvRecs;
+            } else {
+#pragma unroll
+                for (int r = 0; r < kGemvRecs; ++r)
+                    if (left > 0) step(p[r]);
+            }
+            __syncwarp();
+            if (lane == 0 && j + stages < nbatch)
+                gemv_issue(a.w, wb, we, j + stages, ring + s * kGemvStageBytes, &bars[s]);
+            if (++s == stages) s = 0;
+        }
+        if (fail_j >= 0 && lane == 0) {
+            // a stage never completed: wait (bounded) for the copies still in flight into this ring
+            const int jend = fail_j + stages < nbatch ? fail_j + stages : nbatch;
+            for (int j = fail_j; j < jend; ++j)
+                mbar_wait_bounded(&bars[j % stages], (uint32_t)(j / stages) & 1u, 0x102);
         }
     }
 
-    // ---- greedy argmax: warps -> CTA -> the last CTA to arrive
+    // ---- tiles cut between warps: the warp that started one adds the later pieces in warp order
+    __syncthreads();
+    if (tail_tile >= 0) {
+        const int64_t last_rec = tail_tile * kc + kc - 1;
+        const int wl = (int)(((last_rec - rb + 1) * kGemvWarps - 1) / R);   // warp holding the tile's last record
+        const uint32_t tk2 = smem_token();
+        for (int w2 = warp + 1; w2 <= wl; ++w2) {
+            if (__float_as_int(lds32f(smem_addr(s_ptile) + 4u * w2 + tk2)) != (int32_t)tail_tile) continue;
+            const float4 pv = lds128f(smem_addr(s_part) + (uint32_t)(w2 * 32 + lane) * 16u + tk2);
+            tacc[0] += pv.x; tacc[1] += pv.y; tacc[2] += pv.z; tacc[3] += pv.w;
+        }
+        best = gemv_epilogue(a, tail_tile, make_float4(tacc[0], tacc[1], tacc[2], tacc[3]), g, t, rr[0], rr[1], pos,
+                             best);
+    }
+
+    // ---- greedy argmax: warps -> CTA -> one 64-bit atomic max per token; the
+    // last CTA to arrive turns the keys into indices and clears them
     if (a.op == VOX_EP_ARGMAX) {
         if (g == 0) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                s_best_v[warp * 8 + 2 * t + e] = best_v[e];
-                s_best_i[warp * 8 + 2 * t + e] = best_i[e];
-            }
+            s_best_v[warp * 8 + 2 * t] = best.v0;
+            s_best_v[warp * 8 + 2 * t + 1] = best.v1;
+            s_best_i[warp * 8 + 2 * t] = best.i0;
+            s_best_i[warp * 8 + 2 * t + 1] = best.i1;
         }
         __syncthreads();
-        if (warp == 0) {
-            float* bvs = reinterpret_cast<float*>(a.ws + W.best_v);
-            int32_t* bis = reinterpret_cast<int32_t*>(a.ws + W.best_i);
-            int32_t* gcount = reinterpret_cast<int32_t*>(a.ws + W.gcount);
-            if (lane < m) {
+        if (tid == 0) {
+            unsigned long long* keys = reinterpret_cast<unsigned long long*>(a.ws + kGemvWsKeys);
+            uint32_t* count = reinterpret_cast<uint32_t*>(a.ws + kGemvWsCount);
+            for (int i = 0; i < m; ++i) {
                 float bv = -INFINITY;
                 int32_t bi = 0x7fffffff;
                 for (int w = 0; w < kGemvWarps; ++w)
-                    if (argmax_better(s_best_v[w * 8 + lane], s_best_i[w * 8 + lane], bv, bi)) {
-                        bv = s_best_v[w * 8 + lane];
-                        bi = s_best_i[w * 8 + lane];
+                    if (argmax_better(s_best_v[w * 8 + i], s_best_i[w * 8 + i], bv, bi)) {
+                        bv = s_best_v[w * 8 + i];
+                        bi = s_best_i[w * 8 + i];
                     }
-                bvs[b * 8 + lane] = bv;
-                bis[b * 8 + lane] = bi;
+                atomicMax(&keys[i], argmax_key(bv, bi));
             }
-            __syncwarp();
-            int32_t last = 0;
-            if (lane == 0) {
-                __threadfence();
-                const int32_t old = atomicAdd(gcount, 1);
-                last = (old == (int32_t)(G - 1)) ? 1 : 0;
-                if (last) {
-                    __threadfence();
-                    *gcount = 0;
+            if (atom_add_acq_rel_gpu(count, 1u) == gridDim.x - 1) {
+                for (int i = 0; i < m; ++i) {
+                    const unsigned long long key = atomicExch(&keys[i], 0ull);
+                    a.argmax[i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
                 }
-            }
-            last = __shfl_sync(0xffffffffu, last, 0);
-            if (last && lane < m) {
-                float bv = -INFINITY;
-                int32_t bi = 0x7fffffff;
-                for (int64_t bo = 0; bo < G; ++bo) {
-                    const float v = __ldcg(bvs + bo * 8 + lane);
-                    const int32_t ix = __ldcg(bis + bo * 8 + lane);
-                    if (argmax_better(v, ix, bv, bi)) { bv = v; bi = ix; }
-                }
-                a.argmax[lane] = bi;
+                *count = 0u;
             }
         }
     }
-    (void)s_flag;
 }
 
-static int gemv_ctas_per_sm()
+static int env_int(const char* name, int dflt, int lo, int hi)
 {
-    static int v = -1;
-    if (v < 0) {
-        const char* e = getenv("VOX_GEMV_CTAS_PER_SM");
-        v = e ? atoi(e) : 2;
-        if (v < 1) v = 1;
-        if (v > 4) v = 4;
-    }
+    const char* e = getenv(name);
+    int v = e ? atoi(e) : dflt;
+    if (v < lo) v = lo;
+    if (v > hi) v = hi;
     return v;
 }
 
@@ -597,9 +618,16 @@ vox_status launch_q4_gemv(const uint8_t* w, int64_t n, int64_t k, const float* x
     }
     a.argmax = ep ? ep->argmax : nullptr;
     a.ws = static_cast<uint8_t*>(ws);
+    a.vec4 = ((reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (ldx & 3) == 0 &&
+              (!a.g || (reinterpret_cast<uintptr_t>(a.g) & 15u) == 0)) ? 1 : 0;
 
-    const GemvSmem L = gemv_smem_layout(a.kc, a.m);
-    if (L.total > 227 * 1024) return VOX_ERR_SHAPE;           // activations do not fit shared memory
+    int stages = env_int("VOX_GEMV_STAGES", kGemvDefaultStages, 2, kGemvMaxStages);
+    GemvSmem L = gemv_smem_layout(a.kc, a.m, stages);
+    while (stages > 2 && L.total > 227 * 1024) L = gemv_smem_layout(a.kc, a.m, --stages);
+    if (L.total > 227 * 1024) return VOX_ERR_SHAPE;            // activations do not fit shared memory
+    a.stages = stages;
+
+    void (*kern)(GemvArgs) = m == 1 ? q4_gemv_kernel<1> : q4_gemv_kernel<8>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(q4_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
@@ -611,13 +639,17 @@ vox_status launch_q4_gemv(const uint8_t* w, int64_t n, int64_t k, const float* x
         }
         attr_set = true;
     }
-    const int64_t total = (int64_t)a.tiles * a.kc;
-    int64_t G = (int64_t)device_sm_count() * gemv_ctas_per_sm();
-    if (L.total > 110 * 1024) G = device_sm_count();       // two such CTAs do not fit one SM
-    if (G > total) G = total;
-    if (G > kGemvMaxCtas) G = kGemvMaxCtas;
-    if (m == 1) return launch_pdl(q4_gemv_kernel<1>, dim3((unsigned)G), dim3(kGemvThreads), L.total, s, a);
-    return launch_pdl(q4_gemv_kernel<8>, dim3((unsigned)G), dim3(kGemvThreads), L.total, s, a);
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemvThreads, L.total);
+    if (e != cudaSuccess || per_sm < 1) {
+        set_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
+        return VOX_ERR_CUDA;
+    }
+    const int cap = env_int("VOX_GEMV_CTAS_PER_SM", 2, 1, 4);
+    if (per_sm > cap) per_sm = cap;
+    int64_t G = (int64_t)device_sm_count() * per_sm;
+    if (G > a.tiles) G = a.tiles;
+    return launch_pdl(kern, dim3((unsigned)G), dim3(kGemvThreads), L.total, s, a);
 }
 
 }  // namespace vox
