@@ -18,13 +18,17 @@
 // q' and P are split into bf16 hi + lo parts (two MMAs each), so the
 // tensor-core inputs carry about 16 significant bits; K and V are the cache's
 // own bf16 values.  Each CTA writes one (m, l, O) partial per kv head it
-// touched; K5 merges them per query head in CTA order (deterministic).
+// touched, into that head's contiguous run of records; K5 merges each head's
+// run in CTA order (deterministic), one small CTA per query head, all of a
+// head's records loaded in one round before the arithmetic.
 //
 // Programmatic dependent launch: the producer starts streaming before the
 // upstream kernel (the QKV projection that appends this step's k, v) has
 // finished; after griddepcontrol.wait the warp whose slots include the newly
 // written one reloads that row from global memory.
 #include "tma.cuh"
+
+#include <stdlib.h>
 
 namespace vox {
 
@@ -67,10 +71,11 @@ constexpr int kAttnChunk = 64;                 // slots per chunk
 constexpr int kAttnHd = 128;
 constexpr int kAttnWarps = 4;                  // consumer warps, 16 slots each
 constexpr int kAttnThreads = 32 * (1 + kAttnWarps);
-constexpr int kAttnStages = 2;
+constexpr int kAttnMaxStages = 6;
 constexpr int kAttnTileBytes = kAttnChunk * 128;            // one 64 x 64 bf16 box
 constexpr int kAttnStageBytes = 4 * kAttnTileBytes;         // K lo/hi, V lo/hi
 constexpr int kAttnMaxCtas = 592;
+constexpr int kCombineBatch = 20;                  // records of a head loaded per round in K5
 constexpr int kAttnMaxGroup = 8;
 
 struct AttnArgs {
@@ -82,41 +87,61 @@ struct AttnArgs {
     int64_t pos;
     const int64_t* pos_dev;
     float qscale;                              // scale * log2(e)
-    float* ws;
+    float* ws;                                 // partial records
+    int32_t stages;
+    int32_t rec_floats;                        // record stride (floats, a multiple of 4)
+    int32_t rmax;                              // record slots per kv head
 };
 
-// Partial record of (CTA, slot): O[8][hd] then (m, l)[8].
-__host__ __device__ inline size_t attn_rec_floats(int hd) { return (size_t)kAttnMaxGroup * (hd + 2); }
+// Partial record of one CTA for one kv head: O[group][hd], then (m, l) per
+// query head of the group, padded to 16 bytes.  The records of kv head kh
+// are contiguous: slot kh * rmax + (CTA - first CTA of kh).
+__host__ __device__ inline int attn_rec_floats(int group, int hd) { return (group * (hd + 2) + 3) & ~3; }
+__host__ __device__ inline int attn_rmax(int n_kv) { return (kAttnMaxCtas + n_kv - 1) / n_kv + 2; }
+
+static int env_int_attn(const char* name, int dflt, int lo, int hi)
+{
+    const char* e = getenv(name);
+    int v = e ? atoi(e) : dflt;
+    return v < lo ? lo : (v > hi ? hi : v);
+}
 
 static int64_t attn_grid(int n_kv, int window)
 {
     int64_t chunks = (int64_t)n_kv * ceil_div(window, kAttnChunk);
-    int64_t G = 2 * (int64_t)device_sm_count();    // two 82 KB CTAs per SM
+    int64_t G = (int64_t)env_int_attn("VOX_ATTN_CTAS_PER_SM", 1, 1, 2) * device_sm_count();
     if (G > chunks) G = chunks;
     if (G < n_kv) G = n_kv;                    // then no CTA spans more than two kv heads
     if (G > kAttnMaxCtas) G = kAttnMaxCtas;
     return G;
 }
 
+// Workspace: rmax partial records per kv head (room for the largest group).
 size_t attn_workspace_bytes(int n_kv, int hd, int window)
 {
-    int64_t chunks = (int64_t)n_kv * ceil_div(window, kAttnChunk);
-    int64_t G = chunks > kAttnMaxCtas ? kAttnMaxCtas : chunks;
-    if (G < n_kv) G = n_kv;
-    return (size_t)G * 2 * attn_rec_floats(hd) * sizeof(float);
+    (void)window;
+    return ((size_t)n_kv * attn_rmax(n_kv) * attn_rec_floats(kAttnMaxGroup, hd) * sizeof(float) + 255) &
+           ~(size_t)255;
 }
 
 __host__ __device__ inline int64_t attn_begin(int64_t b, int64_t total, int64_t G) { return b * total / G; }
 __host__ __device__ inline int64_t attn_owner(int64_t c, int64_t total, int64_t G) { return ((c + 1) * G - 1) / total; }
 
+// Shared-memory carve-up for `stages` ring stages (host and device).
 struct AttnSmem {
-    static constexpr uint32_t ring = 0;
-    static constexpr uint32_t merge = kAttnStages * kAttnStageBytes;                  // 64 KB
-    static constexpr uint32_t merge_bytes = kAttnWarps * kAttnMaxGroup * (kAttnHd + 2) * 4;
-    static constexpr uint32_t bars = merge + merge_bytes;
-    static constexpr uint32_t flags = bars + 2 * kAttnStages * 8;
-    static constexpr uint32_t total = flags + 16 + 1024;                               // + alignment slack
+    uint32_t ring, merge, bars, flags, total;
 };
+
+__host__ __device__ inline AttnSmem attn_smem_layout(int stages)
+{
+    AttnSmem L;
+    L.ring = 0;
+    L.merge = (uint32_t)stages * kAttnStageBytes;
+    L.bars = L.merge + kAttnWarps * kAttnMaxGroup * (kAttnHd + 2) * 4;
+    L.flags = L.bars + 2u * (uint32_t)stages * 8u;
+    L.total = L.flags + 16 + 1024;             // + alignment slack
+    return L;
+}
 
 __global__ void __launch_bounds__(kAttnThreads, 2)
 gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
@@ -125,16 +150,18 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     extern __shared__ uint8_t smem_raw[];
     // TMA 128-byte-swizzled tiles need a 1024-byte aligned destination.
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + AttnSmem::bars);
-    uint64_t* empty = full + kAttnStages;
-    volatile int32_t* s_fail = reinterpret_cast<volatile int32_t*>(smem + AttnSmem::flags);
+    const int stages = a.stages;
+    const AttnSmem SL = attn_smem_layout(stages);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + SL.bars);
+    uint64_t* empty = full + stages;
+    volatile int32_t* s_fail = reinterpret_cast<volatile int32_t*>(smem + SL.flags);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t G = gridDim.x, b = blockIdx.x;
     const int W = a.window;
 
     if (tid == 0) {
-        for (int s = 0; s < kAttnStages; ++s) {
+        for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kAttnWarps);
         }
@@ -165,14 +192,14 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
                 if (!s_fail[0] && !mbar_wait_bounded(&empty[slot], ph ^ 1u, 0x201)) s_fail[0] = 1;
                 if (s_fail[0]) break;
                 const int32_t row = (int32_t)(kh * W + ci * kAttnChunk);
-                uint8_t* st = smem + AttnSmem::ring + slot * kAttnStageBytes;
+                uint8_t* st = smem + SL.ring + slot * kAttnStageBytes;
                 mbar_arrive_expect_tx(&full[slot], kAttnStageBytes);
                 tma_load_2d(st + 0 * kAttnTileBytes, &kmap, 0, row, &full[slot]);
                 tma_load_2d(st + 1 * kAttnTileBytes, &kmap, 64, row, &full[slot]);
                 tma_load_2d(st + 2 * kAttnTileBytes, &vmap, 0, row, &full[slot]);
                 tma_load_2d(st + 3 * kAttnTileBytes, &vmap, 64, row, &full[slot]);
                 if (++ci == nch) { ci = 0; ++kh; }
-                if (++slot == kAttnStages) { slot = 0; ph ^= 1u; }
+                if (++slot == stages) { slot = 0; ph ^= 1u; }
             }
         }
         return;
@@ -185,8 +212,8 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     pdl_launch_dependents();
     const int64_t new_slot = pos % W;
 
-    float* merge = reinterpret_cast<float*>(smem + AttnSmem::merge);
-    const uint32_t ring_a = smem_addr(smem + AttnSmem::ring);
+    float* merge = reinterpret_cast<float*>(smem + SL.merge);
+    const uint32_t ring_a = smem_addr(smem + SL.ring);
 
     // running softmax state of heads 2t, 2t+1 (replicated over g) and O^T
     // fragments: o[J] = (dim 16J+g | 16J+8+g) x (head 2t | 2t+1)
@@ -198,7 +225,7 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     int64_t seg_head = -1;
     int seg_idx = 0;
 
-    auto flush = [&](int sidx) {
+    auto flush = [&](int sidx, int64_t kh_seg) {
         // merge the four warps' (m, l, O) for the finished kv head, write the partial
         float* mw = merge + warp * kAttnMaxGroup * (kAttnHd + 2);
         if (g == 0) {
@@ -216,7 +243,9 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
             mw[(2 * t + 1) * kAttnHd + 16 * j + 8 + g] = o[j][3];
         }
         named_barrier(1, 32 * kAttnWarps);
-        float* rec = a.ws + ((size_t)b * 2 + sidx) * attn_rec_floats(kAttnHd);
+        (void)sidx;
+        const int64_t bf_seg = attn_owner(kh_seg * nch, total, G);
+        float* rec = a.ws + ((size_t)kh_seg * a.rmax + (size_t)(b - bf_seg)) * a.rec_floats;
         for (int i = tid; i < group * kAttnHd; i += 32 * kAttnWarps) {
             const int hh = i / kAttnHd, cc = i % kAttnHd;
             float M = -INFINITY;
@@ -232,8 +261,8 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
             }
             rec[hh * kAttnHd + cc] = O;
             if (cc == 0) {
-                rec[kAttnMaxGroup * kAttnHd + hh * 2 + 0] = M;
-                rec[kAttnMaxGroup * kAttnHd + hh * 2 + 1] = Lsum;
+                rec[group * kAttnHd + hh * 2 + 0] = M;
+                rec[group * kAttnHd + hh * 2 + 1] = Lsum;
             }
         }
         named_barrier(1, 32 * kAttnWarps);
@@ -245,7 +274,7 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     for (int64_t c = c_begin; c < c_end; ++c) {
         if (kh != seg_head) {
             if (seg_head >= 0) {
-                flush(seg_idx++);
+                flush(seg_idx++, seg_head);
                 m_run[0] = m_run[1] = -INFINITY;
                 l_run[0] = l_run[1] = 0.f;
 #pragma unroll
@@ -270,7 +299,7 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         }
 
         if (!s_fail[0] && !mbar_wait_bounded(&full[slot], ph, 0x202)) s_fail[0] = 1;
-        uint8_t* stp = smem + AttnSmem::ring + slot * kAttnStageBytes;
+        uint8_t* stp = smem + SL.ring + slot * kAttnStageBytes;
         const uint32_t st = ring_a + slot * kAttnStageBytes;
         const int64_t slot0 = ci * kAttnChunk + warp * 16;   // first cache slot of this warp's slice
 
@@ -382,65 +411,80 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         if (touched) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
-        if (++slot == kAttnStages) { slot = 0; ph ^= 1u; }
+        if (++slot == stages) { slot = 0; ph ^= 1u; }
         if (++ci == nch) { ci = 0; ++kh; }
     }
-    if (seg_head >= 0) flush(seg_idx);
+    if (seg_head >= 0) flush(seg_idx, seg_head);
 }
 
 // ------------------------------------------------------------------ K5
-// One CTA per kv head, one thread per (query head of the group, dimension).
-// The CTAs that own chunks of this head form one contiguous range; the list
-// of their records is resolved once into shared memory.
-constexpr int kCombineMaxRecs = 1024;
-
-__global__ void __launch_bounds__(1024) attn_combine_kernel(const AttnArgs a, int64_t G)
+// One 32-thread CTA per (kv head, query head of its group); lane l covers
+// dims 4l .. 4l+3.  The head's records sit in one contiguous run; a CTA in
+// the head's range that owned no chunk (possible when the grid outnumbers
+// the chunks) wrote nothing and is skipped.  Each round loads up to
+// kCombineBatch records, then folds them max-first in CTA order.
+__device__ __forceinline__ bool attn_cta_nonempty(int64_t bo, int64_t total, int64_t G)
 {
-    __shared__ int32_t s_rec[kCombineMaxRecs];
+    if (total < (1 << 20) && G < (1 << 11)) {
+        const uint32_t t32 = (uint32_t)total, g32 = (uint32_t)G, b32 = (uint32_t)bo;
+        return (b32 * t32) / g32 != ((b32 + 1) * t32) / g32;
+    }
+    return attn_begin(bo, total, G) != attn_begin(bo + 1, total, G);
+}
+
+__global__ void __launch_bounds__(32) attn_combine_kernel(const AttnArgs a, int64_t G)
+{
     pdl_wait();
     pdl_launch_dependents();
-    const int kh = blockIdx.x, tid = threadIdx.x;
+    const int group = a.group;
+    const int kh = blockIdx.x / group, gi = blockIdx.x - kh * group, lane = threadIdx.x;
     const int W = a.window;
     const int64_t pos = a.pos_dev ? *a.pos_dev : a.pos;
     const int64_t n_valid = pos + 1 < W ? pos + 1 : W;
     const int64_t nch = (n_valid + kAttnChunk - 1) / kAttnChunk;
     const int64_t total = (int64_t)a.n_kv * nch;
-    const int64_t bf = attn_owner((int64_t)kh * nch, total, G);
-    const int64_t bl = attn_owner((int64_t)kh * nch + nch - 1, total, G);
-    // CTAs in [bf, bl] that own no chunk (possible when the grid outnumbers
-    // the chunks) wrote no record and are skipped; the others are kept in
-    // CTA order so the sum below has a fixed order.
-    for (int64_t bo = bf + tid; bo <= bl; bo += blockDim.x) {
-        const int64_t beg = attn_begin(bo, total, G);
-        if (beg == attn_begin(bo + 1, total, G)) continue;
-        const int sidx = ((int64_t)kh == beg / nch) ? 0 : 1;
-        s_rec[bo - bf] = (int32_t)(bo * 2 + sidx);
-    }
-    for (int64_t bo = bf + tid; bo <= bl; bo += blockDim.x) {
-        if (attn_begin(bo, total, G) == attn_begin(bo + 1, total, G)) s_rec[bo - bf] = -1;
-    }
-    __syncthreads();
+    const int64_t bf = attn_owner((int64_t)kh * nch, total, G), bl = attn_owner((int64_t)kh * nch + nch - 1, total, G);
     const int nrec = (int)(bl - bf + 1);
-    const int gi = tid / a.hd, c = tid % a.hd;
-    if (gi >= a.group) return;
-    const size_t RF = attn_rec_floats(a.hd);
-    float M = -INFINITY;
-    for (int i = 0; i < nrec; ++i) {
-        const int r = s_rec[i];
-        if (r < 0) continue;
-        M = fmaxf(M, a.ws[(size_t)r * RF + kAttnMaxGroup * a.hd + gi * 2]);
+    const float* recs = a.ws + (size_t)kh * a.rmax * a.rec_floats;
+    float M = -INFINITY, L = 0.f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r0 = 0; r0 < nrec; r0 += kCombineBatch) {
+        // lane i decides whether record r0 + i exists
+        const bool mine = r0 + lane < nrec && lane < kCombineBatch && attn_cta_nonempty(bf + r0 + lane, total, G);
+        const uint32_t mask = __ballot_sync(0xffffffffu, mine);
+        float2 ml[kCombineBatch];
+        float4 ov[kCombineBatch];
+#pragma unroll
+        for (int u = 0; u < kCombineBatch; ++u) {
+            ml[u] = make_float2(-INFINITY, 0.f);
+            ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if ((mask >> u) & 1u) {
+                const float* rec = recs + (size_t)(r0 + u) * a.rec_floats;
+                ml[u] = __ldcg(reinterpret_cast<const float2*>(rec + group * kAttnHd) + gi);
+                ov[u] = __ldcg(reinterpret_cast<const float4*>(rec + gi * kAttnHd) + lane);
+            }
+        }
+        float mb = M;
+#pragma unroll
+        for (int u = 0; u < kCombineBatch; ++u) mb = fmaxf(mb, ml[u].x);
+        const float fo = M == -INFINITY ? 0.f : exp2f(M - mb);
+        O = make_float4(O.x * fo, O.y * fo, O.z * fo, O.w * fo);
+        L *= fo;
+#pragma unroll
+        for (int u = 0; u < kCombineBatch; ++u) {
+            if (ml[u].x == -INFINITY) continue;
+            const float f = exp2f(ml[u].x - mb);
+            O.x = fmaf(f, ov[u].x, O.x);
+            O.y = fmaf(f, ov[u].y, O.y);
+            O.z = fmaf(f, ov[u].z, O.z);
+            O.w = fmaf(f, ov[u].w, O.w);
+            L = fmaf(f, ml[u].y, L);
+        }
+        M = mb;
     }
-    float O = 0.f, L = 0.f;
-    for (int i = 0; i < nrec; ++i) {
-        const int r = s_rec[i];
-        if (r < 0) continue;
-        const float* rec = a.ws + (size_t)r * RF;
-        const float mv = rec[kAttnMaxGroup * a.hd + gi * 2];
-        const float f = (mv == -INFINITY) ? 0.f : exp2f(mv - M);
-        O += f * rec[gi * a.hd + c];
-        L += f * rec[kAttnMaxGroup * a.hd + gi * 2 + 1];
-    }
-    a.out[((int64_t)kh * a.group + gi) * a.hd + c] = O / L;
+    const float inv = 1.0f / L;
+    *reinterpret_cast<float4*>(a.out + ((int64_t)kh * group + gi) * kAttnHd + 4 * lane) =
+        make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
 }
 
 vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc, float* out, int n_q, int n_kv,
@@ -470,11 +514,15 @@ vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc
     a.pos_dev = pos_dev;
     a.qscale = scale * 1.4426950408889634f;
     a.ws = static_cast<float*>(ws);
+    a.rec_floats = attn_rec_floats(a.group, hd);
+    a.rmax = attn_rmax(n_kv);
+    a.stages = env_int_attn("VOX_ATTN_STAGES", 3, 2, kAttnMaxStages);
+    const AttnSmem SL = attn_smem_layout(a.stages);
 
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(gqa_decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)AttnSmem::total);
+                                             (int)attn_smem_layout(kAttnMaxStages).total);
         if (e != cudaSuccess) {
             set_cuda_error(e);
             return VOX_ERR_CUDA;
@@ -482,9 +530,9 @@ vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc
         attr_set = true;
     }
     const int64_t G = attn_grid(n_kv, window);
-    st = launch_pdl(gqa_decode_attn_kernel, dim3((unsigned)G), dim3(kAttnThreads), AttnSmem::total, s, kmap, vmap, a);
+    st = launch_pdl(gqa_decode_attn_kernel, dim3((unsigned)G), dim3(kAttnThreads), SL.total, s, kmap, vmap, a);
     if (st != VOX_OK) return st;
-    return launch_pdl(attn_combine_kernel, dim3((unsigned)n_kv), dim3((unsigned)(a.group * hd)), 0, s, a, G);
+    return launch_pdl(attn_combine_kernel, dim3((unsigned)(n_kv * a.group)), dim3(32), 0, s, a, G);
 }
 
 }  // namespace vox

@@ -159,13 +159,14 @@ typedef struct {
  * i < m (1 <= m <= 8) and packed rows j < n, dequantising in registers with no
  * separate pass, then the epilogue.  x: device fp32 [m][ldx]; y: device fp32
  * [m][ldy] (n columns, or n/2 for SILU_MUL).  The product runs on the tensor
- * cores with the activations rounded to fp16 after an exact per-row
- * power-of-two scaling and fp32 accumulation; the result is within 2e-3 of
- * the fp64 product, normalised by |x_i| |w_j|.  workspace: device scratch of
- * vox_q4_gemv_workspace() bytes, 16-byte aligned: per-tile arrival counters
- * (for tiles split between CTAs), partial tiles and argmax candidates.  Zero
- * it once before its first use; every call leaves the counters at zero
- * again.  Calls that share a workspace must not overlap on the GPU.  Limits: m * ceil(k/64)*64 <= 81920.
+ * cores with each 32-column block of x (times the RMSNorm weight) rounded to
+ * fp16 after an exact power-of-two scaling of its own, and fp32
+ * accumulation; the result is within 2e-3 of the fp64 product, normalised by
+ * |x_i| |w_j|.  workspace: device scratch of vox_q4_gemv_workspace() bytes
+ * (256), 16-byte aligned: the argmax keys and arrival counter.  Zero it once
+ * before its first use; every call leaves it at zero again.  Calls that
+ * share a workspace must not overlap on the GPU.  Limits: m * ceil(k/64)*64
+ * <= 81920 (the fp16 activations live in shared memory).
  * Errors: NULL -> VOX_ERR_NULL; m outside 1..8, k % 32, ldx < k, ldy too small,
  * SILU_MUL with n % 16, KV_APPEND rows that do not fit n, or the size limit ->
  * VOX_ERR_SHAPE; weight data not 16-byte aligned -> VOX_ERR_ALIGN; bad
@@ -208,8 +209,9 @@ vox_status vox_kv_append_rolling(void *k_cache, void *v_cache, const void *k_new
  * 16-byte aligned; out: device fp32 [n_q_heads][head_dim].  Split-KV: slot
  * ranges are reduced independently into the workspace (device, at least
  * vox_gqa_decode_attn_workspace() bytes, 16-byte aligned, no initial contents
- * needed) and merged by a log-sum-exp combine.  Calls sharing a workspace
- * must not overlap on the GPU.  head_dim must be 128 (the decoder's).
+ * needed) and merged by a log-sum-exp combine (a second, small kernel).
+ * Calls sharing a workspace must not overlap on the GPU.  head_dim must be
+ * 128 (the decoder's).
  * Errors: NULL -> VOX_ERR_NULL; pos < 0, window <= 0, n_q % n_kv != 0, a
  * group above 8 or more than 512 kv heads -> VOX_ERR_RANGE; other head_dim
  * -> VOX_ERR_SHAPE; short workspace -> VOX_ERR_WORKSPACE; caches or workspace
