@@ -28,6 +28,7 @@
 // written one reloads that row from global memory.
 #include "tma.cuh"
 
+#include <mutex>
 #include <stdlib.h>
 
 namespace vox {
@@ -96,8 +97,8 @@ struct AttnArgs {
 // Partial record of one CTA for one kv head: O[group][hd], then (m, l) per
 // query head of the group, padded to 16 bytes.  The records of kv head kh
 // are contiguous: slot kh * rmax + (CTA - first CTA of kh).
-__host__ __device__ inline int attn_rec_floats(int group, int hd) { return (group * (hd + 2) + 3) & ~3; }
-__host__ __device__ inline int attn_rmax(int n_kv) { return (kAttnMaxCtas + n_kv - 1) / n_kv + 2; }
+__host__ __device__ constexpr int attn_rec_floats(int group, int hd) { return (group * (hd + 2) + 3) & ~3; }
+__host__ __device__ constexpr int attn_rmax(int n_kv) { return (kAttnMaxCtas + n_kv - 1) / n_kv + 2; }
 
 static int env_int_attn(const char* name, int dflt, int lo, int hi)
 {
@@ -535,4 +536,79 @@ vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc
     return launch_pdl(attn_combine_kernel, dim3((unsigned)(n_kv * a.group)), dim3(32), 0, s, a, G);
 }
 
+// --------------------------------------------- allocation-free entry point
+// vox_gqa_decode_attn needs the caller to hand in device scratch for the
+// split-KV partial records.  Some callers cannot: a host program that links
+// only this C library and owns no device allocator, or a real-time audio
+// thread that must not call cudaMalloc (it can block and synchronise the
+// device).  vox_gqa_decode_attn_static serves them from one fixed scratch
+// array in device memory, sized for at most kStaticMaxKv kv heads with
+// groups of at most kStaticMaxGroup query heads at head_dim 128 (the
+// decoder's 8 kv heads x 4).  It allocates nothing: the array is part of the
+// loaded module, and its address is looked up once per device.
+constexpr int kStaticMaxKv = 8;
+constexpr int kStaticMaxGroup = 4;
+constexpr size_t kStaticScratchBytes =
+    (size_t)kStaticMaxKv * attn_rmax(kStaticMaxKv) * attn_rec_floats(kStaticMaxGroup, kAttnHd) * sizeof(float);
+
+static __device__ __align__(256) uint8_t g_attn_static_scratch[kStaticScratchBytes];
+
+// Device address of the scratch array on the current device, looked up with
+// cudaGetSymbolAddress the first time each device is used and kept.
+static vox_status attn_static_scratch(void** out)
+{
+    static std::mutex mu;
+    static void* addr[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_cuda_error(e);
+        return VOX_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= 64) return VOX_ERR_RANGE;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_attn_static_scratch);
+        if (e != cudaSuccess) {
+            set_cuda_error(e);
+            return VOX_ERR_CUDA;
+        }
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return VOX_OK;
+}
+
 }  // namespace vox
+
+extern "C" vox_status vox_gqa_decode_attn_static(const float* q, const void* k_cache, const void* v_cache, float* out,
+                                                 int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                                 int32_t window, int64_t pos, float scale, void* stream)
+{
+    using namespace vox;
+    if (!q || !k_cache || !v_cache || !out) return VOX_ERR_NULL;
+    if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return VOX_ERR_RANGE;
+    if (window < 1 || pos < 0) return VOX_ERR_RANGE;
+    if (head_dim != kAttnHd) return VOX_ERR_SHAPE;
+    if ((int64_t)n_kv_heads * window > 0x7fffff00LL) return VOX_ERR_SHAPE;
+    const int group = n_q_heads / n_kv_heads;
+    if (n_kv_heads > kStaticMaxKv || group > kStaticMaxGroup) {
+        set_error_text("vox_gqa_decode_attn_static: the static scratch holds at most 8 kv heads with groups of "
+                       "at most 4 query heads; use vox_gqa_decode_attn with a workspace");
+        return VOX_ERR_RANGE;
+    }
+    if (((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15u) != 0)
+        return VOX_ERR_ALIGN;
+    // the records this call writes: n_kv runs of rmax records of the group's size
+    const size_t need = (size_t)n_kv_heads * attn_rmax(n_kv_heads) * attn_rec_floats(group, kAttnHd) * sizeof(float);
+    if (need > kStaticScratchBytes) {
+        set_error_text("vox_gqa_decode_attn_static: shape needs more than the static scratch");
+        return VOX_ERR_RANGE;
+    }
+    void* scratch = nullptr;
+    vox_status st = attn_static_scratch(&scratch);
+    if (st != VOX_OK) return st;
+    return launch_gqa_decode_attn(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_dim, window, pos, nullptr,
+                                  scale, scratch, static_cast<cudaStream_t>(stream));
+}

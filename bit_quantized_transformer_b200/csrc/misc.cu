@@ -20,6 +20,11 @@ void set_cuda_error(cudaError_t e)
 
 const char* last_error_text() { return t_last_error; }
 
+void set_error_text(const char* text)
+{
+    snprintf(t_last_error, sizeof(t_last_error), "%s", text);
+}
+
 vox_status check_launch()
 {
     cudaError_t e = cudaGetLastError();

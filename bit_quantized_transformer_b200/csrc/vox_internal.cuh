@@ -25,6 +25,7 @@ __host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return
 
 // ---------------------------------------------------------- host plumbing
 void set_cuda_error(cudaError_t e);
+void set_error_text(const char* text);      // message for vox_last_error
 vox_status check_launch();                  // cudaGetLastError -> VOX_ERR_CUDA
 int device_sm_count();                      // SMs of the current device (cached per device)
 

@@ -81,6 +81,7 @@ _SIGS = {
     "vox_kv_append_rolling": (_I32, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _P]),
     "vox_gqa_decode_attn": (_I32, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _F, _P, _SZ, _P]),
     "vox_gqa_decode_attn_workspace": (_SZ, [_I32, _I32, _I32, _I32]),
+    "vox_gqa_decode_attn_static": (_I32, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _F, _P]),
     "vox_window_attn": (_I32, [_P, _I64, _P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _I32, _I64,
                                _I32, _I32, _I32, _F, _P]),
     "vox_rmsnorm": (_I32, [_P, _I64, _I64, _I64, _F, _P, _P, _I32, _I64, _P]),
@@ -173,6 +174,13 @@ def vox_gqa_decode_attn(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_di
     _check(lib.vox_gqa_decode_attn(ptr(q), ptr(k_cache), ptr(v_cache), ptr(out), n_q_heads, n_kv_heads,
                                    head_dim, window, pos, scale, ptr(workspace), ws_bytes, stream_ptr(stream)),
            "vox_gqa_decode_attn")
+
+
+def vox_gqa_decode_attn_static(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_dim, window, pos, scale,
+                               stream=None):
+    _check(lib.vox_gqa_decode_attn_static(ptr(q), ptr(k_cache), ptr(v_cache), ptr(out), n_q_heads, n_kv_heads,
+                                          head_dim, window, pos, scale, stream_ptr(stream)),
+           "vox_gqa_decode_attn_static")
 
 
 def vox_window_attn(q, ldq, k_hist, v_hist, ld_hist, n_hist, k_new, v_new, ld_new, n_q, out, out_dtype, ldo,

@@ -223,6 +223,28 @@ vox_status vox_gqa_decode_attn(const float *q, const void *k_cache, const void *
 size_t vox_gqa_decode_attn_workspace(int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                                      int32_t window);
 
+/* vox_gqa_decode_attn_static -- an interface of this library with no
+ * counterpart in the source pages: vox_gqa_decode_attn without a caller
+ * workspace, for callers that cannot hand in device scratch (a host program
+ * that links only this library and owns no device allocator; a real-time
+ * audio thread that must not call cudaMalloc, which can block and
+ * synchronise the device).  Same arguments, result and precision as
+ * vox_gqa_decode_attn.  It allocates nothing: the split-KV partial records
+ * go to one fixed array in device memory that is part of the loaded library
+ * (about 1.2 MiB), sized for at most 8 kv heads with at most 4 query heads
+ * per kv head at head_dim 128 (the decoder's 32 / 8 fits); larger shapes
+ * return VOX_ERR_RANGE with a message in vox_last_error().  Nothing in the
+ * array needs to start at zero: every call writes each record it reads.
+ * All calls on one device share the array, so two calls that overlap on the
+ * GPU (other streams, concurrent graph replays) corrupt each other's
+ * results: order them on one stream.  The first call on each device looks
+ * the array's address up (cudaGetSymbolAddress); make that call outside any
+ * stream capture.  Other errors as vox_gqa_decode_attn. */
+vox_status vox_gqa_decode_attn_static(const float *q, const void *k_cache, const void *v_cache,
+                                      float *out, int32_t n_q_heads, int32_t n_kv_heads,
+                                      int32_t head_dim, int32_t window, int64_t pos, float scale,
+                                      void *stream);
+
 /* vox_window_attn -- [ARCH] encoder: causal sliding-window multi-head
  * attention for a chunk of n_q query rows.  Query row i sits at absolute
  * position n_hist + i and sees key position p iff pos_i - window < p <= pos_i.
