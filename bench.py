@@ -44,7 +44,7 @@ FILLED = 8192 + 300
 # of the current Q4_0 GEMV on each decoder shape weighted by the step's launch
 # mix (the GEMV summary under profiles/); set to None when the kernel changes,
 # until it is captured again
-GEMV_TRAFFIC_BYTES_PER_LAUNCH = 18_547_000
+GEMV_TRAFFIC_BYTES_PER_LAUNCH = None
 
 
 def parse_args(argv=None):
@@ -55,6 +55,10 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
+    p.add_argument("--workload", choices=["decoder", "encoder", "sweep"], default="decoder",
+                   help="decoder: the headline line (default); encoder: the 32-layer encoder chunk at M=256 "
+                        "and its GEMMs; sweep: the decoder shapes at M in {1,4,16,64,256} and the attention at "
+                        "KV in {512, 4096, 8192 wrapped}")
     return p.parse_args(argv)
 
 
@@ -379,10 +383,185 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------ supplementary workloads
+def graph_of(fn):
+    """Capture fn (launches on the current stream) into a CUDA graph after
+    one warm-up call on a side stream."""
+    import torch
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def run_encoder(args):
+    """Config 3: the 32-layer encoder chunk (M = 256 rows, dim 1280) plus the
+    adapter GEMM, and the same chunk's Q4_0 GEMMs alone (K2, tcgen05)."""
+    import torch
+
+    import synth
+    from bit_quantized_transformer_b200 import build
+
+    build.build()
+    from bit_quantized_transformer_b200 import vox as V
+    from bit_quantized_transformer_b200 import workloads as WL
+
+    shape = synth.EncoderShape()
+    em = WL.EncoderModel(shape, seed=0)
+    steps = max(3, min(args.steps, 50))
+
+    def chunk():
+        em.reset()
+        em.run()
+
+    g = graph_of(chunk)
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    ms = time_replays(g, steps, 1) / steps
+
+    # the chunk's GEMMs alone: every layer's QKV, O, up, down at M = 256 and the adapter at M = 64
+    R, D, F = shape.rows, shape.dim, shape.ffn
+    xb = torch.randn(R, F, device="cuda").to(torch.bfloat16)
+    yb = torch.empty(R, max(3 * D, F, shape.adapter_out), dtype=torch.bfloat16, device="cuda")
+    calls = []
+    for l in range(em.L):
+        calls += [(em.wqkv[l], R, D, 3 * D), (em.wo[l], R, D, D), (em.wup[l], R, D, F), (em.wdown[l], R, F, D)]
+    calls.append((em.adapter, R // shape.downsample, shape.downsample * D, shape.adapter_out))
+
+    def gemms():
+        for w, m, k, n in calls:
+            V.vox_q4_gemm(w, xb, V.VOX_BF16, m, k, yb, V.VOX_BF16, yb.shape[1])
+
+    gg = graph_of(gemms)
+    for _ in range(3):
+        gg.replay()
+    ms_g = time_replays(gg, steps, 1) / steps
+    flops = em.gemm_flops()
+    peak = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+    tf_g = flops / (ms_g / 1e3) / 1e12
+    line = {"metric": "encoder chunk Q4_0 GEMM TFLOP/s (bf16 tensor cores)", "value": tf_g, "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": ms_g,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 MMA, f32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": "encoder_chunk_32L_M256_dim1280_plus_adapter_M64", "gemm_flops": flops,
+                       "l2": "weights 353.9 MB > L2"},
+            "roofline": {"bound": "tensor", "achieved": tf_g, "peak": peak["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tf_g / peak["bf16_tflops"], "frac_of_sustained": tf_g / peak["bf16_tflops_sustained"],
+                         "traffic": None},
+            "chunk_ms": ms, "chunk_tflops_gemm_only_numerator": flops / (ms / 1e3) / 1e12,
+            "gpu_launches": len(calls) * steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_sweep(args):
+    """Config 4: the decoder projection shapes at M in {1,4,16,64,256} (K1 for
+    M <= 8, K2 for M >= 16, and K1 as two M = 8 launches at M = 16 for the
+    crossover), over weight copies totalling > 2x L2; then the decode
+    attention at KV 512, 4096 and 8192 (wrapped)."""
+    import math
+
+    import numpy as np
+    import torch
+
+    import synth
+    from bit_quantized_transformer_b200 import build
+
+    build.build()
+    from bit_quantized_transformer_b200 import vox as V
+    from bit_quantized_transformer_b200 import workloads as WL
+
+    shapes = [(6144, 3072), (3072, 4096), (18432, 3072), (3072, 9216), (131072, 3072)]
+    Ms = [1, 4, 16, 64, 256]
+    reps = 3
+    out = {}
+    cross = {}
+    x32 = torch.randn(256, 9216, device="cuda")
+    xbf = x32.to(torch.bfloat16)
+    y = torch.empty(256 * 131072, device="cuda")
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    for n, k in shapes:
+        qs, d = synth.q4_blocks(n, k, 0, 77)
+        packed, w0 = WL.pack_q4(qs, d, "cuda")
+        nbytes = packed.numel()
+        copies = max(2, int(math.ceil(300e6 / nbytes)))
+        keep = [packed] + [packed.clone() for _ in range(copies - 1)]
+        wts = [V.weight(t, n, k) for t in keep]
+        res = {}
+        for M in Ms + ["16_gemv"]:
+            if M == "16_gemv":
+                def fn():
+                    for w in wts:
+                        for h in range(2):
+                            V.vox_q4_gemv(w, x32[8 * h:], 8, 9216, y, n, None, ws, 4096)
+            elif M <= 8:
+                def fn(M=M):
+                    for w in wts:
+                        V.vox_q4_gemv(w, x32, M, 9216, y, n, None, ws, 4096)
+            else:
+                def fn(M=M):
+                    for w in wts:
+                        V.vox_q4_gemm(w, xbf, V.VOX_BF16, M, 9216, y, V.VOX_F32, n)
+            g = graph_of(fn)
+            g.replay()
+            us = time_replays(g, reps, 1) / (reps * copies) * 1e3
+            m = 16 if M == "16_gemv" else M
+            res[str(M)] = {"us": us, "weight_gbs": nbytes / us / 1e3, "tflops": 2 * m * n * k / us / 1e6}
+            del g
+        out[f"{n}x{k}"] = res
+        cross[f"{n}x{k}"] = "K2 (tcgen05 GEMM) faster at M=16" if res["16"]["us"] < res["16_gemv"]["us"] else \
+            "K1 (two M=8 GEMVs) faster at M=16"
+        del keep, wts
+        torch.cuda.empty_cache()
+    # attention at three cache lengths
+    n_q, n_kv, hd, W = 32, 8, 128, 8192
+    NL = 26
+    caches = [(torch.randn(n_kv, W, hd, device="cuda").to(torch.bfloat16),
+               torch.randn(n_kv, W, hd, device="cuda").to(torch.bfloat16)) for _ in range(NL)]
+    q = torch.randn(n_q, hd, device="cuda")
+    o = torch.empty(n_q, hd, device="cuda")
+    wsb = V.vox_gqa_decode_attn_workspace(n_q, n_kv, hd, W)
+    wsa = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    attn = {}
+    for pos in (511, 4095, W + 300):
+        def fa(pos=pos):
+            for l in range(NL):
+                V.vox_gqa_decode_attn(q, caches[l][0], caches[l][1], o, n_q, n_kv, hd, W, pos, 1 / math.sqrt(hd),
+                                      wsa, wsb)
+        g = graph_of(fa)
+        g.replay()
+        us = time_replays(g, 5, 1) / (5 * NL) * 1e3
+        nb = 2 * n_kv * min(pos + 1, W) * hd * 2
+        attn[str(min(pos + 1, W)) + (" wrapped" if pos >= W else "")] = {"us_per_layer": us, "gbs": nb / us / 1e3}
+        del g
+    assert V.vox_device_status(True) == 0
+    line = {"metric": "decoder-shape sweep: weight GB/s and TFLOP/s per M; attention GB/s per KV length",
+            "value": out["131072x3072"]["1"]["weight_gbs"], "unit": "GB/s", "n_gpus": 1, "steps": reps,
+            "warmup": 1, "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "q4_0 weights; fp16 (K1) / bf16 (K2) tensor-core inputs; f32 accumulate", "data": "synthetic",
+            "config": {"workload": "decoder_shapes_M_sweep_and_attention_kv_sweep", "M": Ms,
+                       "l2": "weight copies > 2x L2 per shape"},
+            "sweep": out, "crossover": cross, "attention": attn}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "encoder":
+        return run_encoder(args)
+    if args.workload == "sweep":
+        return run_sweep(args)
     return run_ours(args)
 
 

@@ -8,18 +8,24 @@
 // 아키텍처" (dim 1280, FFN 5120, adapter 5120 -> 3072).
 //
 // One CTA computes a 128-weight-row x BN-token tile of Y^T in tensor memory:
-//   warp 0      producer: bulk copies of the 8 packed 576-byte records of the
-//               128 rows for one 64-column chunk, and a TMA tile (128-byte
+//   warp 0      producer: per 64-column chunk, one 2-D TMA load of the 8
+//               packed 576-byte records of the 128 rows (the packed weight
+//               viewed as [tiles][chunks x 576 B]) and one TMA tile (128-byte
 //               swizzle) of BN activation rows x 64 columns;
 //   warp 1      allocates BN tensor-memory columns and, from one thread,
 //               issues tcgen05.mma kind::f16 (M=128, N=BN, K=16, bf16 in, fp32
 //               accumulate) on shared-memory descriptors, committing each
 //               stage back to the producer;
-//   warps 2-9   dequantise: thread (row, block) turns 32 codes into bf16
-//               (q - 8) * d and writes them in the canonical K-major
-//               128-byte-swizzled layout the MMA reads; after the last chunk
-//               they read the accumulator with tcgen05.ld and run the
-//               epilogue (residual add, GELU, fp32 or bf16 store).
+//   warps 2-9   dequantise: warp w takes the record of row tile w, lane
+//               (g, t) its 16 bytes of codes (rows g and g+8, both 32-column
+//               blocks); each 32-bit word gives four bf16 pairs 128 + q by
+//               OR-ing the nibble into the fraction of 128.0 (exact), then
+//               one exact subtraction of 136 and one multiply by d (one
+//               rounding to bf16), stored in the canonical K-major
+//               128-byte-swizzled layout the MMA reads (4-byte stores, free of
+//               bank conflicts); after the last chunk they read the
+//               accumulator with tcgen05.ld and run the epilogue (residual
+//               add, GELU, fp32 or bf16 store).
 #include "tma.cuh"
 
 namespace vox {
@@ -92,11 +98,26 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8])
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// bf16x2 a - b and a * b, one rounding each (b exact in the subtraction here).
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 __device__ __forceinline__ float gelu_erf_g(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
 
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a)
+q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap, const GemmArgs a)
 {
     using C = GemmCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
@@ -139,8 +160,8 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a)
         if (lane == 0) {
             pdl_launch_dependents();
             prefetch_tmap(&xmap);
-            const int ntile = (int)min64(8, a.tiles - group * 8);
-            const uint32_t bytes = (uint32_t)ntile * kChunkBytes + C::xbytes;
+            prefetch_tmap(&wmap);
+            const uint32_t bytes = (uint32_t)kGemmRawBytes + C::xbytes;   // rows past the matrix read as zeros
             for (int kb = 0; kb < kc; ++kb) {
                 const int s = kb % C::stages;
                 const uint32_t ph = (uint32_t)((kb / C::stages) & 1);
@@ -148,9 +169,7 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a)
                 if (s_fail[0]) break;
                 uint8_t* st = smem + s * C::stage;
                 mbar_arrive_expect_tx(&full[s], bytes);
-                for (int tt = 0; tt < ntile; ++tt)
-                    bulk_g2s(st + C::xbytes + kGemmABytes + tt * kChunkBytes,
-                             a.w + ((group * 8 + tt) * (int64_t)kc + kb) * kChunkBytes, kChunkBytes, &full[s]);
+                tma_load_2d(st + C::xbytes + kGemmABytes, &wmap, kb * (kChunkBytes / 4), (int32_t)(group * 8), &full[s]);
                 tma_load_2d(st, &xmap, kb * 64, (int32_t)m0, &full[s]);
             }
         }
@@ -177,36 +196,45 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const GemmArgs a)
         }
     } else {
         // ------------------------------------------------- dequant + epilogue
-        const int dw = warp - 2;                    // 0..7
+        const int dw = warp - 2;                    // 0..7: the row tile this warp dequantises
         const int q = warp & 3;                     // tensor-memory lane quarter of this warp
-        const int r = 32 * q + lane;                // weight row within the CTA tile
-        const int bb = dw >> 2;                     // block (0, 1) of the chunk
-        const int tt = r >> 4, i16 = r & 15, g = i16 & 7, rowsel = i16 >> 3;
+        const int r = 32 * q + lane;                // weight row of the epilogue
+        const int g = lane >> 2, t = lane & 3;
+        const uint32_t M_L = 0x000F000Fu, C_B = 0x43004300u, B136 = 0x43084308u;   // 128.0, 136.0 (bf16x2)
+        const uint32_t row_g = (uint32_t)(dw * 16 + g), row_g8 = row_g + 8u;
         for (int kb = 0; kb < kc; ++kb) {
             const int s = kb % C::stages;
             const uint32_t ph = (uint32_t)((kb / C::stages) & 1);
             if (!s_fail[0] && !mbar_wait_bounded(&full[s], ph, 0x303)) s_fail[0] = 1;
             uint8_t* st = smem + s * C::stage;
-            const uint8_t* rec = st + C::xbytes + kGemmABytes + tt * kChunkBytes;
-            const float d = __half2float(*reinterpret_cast<const __half*>(rec + kChunkQsBytes + 8 * g + 2 * (bb * 2 + rowsel)));
-            uint2 wv[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) wv[t] = *reinterpret_cast<const uint2*>(rec + 16 * (4 * g + t) + 8 * bb);
             uint8_t* A = st + C::xbytes;
+            if (dw * 16 < (int)(a.n - group * kGemmRows)) {
+                const uint8_t* rec = st + C::xbytes + kGemmABytes + dw * kChunkBytes;
+                const uint4 qv = *reinterpret_cast<const uint4*>(rec + 16 * lane);
+                const uint2 dd = *reinterpret_cast<const uint2*>(rec + kChunkQsBytes + 8 * g);
+                // scales as bf16 pairs: d(row g, block 0), d(row g+8, block 0), d(g, 1), d(g+8, 1)
+                const float2 d0 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+                const float2 d1 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+                const uint32_t D[4] = {pack_bf16x2(d0.x, d0.x), pack_bf16x2(d0.y, d0.y), pack_bf16x2(d1.x, d1.x),
+                                       pack_bf16x2(d1.y, d1.y)};
 #pragma unroll
-            for (int uu = 0; uu < 4; ++uu) {
-                const int half = uu >> 1, w = uu & 1;
-                float v[8];
+                for (int bb = 0; bb < 2; ++bb) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int t = j >> 1, elem = j & 1;
-                    const uint32_t word = w ? wv[t].y : wv[t].x;
-                    const int sh = 4 * (rowsel * 2 + half + 4 * elem);
-                    v[j] = (float)((int)((word >> sh) & 15u) - 8) * d;
+                    for (int wi = 0; wi < 2; ++wi) {
+                        const uint32_t w = wi ? (bb ? qv.w : qv.y) : (bb ? qv.z : qv.x);
+                        // nibble pairs: (w, w>>8) low halves, (w>>4, w>>12) high halves; rows g, g+8
+                        const uint32_t src[4] = {w, w >> 8, w >> 4, w >> 12};
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const uint32_t raw = lop3_and_or(src[h], M_L, C_B);            // 128 + q, exact
+                            const uint32_t v = bf16x2_mul(bf16x2_sub(raw, B136), D[bb * 2 + (h & 1)]);
+                            const uint32_t row = (h & 1) ? row_g8 : row_g;
+                            // columns 32 bb + 16 (h >> 1) + 8 wi + 2t, +1: unit 4 bb + 2 (h >> 1) + wi
+                            const uint32_t unit = (uint32_t)(bb * 4 + (h >> 1) * 2 + wi);
+                            *reinterpret_cast<uint32_t*>(A + sw128_offset(row, unit) + 4 * t) = v;
+                        }
+                    }
                 }
-                const uint4 pk = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-                *reinterpret_cast<uint4*>(A + sw128_offset((uint32_t)r, (uint32_t)(bb * 4 + uu))) = pk;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
@@ -253,6 +281,11 @@ static vox_status launch_gemm_bn(const GemmArgs& a, const void* x, int64_t ldx, 
     vox_status st = make_tmap_2d(&xmap, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.k, (uint64_t)a.m,
                                  (uint64_t)ldx * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != VOX_OK) return st;
+    // the packed weight as 32-bit words: [tiles][kc * 144], one box = one chunk of 8 row tiles
+    CUtensorMap wmap;
+    st = make_tmap_2d(&wmap, a.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)a.kc * (kChunkBytes / 4),
+                      (uint64_t)a.tiles, (uint64_t)a.kc * kChunkBytes, kChunkBytes / 4, 8, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != VOX_OK) return st;
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(q4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem);
@@ -263,7 +296,7 @@ static vox_status launch_gemm_bn(const GemmArgs& a, const void* x, int64_t ldx, 
         attr = true;
     }
     dim3 grid((unsigned)ceil_div(a.tiles, 8), (unsigned)ceil_div(a.m, BN));
-    return launch_pdl(q4_gemm_kernel<BN>, grid, dim3(kGemmThreads), (size_t)C::smem, s, xmap, a);
+    return launch_pdl(q4_gemm_kernel<BN>, grid, dim3(kGemmThreads), (size_t)C::smem, s, xmap, wmap, a);
 }
 
 static int pick_bn(int64_t tiles, int64_t m)

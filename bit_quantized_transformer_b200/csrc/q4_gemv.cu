@@ -43,9 +43,11 @@ namespace vox {
 #endif
 constexpr int kGemvWarps = VOX_GEMV_WARPS;
 constexpr int kGemvThreads = 32 * kGemvWarps;
-constexpr int kGemvRecs = 4;                                  // records per ring stage
-constexpr int kGemvStageBytes = kGemvRecs * kChunkBytes;      // 2304
-static_assert(kGemvRecs == 4, "the record loop's fast path adds four records");
+#ifndef VOX_GEMV_RECS
+#define VOX_GEMV_RECS 4
+#endif
+constexpr int kGemvRecs = VOX_GEMV_RECS;                      // records per ring stage (one bulk copy)
+constexpr int kGemvStageBytes = kGemvRecs * kChunkBytes;
 constexpr int kGemvMaxStages = 8;
 constexpr int kGemvDefaultStages = 3;
 #ifndef VOX_GEMV_MIN_CTAS
@@ -78,6 +80,7 @@ struct GemvArgs {
     int32_t* argmax;
     uint8_t* ws;
     int32_t stages;
+    int32_t pre;                             // ring stages issued before griddepcontrol.wait
 };
 
 // Shared-memory carve-up, computed identically on host and device.
@@ -400,7 +403,7 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
         for (int s = 0; s < stages; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        for (int j = 0; j < stages && j < nbatch; ++j)
+        for (int j = 0; j < a.pre && j < nbatch; ++j)
             gemv_issue(a.w, wb, we, j, ring + j * kGemvStageBytes, &bars[j]);
         s_ptile[warp] = -1;
     }
@@ -420,6 +423,10 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
         if (lane == 0) s_sq[warp * 8 + i] = sq;
     }
     __syncthreads();
+    // the rest of the ring, issued once the activations are in
+    if (lane == 0)
+        for (int j = a.pre; j < stages && j < nbatch; ++j)
+            gemv_issue(a.w, wb, we, j, ring + j * kGemvStageBytes, &bars[j]);
 
     // RMSNorm factors of this lane's tokens 2t, 2t+1 (zero for tokens past m)
     float rr[2];
@@ -501,12 +508,23 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
                 ch = ch + 1 == kc ? 0 : ch + 1;
             }
             if (left > kGemvRecs && cin + kGemvRecs < kc) {
-                // no tile end and no range end inside this stage
-                acc[0] += (p[0][0] + p[1][0]) + (p[2][0] + p[3][0]);
-                acc[2] += (p[0][2] + p[1][2]) + (p[2][2] + p[3][2]);
+                // no tile end and no range end inside this stage: pairwise sums of the records
+#pragma unroll
+                for (int w = 1; w < kGemvRecs; w <<= 1)
+#pragma unroll
+                    for (int r = 0; r + w < kGemvRecs; r += 2 * w) {
+                        p[r][0] += p[r + w][0];
+                        p[r][2] += p[r + w][2];
+                        if (MT != 1) {
+                            p[r][1] += p[r + w][1];
+                            p[r][3] += p[r + w][3];
+                        }
+                    }
+                acc[0] += p[0][0];
+                acc[2] += p[0][2];
                 if (MT != 1) {
-                    acc[1] += (p[0][1] + p[1][1]) + (p[2][1] + p[3][1]);
-                    acc[3] += (p[0][3] + p[1][3]) + (p[2][3] + p[3][3]);
+                    acc[1] += p[0][1];
+                    acc[3] += p[0][3];
                 }
                 cin += kGemvRecs;
                 left -= kGemvRecs;
@@ -626,6 +644,7 @@ vox_status launch_q4_gemv(const uint8_t* w, int64_t n, int64_t k, const float* x
     while (stages > 2 && L.total > 227 * 1024) L = gemv_smem_layout(a.kc, a.m, --stages);
     if (L.total > 227 * 1024) return VOX_ERR_SHAPE;            // activations do not fit shared memory
     a.stages = stages;
+    a.pre = env_int("VOX_GEMV_PREFETCH", 1, 0, stages);
 
     void (*kern)(GemvArgs) = m == 1 ? q4_gemv_kernel<1> : q4_gemv_kernel<8>;
     static bool attr_set = false;

@@ -108,11 +108,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
-// Blocking wait on an mbarrier phase: each try_wait may suspend the thread
-// for up to kSuspendHintNs (the hardware resumes it as soon as the phase
-// completes), so waiting warps do not compete for issue slots.  The wait is
-// bounded: after kWaitTries attempts (about one second) it records `where`
-// in the device status word and returns false, and the caller leaves its loop.
+// Blocking wait on an mbarrier phase, bounded: after about one second
+// (globaltimer) it records `where` in the device status word and returns
+// false, and the caller leaves its loop.  The default form polls try_wait
+// without a suspend-time hint (measured faster on B200 than a long hint,
+// whose wake-up adds latency to every wait that has to wait); mode 0 keeps
+// the hinted form, mode 2 polls test_wait.
 constexpr uint32_t kSuspendHintNs = 1u << 20;
 constexpr uint32_t kWaitTries = 1024;
 
@@ -129,10 +130,44 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+#ifndef VOX_WAIT_MODE
+#define VOX_WAIT_MODE 1
+#endif
+
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int32_t where)
 {
+#if VOX_WAIT_MODE == 0
     for (uint32_t it = 0; it < kWaitTries; ++it)
         if (mbar_try_wait_hint(bar, parity)) return true;
+#else
+    if (VOX_WAIT_MODE == 1 ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (VOX_WAIT_MODE == 1 ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity)) return true;
+        if (global_ns() - t0 > 1000000000ull) break;              // about one second
+    }
+#endif
     atomicCAS(&g_vox_device_status, 0, where);
     return false;
 }
