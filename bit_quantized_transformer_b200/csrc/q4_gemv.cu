@@ -240,12 +240,14 @@ struct GemvBest {
 
 // Epilogue of one finished 16-row tile from the MMA accumulator layout:
 // lane (g, t) holds acc[2h + e] = tile row g + 8h, token 2t + e; rr[e] is the
-// RMSNorm factor of token 2t + e (1 without RMSNorm).  Not inlined: it runs
-// once per tile and keeps the record loop small.
+// RMSNorm factor of token 2t + e (1 without RMSNorm).  `pre` (with use_pre)
+// holds the residual values in the same layout, loaded ahead by the caller.
+// Not inlined: it runs once per tile and keeps the record loop small.
 __device__ __noinline__ GemvBest gemv_epilogue(const GemvArgs& a, int64_t tile, float4 acc4, int g, int t, float r0,
-                                               float r1, int64_t pos, GemvBest best)
+                                               float r1, int64_t pos, GemvBest best, float4 pre, int use_pre)
 {
     const float acc[4] = {acc4.x, acc4.y, acc4.z, acc4.w};
+    const float prv[4] = {pre.x, pre.y, pre.z, pre.w};
     const float rr[2] = {r0, r1};
     float best_v[2] = {best.v0, best.v1};
     int32_t best_i[2] = {best.i0, best.i1};
@@ -271,7 +273,7 @@ __device__ __noinline__ GemvBest gemv_epilogue(const GemvArgs& a, int64_t tile, 
             const float val = v[2 * h + e];
             switch (a.op) {
             case VOX_EP_RESIDUAL:
-                yr[row] = a.res[(int64_t)mt * a.ldr + row] + val;
+                yr[row] = (use_pre ? prv[2 * h + e] : a.res[(int64_t)mt * a.ldr + row]) + val;
                 break;
             case VOX_EP_GELU:
                 yr[row] = gelu_erf(val);
@@ -478,7 +480,7 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
                     if (lane == 0) s_ptile[warp] = (int32_t)tile;
                 } else if (cin == kc) {
                     best = gemv_epilogue(a, tile, make_float4(acc[0], acc[1], acc[2], acc[3]), g, t, rr[0], rr[1],
-                                         pos, best);
+                                         pos, best, make_float4(0.f, 0.f, 0.f, 0.f), 0);
                 } else {
                     tacc[0] = acc[0]; tacc[1] = acc[1]; tacc[2] = acc[2]; tacc[3] = acc[3];
                     tail_tile = tile;
@@ -546,7 +548,21 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
         }
     }
 
-    // ---- tiles cut between warps: the warp that started one adds the later pieces in warp order
+    // ---- tiles cut between warps: the warp that started one adds the later pieces in warp order;
+    // its residual values are loaded before the barrier, off the tail's critical path
+    float4 tres = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tail_tile >= 0 && a.op == VOX_EP_RESIDUAL) {
+        float rv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int64_t row = tail_tile * 16 + g + 8 * h;
+                const int mt = 2 * t + e;
+                if (row < a.n && mt < m) rv[2 * h + e] = a.res[(int64_t)mt * a.ldr + row];
+            }
+        tres = make_float4(rv[0], rv[1], rv[2], rv[3]);
+    }
     __syncthreads();
     if (tail_tile >= 0) {
         const int64_t last_rec = tail_tile * kc + kc - 1;
@@ -558,7 +574,7 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
             tacc[0] += pv.x; tacc[1] += pv.y; tacc[2] += pv.z; tacc[3] += pv.w;
         }
         best = gemv_epilogue(a, tail_tile, make_float4(tacc[0], tacc[1], tacc[2], tacc[3]), g, t, rr[0], rr[1], pos,
-                             best);
+                             best, tres, a.op == VOX_EP_RESIDUAL);
     }
 
     // ---- greedy argmax: warps -> CTA -> one 64-bit atomic max per token; the

@@ -417,7 +417,8 @@ def test_window_attention_short_history(env):
 
 # ------------------------------------------------------------------- GEMM
 @pytest.mark.parametrize("n,k,m", [(256, 128, 16), (1280, 1280, 256), (3840, 1280, 256), (1280, 5120, 256),
-                                   (3072, 5120, 64), (130, 320, 37), (6144, 3072, 16), (5120, 1280, 100)])
+                                   (3072, 5120, 64), (130, 320, 37), (6144, 3072, 16), (5120, 1280, 100),
+                                   (48, 192, 20)])
 def test_gemm_parity(env, n, k, m):
     torch, V, WL = env
     qs, d = synth.q4_blocks(n, k, 0, 12000 + n + k)
