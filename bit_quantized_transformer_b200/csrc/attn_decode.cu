@@ -520,16 +520,10 @@ vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc
     a.stages = env_int_attn("VOX_ATTN_STAGES", 3, 2, kAttnMaxStages);
     const AttnSmem SL = attn_smem_layout(a.stages);
 
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gqa_decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)attn_smem_layout(kAttnMaxStages).total);
-        if (e != cudaSuccess) {
-            set_cuda_error(e);
-            return VOX_ERR_CUDA;
-        }
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    st = smem_attr_per_device(reinterpret_cast<const void*>(gqa_decode_attn_kernel),
+                              (int)attn_smem_layout(kAttnMaxStages).total, attr_done);
+    if (st != VOX_OK) return st;
     const int64_t G = attn_grid(n_kv, window);
     st = launch_pdl(gqa_decode_attn_kernel, dim3((unsigned)G), dim3(kAttnThreads), SL.total, s, kmap, vmap, a);
     if (st != VOX_OK) return st;

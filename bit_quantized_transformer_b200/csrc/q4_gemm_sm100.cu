@@ -286,15 +286,9 @@ static vox_status launch_gemm_bn(const GemmArgs& a, const void* x, int64_t ldx, 
     st = make_tmap_2d(&wmap, a.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)a.kc * (kChunkBytes / 4),
                       (uint64_t)a.tiles, (uint64_t)a.kc * kChunkBytes, kChunkBytes / 4, 8, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != VOX_OK) return st;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(q4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem);
-        if (e != cudaSuccess) {
-            set_cuda_error(e);
-            return VOX_ERR_CUDA;
-        }
-        attr = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    st = smem_attr_per_device(reinterpret_cast<const void*>(q4_gemm_kernel<BN>), C::smem, attr_done);
+    if (st != VOX_OK) return st;
     dim3 grid((unsigned)ceil_div(a.tiles, 8), (unsigned)ceil_div(a.m, BN));
     return launch_pdl(q4_gemm_kernel<BN>, grid, dim3(kGemmThreads), (size_t)C::smem, s, xmap, wmap, a);
 }

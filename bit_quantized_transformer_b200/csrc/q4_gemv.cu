@@ -663,17 +663,11 @@ vox_status launch_q4_gemv(const uint8_t* w, int64_t n, int64_t k, const float* x
     a.pre = env_int("VOX_GEMV_PREFETCH", 1, 0, stages);
 
     void (*kern)(GemvArgs) = m == 1 ? q4_gemv_kernel<1> : q4_gemv_kernel<8>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(q4_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(q4_gemv_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) {
-            set_cuda_error(e);
-            return VOX_ERR_CUDA;
-        }
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> attr_done1{0}, attr_done8{0};
+    vox_status st = smem_attr_per_device(reinterpret_cast<const void*>(q4_gemv_kernel<1>), 227 * 1024, attr_done1);
+    if (st == VOX_OK)
+        st = smem_attr_per_device(reinterpret_cast<const void*>(q4_gemv_kernel<8>), 227 * 1024, attr_done8);
+    if (st != VOX_OK) return st;
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemvThreads, L.total);
     if (e != cudaSuccess || per_sm < 1) {

@@ -8,6 +8,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "vox.h"
 
 namespace vox {
@@ -28,6 +30,29 @@ void set_cuda_error(cudaError_t e);
 void set_error_text(const char* text);      // message for vox_last_error
 vox_status check_launch();                  // cudaGetLastError -> VOX_ERR_CUDA
 int device_sm_count();                      // SMs of the current device (cached per device)
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per device (function attributes belong to a device context,
+// so a process that drives several devices sets each one).  `done` is the
+// call site's bitmask of devices already set.
+inline vox_status smem_attr_per_device(const void* kernel, int bytes, std::atomic<unsigned long long>& done)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_cuda_error(e);
+        return VOX_ERR_CUDA;
+    }
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return VOX_OK;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) {
+        set_cuda_error(e);
+        return VOX_ERR_CUDA;
+    }
+    if (bit) done.fetch_or(bit, std::memory_order_release);
+    return VOX_OK;
+}
 
 // Launch a kernel with the programmatic-dependent-launch attribute so that it
 // may start while the previous kernel on the stream drains; the kernel itself
