@@ -542,8 +542,17 @@ vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc
 // loaded module, and its address is looked up once per device.
 constexpr int kStaticMaxKv = 8;
 constexpr int kStaticMaxGroup = 4;
+
+// Records of all heads for the largest n_kv * rmax(n_kv) over n_kv = 1..8
+// (the per-head record count rounds up, so 7 heads need one more than 8).
+constexpr int attn_static_max_records(int n)
+{
+    return n == 0 ? 0
+                  : (n * attn_rmax(n) > attn_static_max_records(n - 1) ? n * attn_rmax(n)
+                                                                        : attn_static_max_records(n - 1));
+}
 constexpr size_t kStaticScratchBytes =
-    (size_t)kStaticMaxKv * attn_rmax(kStaticMaxKv) * attn_rec_floats(kStaticMaxGroup, kAttnHd) * sizeof(float);
+    (size_t)attn_static_max_records(kStaticMaxKv) * attn_rec_floats(kStaticMaxGroup, kAttnHd) * sizeof(float);
 
 static __device__ __align__(256) uint8_t g_attn_static_scratch[kStaticScratchBytes];
 

@@ -58,6 +58,26 @@ def test_static_scratch_matches_workspace_entry(env):
         assert err <= TOL, (call, err)
 
 
+def test_static_scratch_takes_every_documented_shape(env):
+    """Every kv head count up to 8 with groups up to 4 fits the array (a
+    small window, so each call is quick); 16 kv heads or groups of 8 do not."""
+    torch, V, WL = env
+    W, hd = 64, 128
+    c = torch.zeros(8, W, hd, dtype=torch.bfloat16, device="cuda")
+    for n_kv in range(1, 9):
+        for group in (1, 2, 4):
+            q = torch.zeros(n_kv * group, hd, device="cuda")
+            out = torch.empty(n_kv * group, hd, device="cuda")
+            V.vox_gqa_decode_attn_static(q, c, c, out, n_kv * group, n_kv, hd, W, 10, 0.1)
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    q = torch.zeros(64, hd, device="cuda")
+    out = torch.empty(64, hd, device="cuda")
+    st = V.lib.vox_gqa_decode_attn_static(q.data_ptr(), c.data_ptr(), c.data_ptr(), out.data_ptr(), 64, 8, hd, W,
+                                          10, 0.1, None)
+    assert st == V.VOX_ERR_RANGE
+
+
 def test_static_scratch_rejects_shapes_beyond_its_size(env):
     torch, V, WL = env
     q = torch.zeros(64, 128, device="cuda")
