@@ -7,8 +7,11 @@
 // heads).  Readings: slot = pos mod W, the valid slots after writing pos are
 // the first min(pos + 1, W); query head h reads kv head h / (n_q / n_kv).
 //
-// K4 design: the valid (kv head, 64-slot chunk) pairs are split evenly over
-// the CTAs (stream-K), so every CTA streams the same number of cache bytes.
+// K4 design: one 160-thread CTA per SM by default (a TMA producer warp and
+// four consumer warps; tuning knobs VOX_ATTN_CTAS_PER_SM and VOX_ATTN_STAGES,
+// three ring stages of 32 KB by default).  The valid (kv head, 64-slot chunk)
+// pairs are split evenly over the CTAs (stream-K), so every CTA streams the
+// same number of cache bytes.
 // A producer lane loads each chunk's K and V with 2-D TMA tiles (128-byte
 // swizzle, 4 x 8 KB) into a shared-memory ring; four consumer warps each take
 // 16 slots of the chunk:

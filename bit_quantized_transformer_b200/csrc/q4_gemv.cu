@@ -14,24 +14,32 @@
 //    pieces of the following warps in warp order from shared memory:
 //    deterministic, and no CTA ever waits for another.
 //  * Data movement: each warp streams its range through its own ring of
-//    shared-memory stages, one bulk (TMA) copy of two 576-byte records per
-//    stage, completing on a per-stage mbarrier.  The first stages are issued
-//    before griddepcontrol.wait, as weights never depend on upstream kernels;
-//    bytes in flight cost no registers.
+//    shared-memory stages (three by default), one bulk (TMA) copy of four
+//    576-byte records per stage, completing on a per-stage mbarrier.  One
+//    stage is issued before griddepcontrol.wait (weights never depend on
+//    upstream kernels), the others once the activations are in, so the
+//    activation loads do not queue behind a full ring; bytes in flight cost
+//    no registers.
 //  * Dequantisation: each 32-bit word of codes gives four half2 A-fragment
 //    registers with one LOP3 each (OR the nibble into the fraction of 1024.0
 //    or 64.0, whose ulp is 1 at that nibble position: exact 1024+q / 64+q).
-//    The constant offsets are removed through the MMAs' C inputs, preloaded
-//    with -1032 * sum x_lo and -72 * sum x_hi per block.
+//    The MMAs start from zero; the constant offsets come back as one
+//    per-block correction, -(1032 * sum x_lo + 72 * sum x_hi), added to the
+//    MMA result before the scale.
 //  * Tensor cores: mma.sync m16n8k16 fp16 x fp16 -> fp32, the low- and
-//    high-nibble halves of a block as two independent MMAs, and the two
-//    records of a stage issued back to back, so the MMA latency overlaps.
+//    high-nibble halves of a block chained, and the four records of a stage
+//    issued back to back before any bookkeeping, so the MMA latency
+//    overlaps.  A stage with no tile end and no range end takes a fast path
+//    (pairwise sum of the four records, no per-record checks).
 //  * Activations: each 32-column block of x (times the RMSNorm weight) is
 //    scaled by its own exact power of two into [2^13, 2^14) before the fp16
 //    conversion, and the block's inverse scale is folded into its d in fp32.
 //    No row statistic is needed before the main loop: the RMSNorm factor
 //    multiplies the finished dot products in the epilogue.  The prologue is
 //    one round of loads and one CTA barrier.
+//  * Build knobs (tuning, not semantics): VOX_GEMV_WARPS, VOX_GEMV_RECS,
+//    VOX_GEMV_MIN_CTAS, VOX_GEMV_BATCH at compile time; VOX_GEMV_STAGES,
+//    VOX_GEMV_PREFETCH and VOX_GEMV_CTAS_PER_SM in the environment.
 #include "vox_internal.cuh"
 
 #include <stdlib.h>
