@@ -159,6 +159,27 @@ def test_kv_and_attention_validation(V):
     assert a(kc=FAKE + 2) == V.VOX_ERR_ALIGN
 
 
+def test_static_attention_validation(V):
+    """The no-workspace entry point rejects bad arguments, and shapes its
+    fixed scratch cannot hold, on the host (no device call happens first)."""
+    L = V.lib
+    s = lambda nq=32, nkv=8, hd=128, W=8192, pos=0, kc=FAKE: L.vox_gqa_decode_attn_static(
+        FAKE, kc, FAKE, FAKE, nq, nkv, hd, W, pos, 0.088, None)
+    assert s(kc=None) == V.VOX_ERR_NULL
+    assert s(nq=30) == V.VOX_ERR_RANGE
+    assert s(pos=-1) == V.VOX_ERR_RANGE
+    assert s(W=0) == V.VOX_ERR_RANGE
+    assert s(hd=64) == V.VOX_ERR_SHAPE
+    assert s(kc=FAKE + 2) == V.VOX_ERR_ALIGN
+    assert s(nq=64, nkv=16) == V.VOX_ERR_RANGE          # more kv heads than the scratch holds
+    assert b"static scratch" in L.vox_last_error()
+    assert s(nq=64, nkv=8) == V.VOX_ERR_RANGE           # groups of 8 > 4
+    # seven kv heads pass the head / group limits and stop at the alignment
+    # check, still before any device call (the scratch size itself is checked
+    # on the GPU by the static-scratch test)
+    assert s(nq=28, nkv=7, kc=FAKE + 2) == V.VOX_ERR_ALIGN
+
+
 def test_window_attn_and_rmsnorm_validation(V):
     L = V.lib
     w = lambda hd=40, W=750, nq=256, ldq=3840, od=V.VOX_BF16, q=FAKE: L.vox_window_attn(
