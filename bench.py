@@ -402,8 +402,9 @@ def graph_of(fn):
 
 
 def run_encoder(args):
-    """Config 3: the 32-layer encoder chunk (M = 256 rows, dim 1280) plus the
-    adapter GEMM, and the same chunk's Q4_0 GEMMs alone (K2, tcgen05)."""
+    """The 32-layer encoder chunk (M = 256 rows, dim 1280, 32 heads x 40,
+    window 750) plus the 5120 -> 3072 adapter GEMM at 64 rows, and the same
+    chunk's Q4_0 GEMMs alone (K2, tcgen05)."""
     import torch
 
     import synth
@@ -463,7 +464,7 @@ def run_encoder(args):
 
 
 def run_sweep(args):
-    """Config 4: the decoder projection shapes at M in {1,4,16,64,256} (K1 for
+    """The decoder projection shapes at M in {1,4,16,64,256} (K1 for
     M <= 8, K2 for M >= 16, and K1 as two M = 8 launches at M = 16 for the
     crossover), over weight copies totalling > 2x L2; then the decode
     attention at KV 512, 4096 and 8192 (wrapped)."""
