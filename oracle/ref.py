@@ -29,8 +29,11 @@ Definitions followed (page titles as on the pages):
   R10.
 * LM head + greedy argmax, lowest index on ties (R11).
 
-parity unpinned: the composed decoder step and encoder chunk as wholes (no
-published logits exist); each is only the composition of pinned functions.
+One decoder layer and one encoder layer are pinned by closed forms of
+special cases (zero or identity projections, a single visible key).  The
+26-layer step and the 32-layer chunk as wholes are only the composition of
+those pinned layers: beyond that they are parity unpinned (no published
+logits exist).
 """
 from __future__ import annotations
 

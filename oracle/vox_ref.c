@@ -190,8 +190,7 @@ void vr_kv_append(uint16_t *k_cache, uint16_t *v_cache, const float *k_new, cons
 /* GQA decode attention over the rolling cache after position pos was written.
  * Valid slots: 0 .. min(pos+1, W)-1 (R6).  Query head h reads kv head
  * h / (n_q / n_kv) (R7).  s_j = scale * q.k_j, p = softmax(s), o = sum p_j v_j.
- * Also returns, per head, the softmax row maximum and normaliser so the
- * split-KV combine can be checked. */
+ * Only o is returned; the split-KV partials are a NumPy-side reference. */
 void vr_gqa_attn(const float *q /* [n_q][hd] */, const uint16_t *k_cache, const uint16_t *v_cache,
                  int n_q, int n_kv, int hd, int64_t window, int64_t pos, double scale,
                  double *out /* [n_q][hd] */)

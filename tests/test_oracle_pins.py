@@ -138,6 +138,157 @@ def pin_attention_list_model(attn, configs):
                 np.testing.assert_allclose(got[h], want, rtol=1e-12, atol=1e-12)
 
 
+# ------------------------------------------- error metric and composed pins
+def pin_gemv_error(metric):
+    """The normalised GEMV error, worked by hand.  x = (3, 4) has norm 5; the
+    rows w0 = (3, 4) and w1 = (0, 2) have norms 5 and 2 (their columns have
+    norms 3 and sqrt(20), so a row/column slip changes the value)."""
+    x = np.array([[3.0, 4.0]])
+    W = np.array([[3.0, 4.0], [0.0, 2.0]])
+    y_ref = np.array([[25.0, 8.0]])
+    # errors 0.5 on both outputs: 0.5 / (5 * 5) = 0.02 and 0.5 / (5 * 2) = 0.05
+    assert metric(y_ref + 0.5, y_ref, x, W) == 0.05
+    # a second activation row (0, 1), norm 1: an error of -0.3 on output 1
+    # gives 0.3 / (1 * 2) = 0.15, larger than row 0's 0.05
+    x2 = np.array([[3.0, 4.0], [0.0, 1.0]])
+    y2_ref = np.array([[25.0, 8.0], [4.0, 2.0]])
+    y2 = y2_ref + np.array([[0.5, 0.5], [0.0, -0.3]])
+    assert metric(y2, y2_ref, x2, W) == pytest.approx(0.15, rel=1e-15)
+    assert metric(y2_ref, y2_ref, x2, W) == 0.0
+
+
+def pin_attn_error(metric):
+    """The normalised attention error, worked by hand: two kv heads of two
+    valid slots and head_dim 2, group 1.  Head 0: p = (0.6, 0.8) (norm 1),
+    V = [[3, 1], [4, 0]] (columns of norms 5 and 1).  Head 1: p = (1, 0),
+    V = [[0, 2], [0, 0]] (column norms 0 and 2)."""
+    probs = np.array([[0.6, 0.8], [1.0, 0.0]])
+    Vv = np.array([[[3.0, 1.0], [4.0, 0.0]], [[0.0, 2.0], [0.0, 0.0]]])
+    o_ref = np.array([[5.0, 0.6], [0.0, 2.0]])
+    # head 0 errors (0.5, 0.1): 0.5/5 = 0.1, 0.1/1 = 0.1; head 1 error 0.5 on dim 1: 0.5/2 = 0.25
+    o = o_ref + np.array([[0.5, 0.1], [0.0, 0.5]])
+    assert metric(o, o_ref, probs, Vv, 1) == 0.25
+    o = o_ref + np.array([[0.5, -0.3], [0.0, 0.0]])
+    assert metric(o, o_ref, probs, Vv, 1) == pytest.approx(0.3, rel=1e-15)
+    # group 2: both query heads read kv head 0
+    o2_ref = np.array([[5.0, 0.6], [5.0, 0.6]])
+    o2 = o2_ref + np.array([[0.0, 0.0], [1.0, 0.0]])
+    assert metric(o2, o2_ref, np.array([[0.6, 0.8], [0.6, 0.8]]), Vv, 2) == pytest.approx(0.2, rel=1e-15)
+
+
+def pin_attn_probs(probs):
+    """Softmax probabilities of hand-built keys: with scale 1/2, q = (2, 0) and
+    keys (1, 0), (0, 1) the scores are 1 and 0, so p = (e, 1) / (1 + e); one
+    valid key gives p = 1; the second kv head (keys (0, 1), (1, 0)) swaps them."""
+    one, zero = 0x3F80, 0x0000                      # bf16 1.0 and 0.0
+    kc = np.array([[[one, zero], [zero, one], [one, one]],
+                   [[zero, one], [one, zero], [one, one]]], np.uint16)   # n_kv 2, W 3, hd 2
+    q = np.array([[2.0, 0.0], [2.0, 0.0]], np.float32)
+    e = math.e
+    P = probs(q, kc, 1, 0.5)                         # positions 0 and 1 written
+    np.testing.assert_allclose(P, [[e / (1 + e), 1 / (1 + e)], [1 / (1 + e), e / (1 + e)]], rtol=1e-15)
+    assert np.array_equal(probs(q, kc, 0, 0.5), np.ones((2, 1)))
+    # wrapped (pos 7 >= W): all three slots, scores (1, 0, 1) and (0, 1, 1)
+    P = probs(q, kc, 7, 0.5)
+    np.testing.assert_allclose(P[0], np.array([e, 1.0, e]) / (2 * e + 1), rtol=1e-15)
+    np.testing.assert_allclose(P[1], np.array([1.0, e, e]) / (2 * e + 1), rtol=1e-15)
+
+
+def _bf16_round(v):
+    """bf16 (nearest-even) of float32 values by torch's CPU cast, widened back."""
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(np.asarray(v, np.float32))).to(torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+def pin_decoder_layer(layer):
+    """Closed forms of one decoder layer (dim 4, 4 query / 2 kv heads of
+    head_dim 1, FFN 4, window 3) in special cases:
+    (a) Wo = W2 = 0: out = h = x exactly, at any position;
+    (b) position 0 (one valid key): o of query head h is the stored (bf16)
+        v of kv head h // 2;
+    (c) Wo = I, W2 = 0 at position 0: out = x + o, the residual is x;
+    (d) Wq = Wk = 0, Wv picks column 0, Wo = I, W1 = 2I, W3 = 3I, W2 = I:
+        out_i = h_i + silu(2 n2_i) * 3 n2_i with n2 = RMSNorm(h), h = x + o."""
+    rng = np.random.default_rng(21)
+    D, nq, nkv, W = 4, 4, 2, 3
+    eps = ref.RMS_EPS
+    x = np.array([1.5, -0.5, 2.0, -1.0])
+    Z = np.zeros((D, D))
+    I = np.eye(D)
+
+    def weights(**kw):
+        w = {"wq": rng.standard_normal((nq, D)), "wk": rng.standard_normal((nkv, D)),
+             "wv": rng.standard_normal((nkv, D)), "wo": rng.standard_normal((D, nq)),
+             "w1": rng.standard_normal((D, D)), "w3": rng.standard_normal((D, D)),
+             "w2": rng.standard_normal((D, D))}
+        w.update(kw)
+        return w
+
+    def caches():
+        return (synth_bf16((nkv, W, 1), 1), synth_bf16((nkv, W, 1), 2))
+
+    # (a)
+    for pos in (0, 1, 5):
+        kc, vc = caches()
+        st = layer(x, weights(wo=np.zeros((D, nq)), w2=Z), kc, vc, pos, nq, nkv)
+        assert np.array_equal(st["out"], x) and np.array_equal(st["h"], x)
+    # (b) and (c)
+    kc, vc = caches()
+    w = weights(wo=np.eye(D, nq), w2=Z)
+    st = layer(x, w, kc, vc, 0, nq, nkv)
+    n = x / math.sqrt(float(np.mean(x * x)) + eps)
+    v_stored = _bf16_round(w["wv"] @ n)
+    assert np.array_equal(st["o"], v_stored[[0, 0, 1, 1]])
+    assert np.array_equal(st["out"], x + v_stored[[0, 0, 1, 1]])
+    # (d)
+    kc, vc = caches()
+    wv = np.zeros((nkv, D)); wv[:, 0] = 1.0
+    st = layer(x, weights(wq=np.zeros((nq, D)), wk=np.zeros((nkv, D)), wv=wv, wo=np.eye(D, nq),
+                          w1=2 * I, w3=3 * I, w2=I), kc, vc, 0, nq, nkv)
+    o = float(_bf16_round([x[0] / math.sqrt(float(np.mean(x * x)) + eps)])[0])
+    h = x + o
+    r = 1.0 / math.sqrt(sum(v * v for v in h) / D + eps)
+    want = [hi + (2 * hi * r) / (1 + math.exp(-2 * hi * r)) * 3 * hi * r for hi in h]
+    np.testing.assert_allclose(st["out"], want, rtol=1e-14)
+
+
+def synth_bf16(shape, tid):
+    import synth
+
+    return synth.bf16_normal(shape, 0, tid)
+
+
+def pin_encoder_layer(layer):
+    """Closed forms of one encoder layer (3 rows, dim 2, 2 heads of head_dim 1,
+    FFN 2, 2 history rows):
+    (a) Wo = Wdown = 0: out = X exactly;
+    (b) window 1 (a row sees only itself), Wqkv = [0; 0; I] (v = RMSNorm(X)),
+        Wo = I, Wdown = 0: out = X + RMSNorm(X);
+    (c) Wo = 0, Wup = 1.5 I, Wdown = 2 I: out = X + 2 gelu(1.5 RMSNorm(X))."""
+    rng = np.random.default_rng(22)
+    X = np.array([[1.0, -2.0], [0.5, 0.25], [-3.0, 1.0]])
+    D, eps = 2, ref.RMS_EPS
+    kh, vh = rng.standard_normal((2, D)), rng.standard_normal((2, D))
+    Z = np.zeros((D, D))
+
+    def weights(**kw):
+        w = {"wqkv": rng.standard_normal((3 * D, D)), "wo": rng.standard_normal((D, D)),
+             "wup": rng.standard_normal((D, D)), "wdown": rng.standard_normal((D, D))}
+        w.update(kw)
+        return w
+
+    n = np.array([[v / math.sqrt((row[0] ** 2 + row[1] ** 2) / D + eps) for v in row] for row in X])
+    assert np.array_equal(layer(X, weights(wo=Z, wdown=Z), kh, vh, 3, 2, 1), X)
+    wqkv = np.zeros((3 * D, D)); wqkv[2 * D:] = np.eye(D)
+    out = layer(X, weights(wqkv=wqkv, wo=np.eye(D), wdown=Z), kh, vh, 1, 2, 1)
+    np.testing.assert_allclose(out, X + n, rtol=1e-14)
+    out = layer(X, weights(wo=Z, wup=1.5 * np.eye(D), wdown=2 * np.eye(D)), kh, vh, 3, 2, 1)
+    g = np.array([[1.5 * v * (1 + math.erf(1.5 * v / math.sqrt(2))) for v in row] for row in n])
+    np.testing.assert_allclose(out, X + g, rtol=1e-14)
+
+
 # ------------------------------------------------------------------- tests
 def test_half_decode_all_patterns(oracle_c):
     """The C oracle's hand-written fp16 decode equals numpy's cast on all 65536 patterns."""
@@ -337,6 +488,33 @@ def test_rmsnorm_silu_gelu_closed_forms():
     assert abs(ref.gelu(40.0) - 40.0) < 1e-12
 
 
+def test_error_metrics_by_hand():
+    pin_gemv_error(ref.gemv_error)
+    pin_attn_error(ref.attn_error)
+
+
+def test_attention_probabilities_by_hand():
+    pin_attn_probs(ref.attn_probs)
+
+
+def test_bf16_widening_matches_torch():
+    """bf16 -> float64 widening equals torch's bf16 -> fp32 cast on all 65536 patterns."""
+    import torch
+
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    want = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float32).numpy()
+    with np.errstate(invalid="ignore"):               # NaN patterns widen to NaN
+        assert same_bits_or_nan(ref.bf16_to_f64(bits), want.astype(np.float64))
+
+
+def test_decoder_layer_closed_forms():
+    pin_decoder_layer(ref.decoder_layer)
+
+
+def test_encoder_layer_closed_forms():
+    pin_encoder_layer(ref.encoder_layer)
+
+
 def test_window_attention_bruteforce():
     """Encoder sliding window: query i (position q0+i) sees j with p-W < j <= p."""
     rng = np.random.default_rng(9)
@@ -445,3 +623,95 @@ def test_planted_mistakes_are_caught():
 
     with pytest.raises(AssertionError):
         pin_attention_list_model(attn_wrong_group, [(4, 2, 8, 5)])
+
+
+def test_planted_mistakes_in_metric_and_layers_are_caught():
+    """Slips in the error metric, the probabilities and the composed layers fail a pin."""
+    def metric_column_norms(y, y_ref, x, w):         # norms of W's columns, not its rows
+        return ref.gemv_error(y, y_ref, x, np.asarray(w).T)
+
+    def metric_squared_x(y, y_ref, x, w):
+        x = np.atleast_2d(np.asarray(x, np.float64))
+        return ref.gemv_error(y, y_ref, x * np.linalg.norm(x, axis=1, keepdims=True), w)
+
+    def metric_mean(y, y_ref, x, w):
+        y, y_ref = np.atleast_2d(y), np.atleast_2d(y_ref)
+        xn = np.linalg.norm(np.atleast_2d(x), axis=1)[:, None]
+        wn = np.linalg.norm(w, axis=1)[None, :]
+        return float(np.mean(np.abs(y - y_ref) / (xn * wn)))
+
+    for bad in (metric_column_norms, metric_squared_x, metric_mean):
+        with pytest.raises(AssertionError):
+            pin_gemv_error(bad)
+
+    def attn_metric_row_norms(o, o_ref, probs, Vv, group):   # norms over slots of a dim, swapped
+        return ref.attn_error(o, o_ref, probs, np.swapaxes(Vv, 1, 2), group)
+
+    def attn_metric_wrong_group(o, o_ref, probs, Vv, group):
+        return ref.attn_error(o, o_ref, probs, Vv[::-1], group)
+
+    for bad in (attn_metric_row_norms, attn_metric_wrong_group):
+        with pytest.raises(AssertionError):
+            pin_attn_error(bad)
+
+    def probs_no_scale(q, kc, pos, scale=None):
+        return ref.attn_probs(q, kc, pos, 1.0)
+
+    def probs_sign(q, kc, pos, scale=None):
+        return ref.attn_probs(-np.asarray(q), kc, pos, scale)
+
+    def probs_drop_newest(q, kc, pos, scale=None):
+        return ref.attn_probs(q, kc, max(pos - 1, 0), scale)
+
+    for bad in (probs_no_scale, probs_sign, probs_drop_newest):
+        with pytest.raises(AssertionError):
+            pin_attn_probs(bad)
+
+    def layer_residual_from_norm(x, Wd, kc, vc, pos, nq, nkv, eps=ref.RMS_EPS):
+        st = ref.decoder_layer(x, Wd, kc, vc, pos, nq, nkv, eps)
+        h = st["n"] + Wd["wo"] @ st["o"]
+        st["h"] = h
+        st["out"] = h + Wd["w2"] @ (ref.silu(Wd["w1"] @ ref.rmsnorm(h)) * (Wd["w3"] @ ref.rmsnorm(h)))
+        return st
+
+    def layer_ffn_from_first_norm(x, Wd, kc, vc, pos, nq, nkv, eps=ref.RMS_EPS):
+        st = ref.decoder_layer(x, Wd, kc, vc, pos, nq, nkv, eps)
+        st["out"] = st["h"] + Wd["w2"] @ (ref.silu(Wd["w1"] @ st["n"]) * (Wd["w3"] @ st["n"]))
+        return st
+
+    def layer_gate_on_up(x, Wd, kc, vc, pos, nq, nkv, eps=ref.RMS_EPS):
+        st = ref.decoder_layer(x, Wd, kc, vc, pos, nq, nkv, eps)
+        st["out"] = st["h"] + Wd["w2"] @ ((Wd["w1"] @ st["n2"]) * ref.silu(Wd["w3"] @ st["n2"]))
+        return st
+
+    def layer_interleaved_gqa(x, Wd, kc, vc, pos, nq, nkv, eps=ref.RMS_EPS):
+        st = ref.decoder_layer(x, Wd, kc, vc, pos, nq, nkv, eps)
+        hd = kc.shape[2]
+        q = st["q"].reshape(nq, hd)
+        o = np.stack([ref.gqa_attn(q[h:h + 1], kc[h % nkv:h % nkv + 1], vc[h % nkv:h % nkv + 1], pos)[0]
+                      for h in range(nq)]).reshape(-1)
+        st["o"] = o
+        st["h"] = x + Wd["wo"] @ o
+        n2 = ref.rmsnorm(st["h"])
+        st["out"] = st["h"] + Wd["w2"] @ (ref.silu(Wd["w1"] @ n2) * (Wd["w3"] @ n2))
+        return st
+
+    for bad in (layer_residual_from_norm, layer_ffn_from_first_norm, layer_gate_on_up, layer_interleaved_gqa):
+        with pytest.raises(AssertionError):
+            pin_decoder_layer(bad)
+
+    def enc_residual_from_norm(X, Wd, kh, vh, window, nh, hd, eps=ref.RMS_EPS):
+        return ref.encoder_layer(X, Wd, kh, vh, window, nh, hd, eps) - np.asarray(X) + ref.rmsnorm(X)
+
+    def enc_gelu_after_down(X, Wd, kh, vh, window, nh, hd, eps=ref.RMS_EPS):
+        W2 = dict(Wd)
+        W2["wdown"] = np.zeros_like(Wd["wdown"])
+        h = ref.encoder_layer(X, W2, kh, vh, window, nh, hd, eps)
+        return h + ref.gelu((ref.rmsnorm(h) @ Wd["wup"].T) @ Wd["wdown"].T)
+
+    def enc_window_one_wider(X, Wd, kh, vh, window, nh, hd, eps=ref.RMS_EPS):
+        return ref.encoder_layer(X, Wd, kh, vh, window + 1, nh, hd, eps)
+
+    for bad in (enc_residual_from_norm, enc_gelu_after_down, enc_window_one_wider):
+        with pytest.raises(AssertionError):
+            pin_encoder_layer(bad)
