@@ -55,10 +55,15 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
-    p.add_argument("--workload", choices=["decoder", "encoder", "sweep"], default="decoder",
+    p.add_argument("--workload", choices=["decoder", "encoder", "sweep", "kernel"], default="decoder",
                    help="decoder: the headline line (default); encoder: the 32-layer encoder chunk at M=256 "
                         "and its GEMMs; sweep: the decoder shapes at M in {1,4,16,64,256} and the attention at "
-                        "KV in {512, 4096, 8192 wrapped}")
+                        "KV in {512, 4096, 8192 wrapped}; kernel: a few launches of one kernel on one small "
+                        "case (--kernel, --shape, --launches), sized for an ncu capture")
+    p.add_argument("--kernel", choices=["gemv", "attn", "gemm"], default="gemv",
+                   help="kernel workload: gemv N K (M = 1), attn POS (decoder-shaped layer), gemm N K M")
+    p.add_argument("--shape", type=int, nargs="*", default=None)
+    p.add_argument("--launches", type=int, default=4)
     return p.parse_args(argv)
 
 
@@ -555,6 +560,65 @@ def run_sweep(args):
     return 0
 
 
+def run_kernel_case(args):
+    """A few launches of one kernel on one case that holds well under 1 GB on
+    the device (seeded synthetic inputs as in the decoder workload), for an
+    ncu capture; checks the device status word and prints one JSON line.
+      gemv N K   : the Q4_0 GEMV, M = 1, no epilogue, on one packed N x K weight
+      attn POS   : split-KV decode attention, 32 query / 8 kv heads x 128,
+                   8192-slot bf16 rolling cache, after position POS was written
+      gemm N K M : the Q4_0 GEMM (tcgen05), M bf16 activation rows, bf16 output"""
+    import math
+
+    import torch
+
+    import synth
+    from bit_quantized_transformer_b200 import build
+
+    build.build()
+    from bit_quantized_transformer_b200 import vox as V
+    from bit_quantized_transformer_b200 import workloads as WL
+
+    shp = args.shape or {"gemv": [4096, 3072], "attn": [8492], "gemm": [131072, 3072, 256]}[args.kernel]
+    if args.kernel == "gemv":
+        n, k = shp[0], shp[1]
+        qs, d = synth.q4_blocks(n, k, 0, 77)
+        packed, w = WL.pack_q4(qs, d, "cuda")
+        x = WL.to_dev(synth.activations(1, k, 0, 78), "cuda")
+        y = torch.empty(1, n, device="cuda")
+        wsb = V.vox_q4_gemv_workspace(w, 1, None)
+        ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+        for _ in range(args.launches):
+            V.vox_q4_gemv(w, x, 1, k, y, n, None, ws, wsb)
+        what = {"kernel": "q4_gemv_kernel", "n": n, "k": k, "weight_bytes_per_launch": packed.numel()}
+    elif args.kernel == "gemm":
+        n, k, m = shp[0], shp[1], shp[2]
+        qs, d = synth.q4_blocks(n, k, 0, 79)
+        packed, w = WL.pack_q4(qs, d, "cuda")
+        x = WL.bf16_dev(synth.bf16_normal((m, k), 0, 80), "cuda")
+        y = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+        for _ in range(args.launches):
+            V.vox_q4_gemm(w, x, V.VOX_BF16, m, k, y, V.VOX_BF16, n)
+        what = {"kernel": "q4_gemm_kernel", "n": n, "k": k, "m": m, "flop_per_launch": 2 * m * n * k}
+    else:
+        pos = shp[0]
+        n_q, n_kv, hd, W = 32, 8, 128, 8192
+        kc = torch.randn(n_kv, W, hd, device="cuda").to(torch.bfloat16)
+        vc = torch.randn(n_kv, W, hd, device="cuda").to(torch.bfloat16)
+        q = torch.randn(n_q, hd, device="cuda")
+        out = torch.empty(n_q, hd, device="cuda")
+        wsb = V.vox_gqa_decode_attn_workspace(n_q, n_kv, hd, W)
+        ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+        for _ in range(args.launches):
+            V.vox_gqa_decode_attn(q, kc, vc, out, n_q, n_kv, hd, W, pos, 1.0 / math.sqrt(hd), ws, wsb)
+        what = {"kernel": "gqa_decode_attn_kernel", "pos": pos,
+                "cache_bytes_per_launch": 2 * n_kv * min(pos + 1, W) * hd * 2}
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    print(json.dumps({"workload": "kernel case", "launches": args.launches, **what}), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
@@ -563,6 +627,8 @@ def main(argv=None):
         return run_encoder(args)
     if args.workload == "sweep":
         return run_sweep(args)
+    if args.workload == "kernel":
+        return run_kernel_case(args)
     return run_ours(args)
 
 

@@ -202,7 +202,7 @@ vox_status vox_gqa_decode_attn(const float* q, const void* k_cache, const void* 
     if ((int64_t)n_kv_heads * window > 0x7fffff00LL) return VOX_ERR_SHAPE;
     if (!workspace) return VOX_ERR_WORKSPACE;
     if (ws_bytes < vox_gqa_decode_attn_workspace(n_q_heads, n_kv_heads, head_dim, window)) return VOX_ERR_WORKSPACE;
-    if (!al16(k_cache) || !al16(v_cache) || !al16(workspace)) return VOX_ERR_ALIGN;
+    if (!al16(k_cache) || !al16(v_cache) || !al16(workspace) || !al16(out)) return VOX_ERR_ALIGN;
     return launch_gqa_decode_attn(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_dim, window, pos, nullptr,
                                   scale, workspace, S(stream));
 }

@@ -560,11 +560,17 @@ constexpr size_t kStaticScratchBytes =
 static __device__ __align__(256) uint8_t g_attn_static_scratch[kStaticScratchBytes];
 
 // Device address of the scratch array on the current device, looked up with
-// cudaGetSymbolAddress the first time each device is used and kept.
+// cudaGetSymbolAddress the first time each device is used and kept for the
+// life of the process.  Later calls read the kept address with one atomic
+// load and take no lock; only a first lookup takes the mutex.  The address
+// belongs to the device's primary context: after cudaDeviceReset (or any
+// teardown that unloads this module from the device) the kept address is
+// stale, so a process that resets a device must not call this entry point
+// again on it without reloading the library.
 static vox_status attn_static_scratch(void** out)
 {
     static std::mutex mu;
-    static void* addr[64];
+    static std::atomic<void*> addr[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) {
@@ -572,17 +578,20 @@ static vox_status attn_static_scratch(void** out)
         return VOX_ERR_CUDA;
     }
     if (dev < 0 || dev >= 64) return VOX_ERR_RANGE;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_attn_static_scratch);
-        if (e != cudaSuccess) {
-            set_cuda_error(e);
-            return VOX_ERR_CUDA;
+    void* p = addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(mu);
+        p = addr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            e = cudaGetSymbolAddress(&p, g_attn_static_scratch);
+            if (e != cudaSuccess) {
+                set_cuda_error(e);
+                return VOX_ERR_CUDA;
+            }
+            addr[dev].store(p, std::memory_order_release);
         }
-        addr[dev] = p;
     }
-    *out = addr[dev];
+    *out = p;
     return VOX_OK;
 }
 
@@ -604,7 +613,8 @@ extern "C" vox_status vox_gqa_decode_attn_static(const float* q, const void* k_c
                        "at most 4 query heads; use vox_gqa_decode_attn with a workspace");
         return VOX_ERR_RANGE;
     }
-    if (((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15u) != 0)
+    if (((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache) |
+          reinterpret_cast<uintptr_t>(out)) & 15u) != 0)
         return VOX_ERR_ALIGN;
     // the records this call writes: n_kv runs of rmax records of the group's size
     const size_t need = (size_t)n_kv_heads * attn_rmax(n_kv_heads) * attn_rec_floats(group, kAttnHd) * sizeof(float);

@@ -183,6 +183,8 @@ vox_status vox_encoder_chunk(const vox_encoder* e, void* stream)
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const float scale = 1.0f / sqrtf((float)e->head_dim);
     for (int l = 0; l < e->n_layers; ++l) {
+        const bool tap = e->tap && l == e->n_layers - 1;
+        if (tap && (st = launch_cast_rows(e->x, R, D, D, e->tap, VOX_F32, D, s))) return st;
         if ((st = launch_rmsnorm(e->x, R, D, D, e->eps, nullptr, e->xn, VOX_BF16, D, s))) return st;
         if ((st = launch_q4_gemm(static_cast<const uint8_t*>(e->wqkv[l].data), 3 * D, D, e->xn, R, D, e->qkv,
                                  VOX_BF16, 3 * D, nullptr, s)))
@@ -198,6 +200,7 @@ vox_status vox_encoder_chunk(const vox_encoder* e, void* stream)
         if ((st = launch_q4_gemm(static_cast<const uint8_t*>(e->wo[l].data), D, D, e->att, R, D, e->x, VOX_F32, D, &r,
                                  s)))
             return st;
+        if (tap && (st = launch_cast_rows(e->x, R, D, D, e->tap + R * D, VOX_F32, D, s))) return st;
         if ((st = launch_rmsnorm(e->x, R, D, D, e->eps, nullptr, e->xn, VOX_BF16, D, s))) return st;
         vox_epilogue gl = {};
         gl.op = VOX_EP_GELU;

@@ -63,7 +63,8 @@ class vox_encoder(ctypes.Structure):
                 ("wup", ctypes.POINTER(vox_q4_weight)), ("wdown", ctypes.POINTER(vox_q4_weight)),
                 ("adapter", vox_q4_weight),
                 ("k_hist", ctypes.POINTER(_P)), ("v_hist", ctypes.POINTER(_P)),
-                ("x", _P), ("xn", _P), ("qkv", _P), ("att", _P), ("up", _P), ("adapter_out_buf", _P)]
+                ("x", _P), ("xn", _P), ("qkv", _P), ("att", _P), ("up", _P), ("adapter_out_buf", _P),
+                ("tap", _P)]
 
 
 _W = ctypes.POINTER(vox_q4_weight)

@@ -184,7 +184,8 @@ class DecoderModel:
 class EncoderModel:
     """Synthetic encoder chunk: rows x dim input, per-layer history caches, adapter."""
 
-    def __init__(self, shape: synth.EncoderShape, seed: int = 0, device="cuda", n_layers=None, eps: float = 1e-5):
+    def __init__(self, shape: synth.EncoderShape, seed: int = 0, device="cuda", n_layers=None, eps: float = 1e-5,
+                 tap: bool = False):
         self.shape = shape
         self.L = shape.n_layers if n_layers is None else n_layers
         D, F, R = shape.dim, shape.ffn, shape.rows
@@ -226,6 +227,9 @@ class EncoderModel:
         for name in ("x", "xn", "qkv", "att", "up"):
             setattr(e, name, getattr(self, name).data_ptr())
         e.adapter_out_buf = self.out.data_ptr()
+        # the last layer's input and mid-layer residual, for per-kernel checks of that layer
+        self.tap = torch.zeros(2, R, D, dtype=torch.float32, device=device) if tap else None
+        e.tap = self.tap.data_ptr() if tap else None
         self.enc = e
         self.adapter = ad
 

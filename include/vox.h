@@ -206,7 +206,8 @@ vox_status vox_kv_append_rolling(void *k_cache, void *v_cache, const void *k_new
  * reads kv head h / (n_q_heads / n_kv_heads); s_j = scale * q_h . k_j over the
  * valid slots j < min(pos + 1, window); out_h = softmax(s) . V.  q: device fp32
  * [n_q_heads][head_dim]; caches: device bf16 [n_kv_heads][window][head_dim],
- * 16-byte aligned; out: device fp32 [n_q_heads][head_dim].  Split-KV: slot
+ * 16-byte aligned; out: device fp32 [n_q_heads][head_dim], 16-byte aligned
+ * (it is written with 16-byte stores).  Split-KV: slot
  * ranges are reduced independently into the workspace (device, at least
  * vox_gqa_decode_attn_workspace() bytes, 16-byte aligned, no initial contents
  * needed) and merged by a log-sum-exp combine (a second, small kernel).
@@ -214,8 +215,8 @@ vox_status vox_kv_append_rolling(void *k_cache, void *v_cache, const void *k_new
  * 128 (the decoder's).
  * Errors: NULL -> VOX_ERR_NULL; pos < 0, window <= 0, n_q % n_kv != 0, a
  * group above 8 or more than 512 kv heads -> VOX_ERR_RANGE; other head_dim
- * -> VOX_ERR_SHAPE; short workspace -> VOX_ERR_WORKSPACE; caches or workspace
- * not 16-byte aligned -> VOX_ERR_ALIGN. */
+ * -> VOX_ERR_SHAPE; short workspace -> VOX_ERR_WORKSPACE; caches, out or
+ * workspace not 16-byte aligned -> VOX_ERR_ALIGN. */
 vox_status vox_gqa_decode_attn(const float *q, const void *k_cache, const void *v_cache, float *out,
                                int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                                int32_t window, int64_t pos, float scale,
@@ -239,7 +240,10 @@ size_t vox_gqa_decode_attn_workspace(int32_t n_q_heads, int32_t n_kv_heads, int3
  * GPU (other streams, concurrent graph replays) corrupt each other's
  * results: order them on one stream.  The first call on each device looks
  * the array's address up (cudaGetSymbolAddress); make that call outside any
- * stream capture.  Other errors as vox_gqa_decode_attn. */
+ * stream capture.  The address is kept for the life of the process: after
+ * cudaDeviceReset on a device, reload the library before calling this entry
+ * point on that device again.  Other errors (out not 16-byte aligned ->
+ * VOX_ERR_ALIGN included) as vox_gqa_decode_attn. */
 vox_status vox_gqa_decode_attn_static(const float *q, const void *k_cache, const void *v_cache,
                                       float *out, int32_t n_q_heads, int32_t n_kv_heads,
                                       int32_t head_dim, int32_t window, int64_t pos, float scale,
@@ -313,6 +317,10 @@ typedef struct {
     void *att;                   /* device bf16 [rows][dim] scratch                     */
     void *up;                    /* device bf16 [rows][ffn] scratch                     */
     float *adapter_out_buf;      /* device fp32 [rows/4][adapter_out]                   */
+    float *tap;                  /* device fp32 [2][rows][dim], or NULL: receives the last
+                                    layer's input x (tap[0]) and its residual stream h
+                                    after attention (tap[1]), so that layer can be checked
+                                    on its own inputs                                   */
 } vox_encoder;
 
 /* One encoder chunk: 32 x {RMSNorm, QKV GEMM, window attention, O GEMM +

@@ -157,6 +157,10 @@ def test_kv_and_attention_validation(V):
     assert a(wsp=None) == V.VOX_ERR_WORKSPACE
     assert a(wsb=ws - 16) == V.VOX_ERR_WORKSPACE
     assert a(kc=FAKE + 2) == V.VOX_ERR_ALIGN
+    assert L.vox_gqa_decode_attn(FAKE, FAKE, FAKE, FAKE + 4, 32, 8, 128, 8192, 0, 0.088, FAKE, ws,
+                                 None) == V.VOX_ERR_ALIGN
+    assert L.vox_gqa_decode_attn(FAKE, FAKE, FAKE, FAKE + 8, 32, 8, 128, 8192, 0, 0.088, FAKE, ws,
+                                 None) == V.VOX_ERR_ALIGN
 
 
 def test_static_attention_validation(V):
@@ -171,6 +175,9 @@ def test_static_attention_validation(V):
     assert s(W=0) == V.VOX_ERR_RANGE
     assert s(hd=64) == V.VOX_ERR_SHAPE
     assert s(kc=FAKE + 2) == V.VOX_ERR_ALIGN
+    for off in (4, 8):                                  # out is written with 16-byte stores
+        assert L.vox_gqa_decode_attn_static(FAKE, FAKE, FAKE, FAKE + off, 32, 8, 128, 8192, 0, 0.088,
+                                            None) == V.VOX_ERR_ALIGN
     assert s(nq=64, nkv=16) == V.VOX_ERR_RANGE          # more kv heads than the scratch holds
     assert b"static scratch" in L.vox_last_error()
     assert s(nq=64, nkv=8) == V.VOX_ERR_RANGE           # groups of 8 > 4

@@ -6,7 +6,9 @@ forcing, so errors do not compound), at the benchmark's full sizes.
 * the full 26-layer step with the cache filled to 8192 + 300 (wrapped): the
   last layer's attention, FFN and residual, the LM head on sampled rows and
   the argmax;
-* one encoder layer + the adapter GEMM at M = 256.
+* one encoder layer + the adapter GEMM at M = 256, and the last layer of the
+  full 32-layer chunk, each kernel on that layer's own inputs (a tap of the
+  layer's input and mid-layer residual).
 """
 import math
 
@@ -186,23 +188,21 @@ def test_decoder_step_graph_replay_matches_eager(env):
         assert torch.equal(a.k_cache[l].view(torch.int16), b.k_cache[l].view(torch.int16))
 
 
-def test_encoder_layer_and_adapter(env):
-    torch, V, WL = env
-    shape = synth.EncoderShape()
-    em = WL.EncoderModel(shape, seed=0, n_layers=1)
-    em.run()
-    torch.cuda.synchronize()
-    assert V.vox_device_status(True) == 0
+def check_encoder_layer(shape, em, layer, seed):
+    """Every kernel of encoder layer `layer` on the GPU's own inputs to it:
+    the tap holds the layer's input x and its residual h after attention; the
+    qkv / att / up buffers and x hold that layer's values after the call."""
     D, F, R, nh, hd = shape.dim, shape.ffn, shape.rows, shape.n_heads, shape.head_dim
-    w = synth.encoder_layer_weights(shape, 0, 0)
-    x0 = synth.activations(R, D, 0, synth.ENC_X_ID)
+    w = synth.encoder_layer_weights(shape, layer, seed)
+    tap = np_of(em.tap).astype(np.float64)
+    x_in, h = tap[0], tap[1]
     qkv_b = bits(em.qkv)
-    # QKV GEMM on bf16(RMSNorm(x0))
-    xn = ref.bf16_to_f64(ref.f32_to_bf16(ref.rmsnorm(x0).astype(np.float32)))
+    # QKV GEMM on bf16(RMSNorm(x_in)); the output is stored as bf16
+    xn = ref.bf16_to_f64(ref.f32_to_bf16(ref.rmsnorm(x_in).astype(np.float32)))
     err = gemv_err(ref.bf16_to_f64(qkv_b), xn, *w["wqkv"])
-    assert err <= TOL, err
+    assert err <= TOL, ("qkv", err)
     # window attention on the GPU's q, k, v and the history
-    kh, vh = synth.encoder_layer_history(shape, 0, 0)
+    kh, vh = synth.encoder_layer_history(shape, layer, seed)
     Q = ref.bf16_to_f64(qkv_b[:, :D])
     K = np.concatenate([ref.bf16_to_f64(kh), ref.bf16_to_f64(qkv_b[:, D:2 * D])])
     Vv = np.concatenate([ref.bf16_to_f64(vh), ref.bf16_to_f64(qkv_b[:, 2 * D:])])
@@ -213,25 +213,58 @@ def test_encoder_layer_and_adapter(env):
     for ii, i in enumerate(rows):
         p = shape.window + i
         lo = p - shape.window + 1
-        for h in range(nh):
-            sl = slice(h * hd, (h + 1) * hd)
-            s = (K[lo:p + 1, sl] @ Q[i, sl]) / math.sqrt(hd)
-            pr = np.exp(s - s.max()); pr /= pr.sum()
+        for hh in range(nh):
+            sl = slice(hh * hd, (hh + 1) * hd)
+            sc = (K[lo:p + 1, sl] @ Q[i, sl]) / math.sqrt(hd)
+            pr = np.exp(sc - sc.max()); pr /= pr.sum()
             den = np.linalg.norm(pr) * np.linalg.norm(Vv[lo:p + 1, sl], axis=0)
-            assert np.max(np.abs(att[i, sl] - att_ref[ii, sl]) / den) <= TOL
-    # h = x0 + Wo att and x1 = h + Wdown up, checked through h = x1 - Wdown up
+            assert np.max(np.abs(att[i, sl] - att_ref[ii, sl]) / den) <= TOL, ("attention", i, hh)
+    # O GEMM + residual: h = x_in + Wo att
+    err_o = gemv_err(h - x_in, att, *w["wo"])
+    assert err_o <= TOL, ("o", err_o)
+    # up GEMM + GELU on bf16(RMSNorm(h)), stored as bf16
     up = ref.bf16_to_f64(bits(em.up))
-    x1 = np_of(em.x).astype(np.float64)
-    h_est = x1 - up @ ref.q4_weights(*w["wdown"]).T
-    err_o = gemv_err(h_est - x0, att, *w["wo"])
-    err_dn = ref.gemv_error(x1 - h_est, up @ ref.q4_weights(*w["wdown"]).T, up, ref.q4_weights(*w["wdown"]))
-    assert err_o <= 2 * TOL, err_o
-    assert err_dn <= TOL
-    n2 = ref.bf16_to_f64(ref.f32_to_bf16(ref.rmsnorm(h_est).astype(np.float32)))
+    n2 = ref.bf16_to_f64(ref.f32_to_bf16(ref.rmsnorm(h).astype(np.float32)))
     Wup = ref.q4_weights(*w["wup"])
-    assert ref.gemv_error(up, ref.gelu(n2 @ Wup.T), n2, Wup) <= 2 * TOL
+    err_up = ref.gemv_error(up, ref.gelu(n2 @ Wup.T), n2, Wup)
+    assert err_up <= TOL, ("up", err_up)
+    # down GEMM + residual: x_out = h + Wdown up
+    x_out = np_of(em.x).astype(np.float64)
+    err_dn = gemv_err(x_out - h, up, *w["wdown"])
+    assert err_dn <= TOL, ("down", err_dn)
+    return x_out
+
+
+def test_encoder_layer_and_adapter(env):
+    torch, V, WL = env
+    shape = synth.EncoderShape()
+    em = WL.EncoderModel(shape, seed=0, n_layers=1, tap=True)
+    em.run()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    D, R = shape.dim, shape.rows
+    x0 = synth.activations(R, D, 0, synth.ENC_X_ID)
+    assert np.array_equal(np_of(em.tap[0]), x0)                 # layer 0's input is the chunk input
+    x1 = check_encoder_layer(shape, em, 0, 0)
     # adapter on the downsampled bf16 rows of x1
     aq, ad = synth.q4_blocks(shape.adapter_out, 4 * D, 0, synth.ADAPTER_ID)
     xd = ref.downsample_rows(ref.bf16_to_f64(ref.f32_to_bf16(x1.astype(np.float32))), 4)
+    err_ad = gemv_err(np_of(em.out), xd, aq, ad)
+    assert err_ad <= TOL, err_ad
+
+
+def test_encoder_chunk_last_layer(env):
+    """The full 32-layer chunk that the bench times: its last layer checked
+    kernel by kernel on that layer's own GPU inputs, and the adapter."""
+    torch, V, WL = env
+    shape = synth.EncoderShape()
+    em = WL.EncoderModel(shape, seed=0, tap=True)
+    em.run()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    x_out = check_encoder_layer(shape, em, shape.n_layers - 1, 0)
+    assert np.all(np.isfinite(x_out))
+    aq, ad = synth.q4_blocks(shape.adapter_out, 4 * shape.dim, 0, synth.ADAPTER_ID)
+    xd = ref.downsample_rows(ref.bf16_to_f64(ref.f32_to_bf16(x_out.astype(np.float32))), 4)
     err_ad = gemv_err(np_of(em.out), xd, aq, ad)
     assert err_ad <= TOL, err_ad

@@ -1,9 +1,23 @@
-"""vox_gqa_decode_attn_static, the entry point that allocates nothing, against
-vox_gqa_decode_attn with a caller workspace: the same decoder-shaped inputs
-(32 query / 8 kv heads x 128, 8192-slot rolling cache), two calls in a row at
-different positions (the second after the window has wrapped), each within
-the attention tolerance of the workspace entry point's output.  The file
-sorts last so that it also runs after every other GPU test."""
+"""vox_gqa_decode_attn_static, the entry point that allocates nothing.
+
+It serves callers that cannot hand the library device scratch (a host
+program that links only this C library and owns no device allocator; a
+real-time audio thread that must not call cudaMalloc, which can block and
+synchronise the device).  Its split-KV records live in one fixed array inside
+the loaded library.  These tests call it through the C ABI and check:
+
+* on the decoder's shape (32 query / 8 kv heads x 128, 8192-slot rolling
+  cache), two calls in a row at different positions (the second after the
+  window has wrapped): the output equals the workspace entry point's bit for
+  bit (same kernels, same grid, deterministic combine) and is within the
+  attention tolerance of the fp64 oracle;
+* every documented shape (1..8 kv heads, groups of 1, 2 and 4) on seeded
+  random caches, against the workspace entry point (bit for bit) and the
+  oracle, including 7 kv heads x 4 at the full 8192-slot window, the shape
+  that needs the most records;
+* shapes beyond the array are refused with VOX_ERR_RANGE.
+
+The file sorts last so that it also runs after every other GPU test."""
 import math
 
 import numpy as np
@@ -31,51 +45,60 @@ def env():
     return torch, V, WL
 
 
-def test_static_scratch_matches_workspace_entry(env):
+def run_both(env, q, kb, vb, n_q, n_kv, W, pos):
+    """Static and workspace entry points on the same inputs; the workspace
+    starts filled with 0xFF bytes (its contract needs no initial contents)."""
     torch, V, WL = env
+    hd = 128
+    kc, vc = WL.bf16_dev(kb, "cuda"), WL.bf16_dev(vb, "cuda")
+    qd = WL.to_dev(q, "cuda")
+    wsb = V.vox_gqa_decode_attn_workspace(n_q, n_kv, hd, W)
+    ws = torch.full((wsb,), 0xFF, dtype=torch.uint8, device="cuda")
+    out_ws = torch.full((n_q, hd), float("nan"), device="cuda")
+    out_st = torch.full((n_q, hd), float("nan"), device="cuda")
+    scale = 1.0 / math.sqrt(hd)
+    V.vox_gqa_decode_attn(qd, kc, vc, out_ws, n_q, n_kv, hd, W, pos, scale, ws, wsb)
+    V.vox_gqa_decode_attn_static(qd, kc, vc, out_st, n_q, n_kv, hd, W, pos, scale)
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    return out_st.cpu().numpy(), out_ws.cpu().numpy()
+
+
+def oracle_err(o, q, kb, vb, n_q, n_kv, W, pos):
+    nv = min(pos + 1, W)
+    o_ref = ref.c_gqa_attn(q, kb, vb, pos)
+    return ref.attn_error(o, o_ref, ref.attn_probs(q, kb, pos), ref.bf16_to_f64(vb[:, :nv]), n_q // n_kv)
+
+
+def test_static_scratch_matches_workspace_entry(env):
     n_q, n_kv, hd, W = 32, 8, 128, 8192
     kb = synth.bf16_normal((n_kv, W, hd), 0, 61)
     vb = synth.bf16_normal((n_kv, W, hd), 0, 62)
-    kc, vc = WL.bf16_dev(kb, "cuda"), WL.bf16_dev(vb, "cuda")
-    wsb = V.vox_gqa_decode_attn_workspace(n_q, n_kv, hd, W)
-    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
-    scale = 1.0 / math.sqrt(hd)
     for call, pos in enumerate((1500, W + 300)):
         q = synth.activations(n_q, hd, 0, 63 + call) * 2.0
-        qd = WL.to_dev(q, "cuda")
-        out_ws = torch.empty(n_q, hd, device="cuda")
-        out_st = torch.full((n_q, hd), float("nan"), device="cuda")
-        V.vox_gqa_decode_attn(qd, kc, vc, out_ws, n_q, n_kv, hd, W, pos, scale, ws, wsb)
-        V.vox_gqa_decode_attn_static(qd, kc, vc, out_st, n_q, n_kv, hd, W, pos, scale)
-        torch.cuda.synchronize()
-        assert V.vox_device_status(True) == 0
-        o_ws = out_ws.cpu().numpy()
-        o_st = out_st.cpu().numpy()
+        o_st, o_ws = run_both(env, q, kb, vb, n_q, n_kv, W, pos)
         assert np.all(np.isfinite(o_st))
-        nv = min(pos + 1, W)
-        err = ref.attn_error(o_st, o_ws.astype(np.float64), ref.attn_probs(q, kb, pos),
-                             ref.bf16_to_f64(vb[:, :nv]), n_q // n_kv)
+        assert np.array_equal(o_st.view(np.uint32), o_ws.view(np.uint32)), call
+        err = oracle_err(o_st, q, kb, vb, n_q, n_kv, W, pos)
         assert err <= TOL, (call, err)
 
 
 def test_static_scratch_takes_every_documented_shape(env):
-    """Every kv head count up to 8 with groups up to 4 fits the array (a
-    small window, so each call is quick); 16 kv heads or groups of 8 do not."""
-    torch, V, WL = env
-    W, hd = 64, 128
-    c = torch.zeros(8, W, hd, dtype=torch.bfloat16, device="cuda")
-    for n_kv in range(1, 9):
-        for group in (1, 2, 4):
-            q = torch.zeros(n_kv * group, hd, device="cuda")
-            out = torch.empty(n_kv * group, hd, device="cuda")
-            V.vox_gqa_decode_attn_static(q, c, c, out, n_kv * group, n_kv, hd, W, 10, 0.1)
-    torch.cuda.synchronize()
-    assert V.vox_device_status(True) == 0
-    q = torch.zeros(64, hd, device="cuda")
-    out = torch.empty(64, hd, device="cuda")
-    st = V.lib.vox_gqa_decode_attn_static(q.data_ptr(), c.data_ptr(), c.data_ptr(), out.data_ptr(), 64, 8, hd, W,
-                                          10, 0.1, None)
-    assert st == V.VOX_ERR_RANGE
+    """Every kv head count up to 8 with groups up to 4 fits the array and
+    gives the workspace entry point's output bit for bit, within the oracle's
+    tolerance; 7 kv heads x 4 also at the full window."""
+    cases = [(n_kv, group, 1024, 1500) for n_kv in range(1, 9) for group in (1, 2, 4)]
+    cases.append((7, 4, 8192, 8192 + 300))
+    for n_kv, group, W, pos in cases:
+        n_q = n_kv * group
+        tid = 700 + 4 * (n_kv * 8 + group) + (W > 1024)
+        kb = synth.bf16_normal((n_kv, W, 128), 0, tid)
+        vb = synth.bf16_normal((n_kv, W, 128), 0, tid + 1)
+        q = synth.activations(n_q, 128, 0, tid + 2)
+        o_st, o_ws = run_both(env, q, kb, vb, n_q, n_kv, W, pos)
+        assert np.array_equal(o_st.view(np.uint32), o_ws.view(np.uint32)), (n_kv, group, W)
+        err = oracle_err(o_st, q, kb, vb, n_q, n_kv, W, pos)
+        assert err <= TOL, (n_kv, group, W, err)
 
 
 def test_static_scratch_rejects_shapes_beyond_its_size(env):
@@ -83,7 +106,8 @@ def test_static_scratch_rejects_shapes_beyond_its_size(env):
     q = torch.zeros(64, 128, device="cuda")
     c = torch.zeros(16, 64, 128, dtype=torch.bfloat16, device="cuda")
     out = torch.empty(64, 128, device="cuda")
-    st = V.lib.vox_gqa_decode_attn_static(q.data_ptr(), c.data_ptr(), c.data_ptr(), out.data_ptr(), 64, 16, 128,
-                                          64, 10, 0.1, None)
-    assert st == V.VOX_ERR_RANGE
-    assert b"static scratch" in V.lib.vox_last_error()
+    for n_q, n_kv in ((64, 16), (64, 8)):            # 16 kv heads; groups of 8
+        st = V.lib.vox_gqa_decode_attn_static(q.data_ptr(), c.data_ptr(), c.data_ptr(), out.data_ptr(), n_q, n_kv,
+                                              128, 64, 10, 0.1, None)
+        assert st == V.VOX_ERR_RANGE
+        assert b"static scratch" in V.lib.vox_last_error()
