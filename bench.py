@@ -27,9 +27,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -40,11 +38,10 @@ METRIC = "Q4_0 GEMV weight GB/s (% of HBM peak); 26-layer decoder ms/step on 1 B
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 FILLED = 8192 + 300
-# dram bytes (read + write) per launch of the dominant kernel, from ncu captures
-# of the current Q4_0 GEMV on each decoder shape weighted by the step's launch
-# mix (the GEMV summary under profiles/); set to None when the kernel changes,
-# until it is captured again
-GEMV_TRAFFIC_BYTES_PER_LAUNCH = 18_535_412
+# dram bytes (read + write) per launch of the dominant kernel (the persistent
+# step) from an ncu capture of the current kernel (profiles/); None until the
+# kernel as it stands has been captured
+STEP_TRAFFIC_BYTES_PER_LAUNCH = None
 
 
 def parse_args(argv=None):
@@ -55,8 +52,10 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
-    p.add_argument("--workload", choices=["decoder", "encoder", "sweep", "kernel"], default="decoder",
-                   help="decoder: the headline line (default); encoder: the 32-layer encoder chunk at M=256 "
+    p.add_argument("--workload", choices=["decoder", "gemv", "layer", "encoder", "sweep", "kernel"],
+                   default="decoder",
+                   help="decoder: the headline line (default); gemv: the single 4096x3072 GEMV; layer: one "
+                        "decoder layer at KV 1024; encoder: the 32-layer encoder chunk at M=256 "
                         "and its GEMMs; sweep: the decoder shapes at M in {1,4,16,64,256} and the attention at "
                         "KV in {512, 4096, 8192 wrapped}; kernel: a few launches of one kernel on one small "
                         "case (--kernel, --shape, --launches), sized for an ncu capture")
@@ -79,52 +78,74 @@ def measured_peaks():
 
 # ------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampled every 200 ms during the timed region."""
+    """SM clock and throttle reasons of this rank's GPU, read through NVML
+    (read-only queries) every `period_s` by a background thread during the
+    timed region; short regions still get samples."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    def __init__(self, torch_device: int, period_s: float = 0.002):
+        self.dev = torch_device
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.err = None
+        self._stop = None
+        self._thr = None
+
+    def _handle(self, nv):
+        import torch
+
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.dev)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
-        os.close(fd)
+        import threading
+
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", "-i", str(self.gpu)],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            masks = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+        except Exception as e:                       # no NVML: report it, time anyway
+            self.err = f"nvml unavailable: {e}"
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    for name, m in masks:
+                        if r & m:
+                            self.reasons.add(name)
+                except Exception as e:
+                    self.err = str(e)
+                    return
+                self._stop.wait(self.period)
+
+        self._thr = threading.Thread(target=loop, daemon=True)
+        self._thr.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sms, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sms.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sms)}
+        if self._thr is not None:
+            self._stop.set()
+            self._thr.join(timeout=5)
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+               "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml, 2 ms period"}
+        if self.err:
+            out["error"] = self.err
+        return out
 
 
 # ------------------------------------------------------- distributed
@@ -183,7 +204,7 @@ def time_replays(g, n, world):
 
 
 # ------------------------------------------------------- CPU oracle
-def oracle_decoder_sample(budget_s: float, layers=None):
+def oracle_decoder_sample(budget_s: float, layers=None, filled=FILLED):
     """The oracle's decoder layer (C oracle matvec + attention, numpy norms) on
     the first `layers` (default 4) layers of the same workload, cycled until
     `budget_s` of CPU time is spent.  Returns (bytes processed, seconds,
@@ -205,8 +226,8 @@ def oracle_decoder_sample(budget_s: float, layers=None):
         n = ref.rmsnorm(x).astype(np.float32)
         qkv = np.concatenate([ref.c_matvec(*w[k], n)[0] for k in ("wq", "wk", "wv")])
         ref.c_kv_append(kc, vc, qkv[QD:QD + KVD].reshape(shape.n_kv_heads, -1),
-                        qkv[QD + KVD:].reshape(shape.n_kv_heads, -1), FILLED)
-        o = ref.c_gqa_attn(qkv[:QD].reshape(shape.n_q_heads, -1).astype(np.float32), kc, vc, FILLED).reshape(-1)
+                        qkv[QD + KVD:].reshape(shape.n_kv_heads, -1), filled)
+        o = ref.c_gqa_attn(qkv[:QD].reshape(shape.n_q_heads, -1).astype(np.float32), kc, vc, filled).reshape(-1)
         h = x + ref.c_matvec(*w["wo"], o.astype(np.float32))[0]
         n2 = ref.rmsnorm(h).astype(np.float32)
         a = ref.silu(ref.c_matvec(*w["w1"], n2)[0]) * ref.c_matvec(*w["w3"], n2)[0]
@@ -214,7 +235,7 @@ def oracle_decoder_sample(budget_s: float, layers=None):
         t_tot += time.perf_counter() - t0
         done += 1
         nw = sum(v[0].shape[0] * v[0].shape[1] * 32 for v in w.values())
-        bytes_tot += nw * 18 // 32 + 2 * shape.n_kv_heads * min(FILLED + 1, shape.window) * shape.head_dim * 2
+        bytes_tot += nw * 18 // 32 + 2 * shape.n_kv_heads * min(filled + 1, shape.window) * shape.head_dim * 2
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return bytes_tot, t_tot, done, threads
 
@@ -266,7 +287,7 @@ def run_reference(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "decoder_step_q4_26L_kv8192wrapped_M1 (oracle row sample)", "l2": "n/a (host)"},
+            "config": decoder_config(shape, world),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -275,6 +296,37 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------- ours
+def try_graph(fn):
+    """Capture fn into a CUDA graph (after one warm-up call on a side stream);
+    None if the runtime refuses the capture."""
+    import torch
+
+    try:
+        return graph_of(fn)
+    except Exception:
+        torch.cuda.synchronize()
+        return None
+
+
+def time_fn(fn, n, world, stream=None):
+    """Device time of n calls of fn on the current stream, bracketed by a
+    barrier and a synchronize on both sides (CUDA events on the launching
+    stream)."""
+    import torch
+
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream() if stream is None else stream
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(n):
+        fn()
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    return e0.elapsed_time(e1)
+
+
 def run_ours(args):
     import torch
 
@@ -288,64 +340,71 @@ def run_ours(args):
         build.build()
     barrier(world)
     import synth
+    from bit_quantized_transformer_b200 import vox as V
     from bit_quantized_transformer_b200 import workloads as WL
 
     shape = synth.DecoderShape()
     dm = WL.DecoderModel(shape, seed=0, filled=FILLED, token=17)
-    g = dm.capture()
-    for _ in range(max(3, args.warmup)):
-        g.replay()
-    torch.cuda.synchronize()
     step_bytes = dm.weight_bytes() + dm.kv_bytes(FILLED)
+    assert step_bytes == sum(decoder_bytes(shape))
+    peak, peak_src = measured_peaks()
+
+    # the product: one persistent launch per token step, replayed from a CUDA
+    # graph when the runtime captures the cooperative launch, else launched
+    g = try_graph(dm.step)
+    step = g.replay if g is not None else dm.step
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0, "device status after warm-up"
 
     clocks = ClockSampler(local)
     clocks.start()
-    local_ms = time_replays(g, args.steps, world)
+    local_ms = time_fn(step, args.steps, world)
     clk = clocks.stop()
+    assert V.vox_device_status(True) == 0, "device status after the timed steps"
     max_ms, value = aggregate(local_ms, args.steps, step_bytes, world)
     ms_step = max_ms / args.steps
+    achieved = step_bytes / (local_ms / args.steps / 1e3) / 1e9
 
-    # dominant kernel: the step's 105 GEMV launches captured alone, same chaining
+    # the same step as the library's per-kernel launch sequence (159 launches), for comparison
+    gk = dm.capture(dm.step_kernels)
+    for _ in range(3):
+        gk.replay()
+    reps = max(10, min(200, args.steps))
+    ms_k = time_fn(gk.replay, reps, world) / reps
+    # the per-projection GEMV kernel (K1) and the split-KV attention kernel (K4) alone
     gg = dm.capture(dm.gemv_chain)
     for _ in range(3):
         gg.replay()
-    reps = max(20, min(400, args.steps // 4))
-    ms_g = time_replays(gg, reps, world)
-    launches = dm.gemv_chain_launches()
-    per_launch_bytes = dm.gemv_chain_bytes() / launches
-    per_launch_ms = ms_g / (reps * launches)
-    achieved = per_launch_bytes / (per_launch_ms / 1e3) / 1e9
-    peak, peak_src = measured_peaks()
-
-    # attention alone (reported beside the roofline)
+    ms_g = time_fn(gg.replay, reps, world) / reps
+    k1_gbs = dm.gemv_chain_bytes() / (ms_g / 1e3) / 1e9
     pos_now = int(dm.pos.item())
     ga = dm.capture(lambda: dm.attn_chain(pos_now))
     for _ in range(3):
         ga.replay()
-    ms_a = time_replays(ga, reps, world)
+    ms_a = time_fn(ga.replay, reps, world) / reps
     attn_bytes = dm.kv_bytes(pos_now)
-    attn_gbs = attn_bytes * reps / (ms_a / 1e3) / 1e9
 
-    # end to end through the Python API: token H2D, graph replay, token D2H
+    # end to end through the C ABI: every step copies the token from pinned
+    # host memory, calls vox_decoder_step (one launch) and reads the new token back
     e2e_steps = max(10, min(args.steps, 500))
     tok_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
     out_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
     tok_h[0] = 17
-    barrier(world)
-    torch.cuda.synchronize()
     s = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
-    for _ in range(e2e_steps):
+
+    def e2e_step():
         dm.token.copy_(tok_h, non_blocking=True)
-        g.replay()
+        V.vox_decoder_step(dm.dec, s)
         out_h.copy_(dm.token, non_blocking=True)
         s.synchronize()
-        tok_h[0] = out_h[0]                                   # the host feeds the next token back
-    e1.record(s)
-    torch.cuda.synchronize()
-    e2e_local = e0.elapsed_time(e1)
+        tok_h[0] = out_h[0]                                   # the host feeds the token back
+
+    e2e_step()
+    e2e_local = time_fn(e2e_step, e2e_steps, world)
     _, e2e_value = aggregate(e2e_local, e2e_steps, step_bytes, world)
+    assert V.vox_device_status(True) == 0, "device status after the end-to-end steps"
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -357,35 +416,58 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "q4_0 weights, fp16/bf16 tensor-core inputs, f32 accumulate",
             "data": "synthetic",
-            "config": {"workload": "decoder_step_q4_26L_kv8192wrapped_M1", "layers": shape.n_layers,
-                       "dim": shape.dim, "heads": "32q/8kv x 128", "ffn": shape.ffn, "vocab": shape.vocab,
-                       "kv_window": shape.window, "kv_filled": FILLED, "bytes_per_step": step_bytes,
-                       "weight_bytes_per_step": dm.weight_bytes(), "kv_bytes_per_step": dm.kv_bytes(FILLED),
-                       "l2": "inputs larger than L2 (2.8 GB per step, no flush)",
-                       "replicas": world, "graph": "one CUDA graph per step, PDL between kernels"},
-            "roofline": {"bound": "hbm", "kernel": "q4_gemv_kernel", "achieved": achieved, "peak": peak,
-                         "unit": "GB/s", "frac": achieved / peak, "traffic": GEMV_TRAFFIC_BYTES_PER_LAUNCH,
-                         "peak_source": peak_src, "launches_timed": reps * launches,
-                         "algorithmic_bytes_per_launch": per_launch_bytes,
-                         "avg_launch_us": per_launch_ms * 1e3},
-            "attention": {"kernel": "gqa_decode_attn_kernel+attn_combine_kernel", "gbs": attn_gbs,
-                          "frac": attn_gbs / peak, "bytes_per_step": attn_bytes,
-                          "us_per_layer": ms_a / reps / dm.L * 1e3},
+            "config": decoder_config(shape, world),
+            "launch": "one persistent cooperative launch per step" + (
+                ", replayed from a CUDA graph" if g is not None else ", launched directly"),
+            "roofline": {"bound": "hbm", "kernel": "decoder_step_kernel", "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": STEP_TRAFFIC_BYTES_PER_LAUNCH,
+                         "peak_source": peak_src, "launches_timed": args.steps,
+                         "algorithmic_bytes_per_launch": step_bytes, "avg_launch_us": local_ms / args.steps * 1e3,
+                         "note": "one launch is the whole token step, so the dominant kernel is the step"},
             "decoder_ms_per_step": ms_step,
             "hbm_frac_step": value / world / peak,
+            "kernel_sequence": {"api": "vox_decoder_step_kernels", "launches_per_step": dm.step_kernels_launches(),
+                                "ms_per_step": ms_k, "gbs": step_bytes / (ms_k / 1e3) / 1e9},
+            "k1_gemv": {"kernel": "q4_gemv_kernel", "launches": dm.gemv_chain_launches(),
+                        "us_per_launch": ms_g / dm.gemv_chain_launches() * 1e3, "gbs": k1_gbs,
+                        "frac": k1_gbs / peak},
+            "k4_attention": {"kernel": "gqa_decode_attn_kernel+attn_combine_kernel", "gbs":
+                             attn_bytes / (ms_a / 1e3) / 1e9, "us_per_layer": ms_a / dm.L * 1e3},
             "gpu_launches": dm.step_launches() * args.steps,
             "clocks": clk,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4,
-                    "ms_per_step": e2e_local / e2e_steps, "api": "DecoderModel graph replay via vox_decoder_step"},
+                    "ms_per_step": e2e_local / e2e_steps,
+                    "api": "vox_decoder_step through the C ABI each step, token H2D before and D2H after, "
+                           "host synchronised every step"},
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    del g, gg, ga
+    del g, gk, gg, ga
     if world > 1:
         import torch.distributed as dist
 
         dist.destroy_process_group()
     return 0
+
+
+def decoder_bytes(shape, filled=FILLED):
+    """Algorithmic bytes of one decoder step, from the shapes alone: packed
+    Q4_0 weights of every layer and the LM head, one embedding row, and the
+    bf16 K and V rows the attention reads after position `filled` is written."""
+    D, QD, KVD, F, V = shape.dim, shape.q_dim, shape.kv_dim, shape.ffn, shape.vocab
+    per_layer = (QD + 2 * KVD) * D + D * QD + 2 * F * D + D * F
+    weights = (shape.n_layers * per_layer + V * D + D) * 18 // 32
+    kv = shape.n_layers * 2 * shape.n_kv_heads * min(filled + 1, shape.window) * shape.head_dim * 2
+    return weights, kv
+
+
+def decoder_config(shape, world):
+    weights, kv = decoder_bytes(shape)
+    return {"workload": "decoder_step_q4_26L_kv8192wrapped_M1", "layers": shape.n_layers,
+            "dim": shape.dim, "heads": "32q/8kv x 128", "ffn": shape.ffn, "vocab": shape.vocab,
+            "kv_window": shape.window, "kv_filled": FILLED, "bytes_per_step": weights + kv,
+            "weight_bytes_per_step": weights, "kv_bytes_per_step": kv,
+            "l2": "inputs larger than L2 (2.8 GB per step, no flush)", "replicas": world}
 
 
 # ------------------------------------------------ supplementary workloads
@@ -560,6 +642,161 @@ def run_sweep(args):
     return 0
 
 
+def run_gemv(args):
+    """Config 0: the single Q4_0 GEMV, 4096 x 3072 at M = 1 (weights seed 0,
+    activation N(0, 1)), through vox_q4_gemv.  Timed two ways: a CUDA graph of
+    launches cycling over distinct weight copies that total more than 2x L2
+    (every launch streams weights that are not in L2), and single calls, each
+    after an L2 flush (a 256 MB write) between its CUDA events."""
+    import numpy as np
+    import torch
+
+    import synth
+    from bit_quantized_transformer_b200 import build
+
+    build.build()
+    from bit_quantized_transformer_b200 import vox as V
+    from bit_quantized_transformer_b200 import workloads as WL
+    from oracle import ref
+
+    n, k = 4096, 3072
+    qs, d = synth.q4_blocks(n, k, 0, synth.X_ID + 100)
+    xh = synth.activations(1, k, 0, synth.X_ID)
+    packed, w0 = WL.pack_q4(qs, d, "cuda")
+    nbytes = packed.numel()
+    copies = 40                                           # 40 x 7.08 MB = 283 MB > 2 x 126 MB
+    keep = [packed] + [packed.clone() for _ in range(copies - 1)]
+    ws_ = [V.weight(t, n, k) for t in keep]
+    x = WL.to_dev(xh, "cuda")
+    y = torch.empty(1, n, device="cuda")
+    wsb = V.vox_q4_gemv_workspace(w0, 1, None)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    V.vox_q4_gemv(w0, x, 1, k, y, n, None, ws, wsb)
+    torch.cuda.synchronize()
+    W = ref.q4_weights(qs, d)
+    err = ref.gemv_error(y.cpu().numpy(), xh.astype(np.float64) @ W.T, xh, W)
+    assert err <= 2e-3, err
+
+    def chain():
+        for w in ws_:
+            V.vox_q4_gemv(w, x, 1, k, y, n, None, ws, wsb)
+
+    g = graph_of(chain)
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    reps = max(3, args.steps)
+    clocks = ClockSampler(0)
+    clocks.start()
+    ms = time_fn(g.replay, reps, 1)
+    clk = clocks.stop()
+    us = ms / (reps * copies) * 1e3
+    gbs = nbytes / us / 1e3
+    # cold single calls: flush L2 with a 256 MB write, then time one launch
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    s = torch.cuda.current_stream()
+    cold = []
+    for i in range(max(5, min(args.steps, 50))):
+        flush.fill_(float(i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        V.vox_q4_gemv(ws_[i % copies], x, 1, k, y, n, None, ws, wsb)
+        e1.record(s)
+        torch.cuda.synchronize()
+        cold.append(e0.elapsed_time(e1) * 1e3)
+    cold_us = statistics.median(cold)
+    peak, peak_src = measured_peaks()
+    cpu = None
+    if not args.no_cpu_baseline:
+        t0 = time.perf_counter()
+        done = 0
+        while time.perf_counter() - t0 < min(args.cpu_seconds, 10.0):
+            ref.c_matvec(qs, d, xh)
+            done += 1
+        dt = time.perf_counter() - t0
+        cpu = {"value": done * nbytes / dt / 1e9, "unit": "GB/s", "cores": omp_threads(), "kind": "oracle",
+               "sample": f"{done} full 4096 x 3072 GEMVs (fp64 C oracle, OpenMP over rows) in {dt:.1f} s"}
+    line = {"metric": "Q4_0 GEMV weight GB/s, 4096 x 3072, M = 1", "value": gbs, "unit": "GB/s", "n_gpus": 1,
+            "steps": reps, "warmup": max(3, args.warmup), "ms_per_step": ms / reps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "q4_0 weights, fp16 tensor-core inputs, f32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": "q4_gemv_4096x3072_M1", "weight_bytes": nbytes, "copies": copies,
+                       "l2": "graph of launches over 40 weight copies (283 MB > 2x L2); cold calls after a 256 MB "
+                             "L2 flush"},
+            "roofline": {"bound": "hbm", "kernel": "q4_gemv_kernel", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                         "frac": gbs / peak, "traffic": None, "peak_source": peak_src,
+                         "avg_launch_us": us, "ideal_us": nbytes / peak / 1e3},
+            "cold_call": {"us": cold_us, "gbs": nbytes / cold_us / 1e3, "calls": len(cold)},
+            "parity_error": err, "gpu_launches": reps * copies, "clocks": clk, "cpu_baseline": cpu}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_layer(args):
+    """Config 1: one decoder layer at M = 1, KV length 1024 (each step writes
+    one more position and attends over 1025 keys), all Q4_0 weights drawn as in
+    config 0.  Four distinct layers (rotated, 279 MB > 2x L2) run as one
+    persistent step whose embedding table and LM head have 16 rows (27 KB,
+    under 0.1% of the step); the per-layer time is the step time / 4.  The
+    window is 1025 positions, already wrapped, so every step attends over
+    exactly 1025 keys."""
+    import torch
+
+    import synth
+    from bit_quantized_transformer_b200 import build
+
+    build.build()
+    from bit_quantized_transformer_b200 import vox as V
+    from bit_quantized_transformer_b200 import workloads as WL
+
+    shape = synth.DecoderShape(n_layers=4, vocab=16, window=1025)
+    dm = WL.DecoderModel(shape, seed=0, filled=2 * 1025, token=3)
+    wbytes, kv = decoder_bytes(shape, 2 * 1025)
+    layer_bytes = (wbytes - (shape.vocab * shape.dim + shape.dim) * 18 // 32 + kv) // shape.n_layers
+    step_bytes = wbytes + kv
+    g = try_graph(dm.step)
+    step = g.replay if g is not None else dm.step
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    reps = max(3, args.steps)
+    clocks = ClockSampler(0)
+    clocks.start()
+    ms = time_fn(step, reps, 1)
+    clk = clocks.stop()
+    assert V.vox_device_status(True) == 0
+    us_layer = ms / reps / shape.n_layers * 1e3
+    gbs = layer_bytes / us_layer / 1e3
+    gk = dm.capture(dm.step_kernels)
+    for _ in range(3):
+        gk.replay()
+    ms_k = time_fn(gk.replay, reps, 1) / reps
+    peak, peak_src = measured_peaks()
+    cpu = None
+    if not args.no_cpu_baseline:
+        b, t, n_done, threads = oracle_decoder_sample(min(args.cpu_seconds, 15.0), layers=4, filled=1024)
+        cpu = {"value": b / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n_done} decoder-layer passes at KV 1025 (fp64 C oracle), {b / 1e6:.1f} MB in {t:.1f} s"}
+    line = {"metric": "decoder layer GB/s (weights + KV), M = 1, KV 1024", "value": gbs, "unit": "GB/s",
+            "n_gpus": 1, "steps": reps, "warmup": max(3, args.warmup), "ms_per_step": ms / reps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "q4_0 weights, fp16/bf16 tensor-core inputs, f32 accumulate", "data": "synthetic",
+            "config": {"workload": "decoder_layer_q4_kv1024_M1", "layers_rotated": shape.n_layers,
+                       "bytes_per_layer": layer_bytes, "kv_keys": 1025,
+                       "l2": "4 distinct layers per step (279 MB > 2x L2), no flush"},
+            "us_per_layer": us_layer,
+            "roofline": {"bound": "hbm", "kernel": "decoder_step_kernel", "achieved": gbs, "peak": peak,
+                         "unit": "GB/s", "frac": gbs / peak, "traffic": None, "peak_source": peak_src},
+            "kernel_sequence_us_per_layer": ms_k / shape.n_layers * 1e3,
+            "gpu_launches": reps, "clocks": clk, "cpu_baseline": cpu}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def omp_threads():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
 def run_kernel_case(args):
     """A few launches of one kernel on one case that holds well under 1 GB on
     the device (seeded synthetic inputs as in the decoder workload), for an
@@ -629,6 +866,10 @@ def main(argv=None):
         return run_sweep(args)
     if args.workload == "kernel":
         return run_kernel_case(args)
+    if args.workload == "gemv":
+        return run_gemv(args)
+    if args.workload == "layer":
+        return run_layer(args)
     return run_ours(args)
 
 

@@ -40,9 +40,16 @@ vox_status launch_q4_gemm(const uint8_t*, int64_t, int64_t, const void*, int64_t
 vox_status launch_window_attn(const void*, int64_t, const void*, const void*, int64_t, int64_t, const void*,
                               const void*, int64_t, int64_t, void*, int, int64_t, int, int, int, float,
                               cudaStream_t);
+size_t decoder_step_ws_bytes(int n_layers, int n_kv, int group);
+const char* decoder_step_unsupported(const vox_decoder* d);
+bool decoder_step_fits(const vox_decoder* d);
+vox_status launch_decoder_step(const vox_decoder* d, uint8_t* ws, cudaStream_t s);
+void set_error_text(const char* text);
 }  // namespace vox
 
 using namespace vox;
+
+extern "C" size_t vox_decoder_workspace(const vox_decoder* d);
 
 namespace {
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -61,18 +68,17 @@ vox_status check_w(const vox_q4_weight& w, int64_t n, int64_t k)
     if (!al16(w.data)) return VOX_ERR_ALIGN;
     return VOX_OK;
 }
-}  // namespace
 
-extern "C" {
-
-size_t vox_decoder_workspace(const vox_decoder* d)
+// Offset of the persistent step's part of the decoder workspace (after the
+// per-kernel sequence's GEMV and attention parts).
+size_t dec_ps_offset(const vox_decoder* d)
 {
-    if (!d || d->dim < 32 || d->vocab < 1 || d->n_kv_heads < 1 || d->window < 1) return 0;
-    size_t g = (dec_gemv_ws(d) + 255) & ~(size_t)255;
-    return g + attn_workspace_bytes(d->n_kv_heads, d->head_dim, d->window);
+    const size_t g = (dec_gemv_ws(d) + 255) & ~(size_t)255;
+    return g + ((attn_workspace_bytes(d->n_kv_heads, d->head_dim, d->window) + 255) & ~(size_t)255);
 }
 
-vox_status vox_decoder_step(const vox_decoder* d, void* stream)
+// Host-side checks shared by both forms of the decoder step.
+vox_status check_decoder(const vox_decoder* d)
 {
     if (!d) return VOX_ERR_NULL;
     if (!d->wqkv || !d->wo || !d->w13 || !d->w2 || !d->k_cache || !d->v_cache || !d->token || !d->pos || !d->x ||
@@ -86,7 +92,10 @@ vox_status vox_decoder_step(const vox_decoder* d, void* stream)
     if (!al16(d->workspace)) return VOX_ERR_ALIGN;
     const int64_t D = d->dim, QD = (int64_t)d->n_q_heads * d->head_dim, KVD = (int64_t)d->n_kv_heads * d->head_dim;
     const int64_t F = d->ffn;
-    if (QD * 1 > 81920 || F > 81920) return VOX_ERR_SHAPE;
+    if (QD > 81920 || F > 81920) return VOX_ERR_SHAPE;
+    if ((int64_t)d->n_kv_heads * d->window > 0x7fffff00LL) return VOX_ERR_SHAPE;
+    if (!al16(d->x) || !al16(d->h) || !al16(d->qkv) || !al16(d->attn) || !al16(d->act) || !al16(d->logits))
+        return VOX_ERR_ALIGN;
     vox_status st;
     for (int l = 0; l < d->n_layers; ++l) {
         if ((st = check_w(d->wqkv[l], QD + 2 * KVD, D))) return st;
@@ -98,11 +107,47 @@ vox_status vox_decoder_step(const vox_decoder* d, void* stream)
     }
     if ((st = check_w(d->embedding, d->vocab, D))) return st;
     if ((st = check_w(d->lm_head, d->vocab, D))) return st;
+    return VOX_OK;
+}
+}  // namespace
 
+extern "C" {
+
+size_t vox_decoder_workspace(const vox_decoder* d)
+{
+    if (!d || d->dim < 32 || d->vocab < 1 || d->n_kv_heads < 1 || d->window < 1 || d->n_layers < 1 ||
+        d->n_q_heads < d->n_kv_heads)
+        return 0;
+    return dec_ps_offset(d) + decoder_step_ws_bytes(d->n_layers, d->n_kv_heads, d->n_q_heads / d->n_kv_heads);
+}
+
+vox_status vox_decoder_step(const vox_decoder* d, void* stream)
+{
+    vox_status st = check_decoder(d);
+    if (st) return st;
+    if (const char* why = decoder_step_unsupported(d)) {
+        set_error_text(why);
+        return VOX_ERR_SHAPE;
+    }
+    if (!decoder_step_fits(d)) {
+        set_error_text("the activations of the widest projection do not fit shared memory");
+        return VOX_ERR_SHAPE;
+    }
+    return launch_decoder_step(d, static_cast<uint8_t*>(d->workspace) + dec_ps_offset(d),
+                               static_cast<cudaStream_t>(stream));
+}
+
+vox_status vox_decoder_step_kernels(const vox_decoder* d, void* stream)
+{
+    vox_status st = check_decoder(d);
+    if (st) return st;
+    const int64_t D = d->dim, QD = (int64_t)d->n_q_heads * d->head_dim, KVD = (int64_t)d->n_kv_heads * d->head_dim;
+    const int64_t F = d->ffn;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t* ws_g = static_cast<uint8_t*>(d->workspace);
     uint8_t* ws_a = ws_g + ((dec_gemv_ws(d) + 255) & ~(size_t)255);
     const float scale = 1.0f / sqrtf((float)d->head_dim);
+
 
     // x = embedding row of the token (exact fp32 weights)
     if ((st = launch_q4_dequant(static_cast<const uint8_t*>(d->embedding.data), d->vocab, D, 0, d->token, 1, d->x,

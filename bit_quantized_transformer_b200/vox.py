@@ -88,6 +88,7 @@ _SIGS = {
     "vox_rmsnorm": (_I32, [_P, _I64, _I64, _I64, _F, _P, _P, _I32, _I64, _P]),
     "vox_decoder_workspace": (_SZ, [ctypes.POINTER(vox_decoder)]),
     "vox_decoder_step": (_I32, [ctypes.POINTER(vox_decoder), _P]),
+    "vox_decoder_step_kernels": (_I32, [ctypes.POINTER(vox_decoder), _P]),
     "vox_encoder_chunk": (_I32, [ctypes.POINTER(vox_encoder), _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -202,6 +203,10 @@ def vox_decoder_workspace(dec: vox_decoder) -> int:
 
 def vox_decoder_step(dec: vox_decoder, stream=None):
     _check(lib.vox_decoder_step(ctypes.byref(dec), stream_ptr(stream)), "vox_decoder_step")
+
+
+def vox_decoder_step_kernels(dec: vox_decoder, stream=None):
+    _check(lib.vox_decoder_step_kernels(ctypes.byref(dec), stream_ptr(stream)), "vox_decoder_step_kernels")
 
 
 def vox_encoder_chunk(enc: vox_encoder, stream=None):

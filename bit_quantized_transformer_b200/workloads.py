@@ -111,7 +111,12 @@ class DecoderModel:
         self.emb, self.lm = emb, lm
 
     def step(self, stream=None):
+        """One token step as one persistent launch (vox_decoder_step)."""
         V.vox_decoder_step(self.dec, stream)
+
+    def step_kernels(self, stream=None):
+        """The same step as the library's per-kernel launch sequence."""
+        V.vox_decoder_step_kernels(self.dec, stream)
 
     # ----------------------------------------------------------- graphs
     def capture(self, fn=None):
@@ -168,6 +173,10 @@ class DecoderModel:
 
     def step_launches(self) -> int:
         """Kernels one vox_decoder_step launches."""
+        return 1
+
+    def step_kernels_launches(self) -> int:
+        """Kernels one vox_decoder_step_kernels launches."""
         return 1 + self.L * 6 + 1 + 1
 
     def weight_bytes(self) -> int:

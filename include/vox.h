@@ -290,16 +290,48 @@ typedef struct {
     int64_t *pos;                /* device [1]: this step's position; incremented at end   */
     float *x, *h, *qkv, *attn, *act, *logits;  /* device activations: dim, dim,
                                     q+2kv, q_dim, ffn, vocab floats                     */
-    void *workspace;             /* device, vox_decoder_workspace() bytes, zero-filled once */
+    void *workspace;             /* device, vox_decoder_workspace() bytes, zero-filled once  */
     size_t ws_bytes;
 } vox_decoder;
 
+/* Bytes of decoder workspace (device, 16-byte aligned) that both forms of
+ * the step below need on the calling thread's current device.  Zero it once
+ * before the first step; every successful step leaves it ready for the next.
+ * After a step that left a non-zero device status (vox_device_status),
+ * zero it again before the next step. */
 size_t vox_decoder_workspace(const vox_decoder *dec);
-/* One greedy decode step: x = embedding[token]; 26 x {RMSNorm + QKV GEMV with
- * rolling append, GQA attention, Wo GEMV + residual, RMSNorm + W1||W3 GEMV +
- * SiLU*mul, W2 GEMV + residual}; RMSNorm + LM head GEMV + argmax -> token;
- * pos += 1. */
+
+/* vox_decoder_step -- [ARCH], [ROLL], [BATCH]: one greedy decode step as ONE
+ * kernel launch (the pages' single GPU submission per token step):
+ * x = embedding[token]; n_layers x {RMSNorm + QKV GEMV with rolling append,
+ * GQA attention, Wo GEMV + residual, RMSNorm + W1||W3 GEMV + SiLU*mul, W2 GEMV
+ * + residual}; RMSNorm + LM head GEMV + argmax -> token; pos += 1.  A
+ * persistent cooperative grid of one CTA per SM runs the phases back to back
+ * with grid-wide barriers; it occupies the whole device while it runs.  The
+ * same arithmetic as the kernels of vox_decoder_step_kernels (register
+ * dequantisation, fp16 activations scaled per block, fp32 accumulation;
+ * split-KV attention with bf16 hi + lo operands), summed in another fixed
+ * order: results agree within the library's tolerance, not bit for bit, and
+ * are the same from run to run.  Every device-side wait is bounded (about one
+ * second); one that gives up sets the device status word (0x501, 0x502 ring
+ * waits, 0x510 grid barrier, 0x520 drain) and the step returns early.
+ * Limits: n_layers <= 32, head_dim 128, at most 4 query heads per kv head,
+ * dim % 4 == 0, and the widest projection's activations in shared memory
+ * (dim, n_q_heads * 128 and ffn up to about 10000); otherwise VOX_ERR_SHAPE
+ * with the reason in vox_last_error() (vox_decoder_step_kernels has none of
+ * these limits).  Other errors as vox_decoder_step_kernels. */
 vox_status vox_decoder_step(const vox_decoder *dec, void *stream);
+
+/* vox_decoder_step_kernels -- the same step as a sequence of launches of the
+ * library's kernels on one stream (embedding row, per layer the QKV GEMV with
+ * rolling append, attention + combine, Wo, W1||W3 and W2 GEMVs, then the LM
+ * head with argmax and the position advance), each with programmatic
+ * dependent launch; the sequence can be captured in a CUDA graph.  Errors:
+ * NULL fields -> VOX_ERR_NULL; shapes that do not match the weights, a group
+ * above 8 or head_dim != 128 -> VOX_ERR_SHAPE; window < 1 -> VOX_ERR_RANGE;
+ * a short workspace -> VOX_ERR_WORKSPACE; a workspace, cache or activation
+ * buffer that is not 16-byte aligned -> VOX_ERR_ALIGN. */
+vox_status vox_decoder_step_kernels(const vox_decoder *dec, void *stream);
 
 typedef struct {
     int32_t n_layers, dim, n_heads, head_dim, ffn, window, rows, adapter_out;

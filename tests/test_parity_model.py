@@ -6,6 +6,9 @@ forcing, so errors do not compound), at the benchmark's full sizes.
 * the full 26-layer step with the cache filled to 8192 + 300 (wrapped): the
   last layer's attention, FFN and residual, the LM head on sampled rows and
   the argmax;
+* each decoder check for both forms of the step: the single persistent
+  launch and the per-kernel launch sequence, and small shapes on which nearly
+  every tile of the persistent step is cut between warps and CTAs;
 * one encoder layer + the adapter GEMM at M = 256, and the last layer of the
   full 32-layer chunk, each kernel on that layer's own inputs (a tap of the
   layer's input and mid-layer residual).
@@ -94,12 +97,25 @@ def check_layer_tail(shape, layer, dm, seed, pos_written):
     return w, o
 
 
-def test_decoder_layer_kv1024(env):
+FORMS = ["persistent", "kernels"]
+
+
+def run_step(dm, form, stream=None):
+    """One decoder step in the given form: one persistent launch
+    (vox_decoder_step) or the per-kernel launch sequence."""
+    if form == "persistent":
+        dm.step(stream)
+    else:
+        dm.step_kernels(stream)
+
+
+@pytest.mark.parametrize("form", FORMS)
+def test_decoder_layer_kv1024(env, form):
     torch, V, WL = env
     shape = synth.DecoderShape()
     tok = 4242
     dm = WL.DecoderModel(shape, seed=0, n_layers=1, filled=1024, token=tok)
-    dm.step()
+    run_step(dm, form)
     torch.cuda.synchronize()
     assert V.vox_device_status(True) == 0
     assert int(dm.pos.item()) == 1025
@@ -136,56 +152,131 @@ def test_decoder_layer_kv1024(env):
 
 
 def test_decoder_step_full_wrapped(env):
+    """The bench's workload: 26 layers, cache filled to 8192 + 300.  Both
+    forms of the step run from the same state (the written cache slots, the
+    position and the token are restored in between); each is checked kernel
+    by kernel on its own inputs, and a second step of each advances the ring."""
     torch, V, WL = env
     shape = synth.DecoderShape()
     filled = 8192 + 300
     dm = WL.DecoderModel(shape, seed=0, filled=filled, token=17)
-    dm.step()
-    torch.cuda.synchronize()
-    assert V.vox_device_status(True) == 0
-    assert int(dm.pos.item()) == filled + 1
-    check_layer_tail(shape, shape.n_layers - 1, dm, 0, filled)
+    slot = filled % dm.W
+    saved = [(dm.k_cache[l][:, slot:slot + 2].clone(), dm.v_cache[l][:, slot:slot + 2].clone()) for l in range(dm.L)]
     lq, ld = synth.q4_blocks(shape.vocab, shape.dim, 0, synth.LM_HEAD_ID)
-    logits = np_of(dm.logits)
-    xf = ref.rmsnorm(np_of(dm.x))
-    rows = np.unique(np.concatenate([np.random.default_rng(2).integers(0, shape.vocab, 512),
-                                     [int(np.argmax(logits))]]))
-    err_lm = gemv_err(logits[rows][None], xf[None], lq[rows], ld[rows])
-    assert err_lm <= TOL, err_lm
-    assert int(dm.token.item()) == int(np.argmax(logits))
-    # a second step advances the ring by one slot and reads the new token
-    dm.step()
-    torch.cuda.synchronize()
-    assert V.vox_device_status(True) == 0
-    assert int(dm.pos.item()) == filled + 2
-    assert int(dm.token.item()) == int(np.argmax(np_of(dm.logits)))
+    tokens = {}
+    for form in FORMS:
+        for l in range(dm.L):
+            dm.k_cache[l][:, slot:slot + 2].copy_(saved[l][0])
+            dm.v_cache[l][:, slot:slot + 2].copy_(saved[l][1])
+        dm.pos.fill_(filled)
+        dm.token.fill_(17)
+        run_step(dm, form)
+        torch.cuda.synchronize()
+        assert V.vox_device_status(True) == 0
+        assert int(dm.pos.item()) == filled + 1
+        check_layer_tail(shape, shape.n_layers - 1, dm, 0, filled)
+        logits = np_of(dm.logits)
+        xf = ref.rmsnorm(np_of(dm.x))
+        rows = np.unique(np.concatenate([np.random.default_rng(2).integers(0, shape.vocab, 512),
+                                         [int(np.argmax(logits))]]))
+        err_lm = gemv_err(logits[rows][None], xf[None], lq[rows], ld[rows])
+        assert err_lm <= TOL, (form, err_lm)
+        assert int(dm.token.item()) == int(np.argmax(logits))
+        top2 = np.sort(logits)[-2:]
+        tokens[form] = (int(dm.token.item()), float(top2[1] - top2[0]), float(np.abs(logits).max()))
+        # a second step advances the ring by one slot and reads the new token
+        run_step(dm, form)
+        torch.cuda.synchronize()
+        assert V.vox_device_status(True) == 0
+        assert int(dm.pos.item()) == filled + 2
+        assert int(dm.token.item()) == int(np.argmax(np_of(dm.logits)))
+    # the two forms pick the same token unless the top two logits are within rounding
+    (ta, ma, sa), (tb, mb, sb) = tokens["persistent"], tokens["kernels"]
+    if min(ma, mb) > 1e-3 * max(sa, sb):
+        assert ta == tb, tokens
 
 
-def test_decoder_step_graph_replay_matches_eager(env):
+@pytest.mark.parametrize("form", FORMS)
+def test_decoder_step_graph_replay_matches_eager(env, form):
     """The captured step replays exactly what the eager step computes."""
     torch, V, WL = env
     shape = synth.DecoderShape(n_layers=2)
     a = WL.DecoderModel(shape, seed=3, filled=500, token=9)
     b = WL.DecoderModel(shape, seed=3, filled=500, token=9)
     for _ in range(3):
-        a.step()
+        run_step(a, form)
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        b.step(s)                                        # warm-up outside capture
+        run_step(b, form, s)                              # warm-up outside capture
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        b.step()
+        run_step(b, form)
     g.replay()
     g.replay()
     torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
     assert int(a.pos.item()) == int(b.pos.item()) == 503
     assert int(a.token.item()) == int(b.token.item())
     assert torch.equal(a.logits, b.logits)
     for l in range(2):
         assert torch.equal(a.k_cache[l].view(torch.int16), b.k_cache[l].view(torch.int16))
+
+
+SMALL = dict(n_layers=2, dim=256, n_q_heads=4, n_kv_heads=2, head_dim=128, ffn=512, vocab=1024)
+
+
+@pytest.mark.parametrize("window,filled", [(64, 70), (100, 30), (100, 0), (48, 47), (8192, 8492)])
+def test_persistent_step_small_shapes(env, window, filled):
+    """A small decoder whose projections have a handful of 16-row tiles, so
+    nearly every tile is cut between warps and CTAs; windows that are not a
+    multiple of the 16-slot unit, a cache with one valid slot, and a full
+    window.  Every kernel of the last layer, the LM head and the argmax are
+    checked against the oracle; the per-kernel sequence must agree."""
+    torch, V, WL = env
+    shape = synth.DecoderShape(window=window, **SMALL)
+    out = {}
+    for form in FORMS:
+        dm = WL.DecoderModel(shape, seed=5, filled=filled, token=3)
+        run_step(dm, form)
+        torch.cuda.synchronize()
+        assert V.vox_device_status(True) == 0
+        assert int(dm.pos.item()) == filled + 1
+        check_layer_tail(shape, shape.n_layers - 1, dm, 5, filled)
+        lq, ld = synth.q4_blocks(shape.vocab, shape.dim, 5, synth.LM_HEAD_ID)
+        logits = np_of(dm.logits)
+        xf = ref.rmsnorm(np_of(dm.x))
+        err = gemv_err(logits[None], xf[None], lq, ld)
+        assert err <= TOL, (form, err)
+        assert int(dm.token.item()) == int(np.argmax(logits))
+        out[form] = np_of(dm.x)
+    # the two forms reach the same residual stream within the tolerance's scale
+    assert np.max(np.abs(out["persistent"] - out["kernels"])) <= 1e-2 * np.max(np.abs(out["kernels"]))
+
+
+def test_persistent_step_first_layer_from_embedding(env):
+    """The persistent step reads layer 0's input straight from the packed
+    embedding table: x after the step's embedding is the exact fp32 row, and
+    the first layer's QKV is checked on it."""
+    torch, V, WL = env
+    shape = synth.DecoderShape(window=64, **dict(SMALL, n_layers=1))
+    tok = 777
+    dm = WL.DecoderModel(shape, seed=6, filled=10, token=tok)
+    run_step(dm, "persistent")
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    eq, ed = synth.q4_blocks(shape.vocab, shape.dim, 6, synth.EMB_ID)
+    x0 = ref.c_dequant_f32(eq, ed, row0=tok, nrows=1)[0]
+    # h = x0 + Wo o: the residual used the embedding row exactly
+    w = synth.decoder_layer_weights(shape, 0, 6)
+    err_wo = gemv_err((np_of(dm.h) - x0)[None], np_of(dm.attn)[None], *w["wo"])
+    assert err_wo <= TOL, err_wo
+    qs = np.concatenate([w["wq"][0], w["wk"][0], w["wv"][0]])
+    ds = np.concatenate([w["wq"][1], w["wk"][1], w["wv"][1]])
+    err_qkv = gemv_err(np_of(dm.qkv)[None], ref.rmsnorm(x0)[None], qs, ds)
+    assert err_qkv <= TOL, err_qkv
 
 
 def check_encoder_layer(shape, em, layer, seed):
