@@ -383,6 +383,15 @@ def encoder_layer(X, Wd, k_hist, v_hist, window, n_heads, head_dim, eps=RMS_EPS)
     return h + u @ Wd["wdown"].T
 
 
+def adapter(Xd, W1, W2):
+    """The audio-to-decoder adapter on downsampled rows: Linear(5120 -> 3072),
+    exact-erf GELU, Linear(3072 -> 3072), no biases ("Mistral Voxtral Realtime
+    4B ... 순수 C 기반 CPU 전용 추론 구현", "모델 아키텍처": adapter
+    Linear -> GELU -> Linear; GELU form and no bias are readings R8)."""
+    Xd = np.asarray(Xd, np.float64)
+    return gelu(Xd @ np.asarray(W1, np.float64).T) @ np.asarray(W2, np.float64).T
+
+
 def downsample_rows(X, factor=4):
     """Conv-4x downsample as a reshape: rows factor*r .. factor*r+factor-1
     concatenated in order form row r (R10)."""

@@ -535,6 +535,32 @@ def test_window_attention_bruteforce():
             np.testing.assert_allclose(got[i, sl], want, rtol=1e-12)
 
 
+def pin_adapter(fn):
+    """Closed forms of the adapter: with W1 = a [I | 0] (picking the first
+    columns) and W2 = b I the output is b gelu(a x[:, :n]); W2 = 0 gives 0."""
+    rng = np.random.default_rng(31)
+    X = rng.standard_normal((3, 8))
+    W1 = np.zeros((4, 8)); W1[:, :4] = 1.5 * np.eye(4)
+    out = fn(X, W1, -2.0 * np.eye(4))
+    want = [[-2.0 * 0.5 * 1.5 * v * (1 + math.erf(1.5 * v / math.sqrt(2))) for v in row[:4]] for row in X]
+    np.testing.assert_allclose(out, want, rtol=1e-14)
+    assert np.array_equal(fn(X, rng.standard_normal((4, 8)), np.zeros((4, 4))), np.zeros((3, 4)))
+
+
+def test_adapter_closed_forms():
+    pin_adapter(ref.adapter)
+
+    def gelu_after_second(Xd, W1, W2):
+        return ref.gelu(np.asarray(Xd) @ np.asarray(W1).T @ np.asarray(W2).T)
+
+    def no_gelu(Xd, W1, W2):
+        return np.asarray(Xd) @ np.asarray(W1).T @ np.asarray(W2).T
+
+    for bad in (gelu_after_second, no_gelu):
+        with pytest.raises(AssertionError):
+            pin_adapter(bad)
+
+
 def test_downsample_order():
     X = np.arange(8 * 3).reshape(8, 3)
     Y = ref.downsample_rows(X, 4)
