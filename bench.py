@@ -522,6 +522,7 @@ def run_encoder(args):
     for l in range(em.L):
         calls += [(em.wqkv[l], R, D, 3 * D), (em.wo[l], R, D, D), (em.wup[l], R, D, F), (em.wdown[l], R, F, D)]
     calls.append((em.adapter, R // shape.downsample, shape.downsample * D, shape.adapter_out))
+    calls.append((em.adapter2, R // shape.downsample, shape.adapter_out, shape.adapter_out))
 
     def gemms():
         for w, m, k, n in calls:

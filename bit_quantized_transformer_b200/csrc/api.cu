@@ -24,6 +24,7 @@ vox_status launch_window_attn(const void*, int64_t, const void*, const void*, in
                               cudaStream_t);
 vox_status launch_rmsnorm(const float*, int64_t, int64_t, int64_t, float, const float*, void*, int, int64_t,
                           cudaStream_t);
+vox_status launch_cast_rows(const float*, int64_t, int64_t, int64_t, void*, int, int64_t, cudaStream_t);
 }  // namespace vox
 
 using namespace vox;
@@ -170,6 +171,47 @@ vox_status vox_q4_gemm(const vox_q4_weight* w, const void* x, int32_t x_dtype, i
     if (ep && ep->op == VOX_EP_RESIDUAL && y_dtype != VOX_F32) return VOX_ERR_DTYPE;
     return launch_q4_gemm(static_cast<const uint8_t*>(w->data), w->n, w->k, x, m, ldx, y, y_dtype, ldy, ep,
                           S(stream));
+}
+
+// Largest m that vox_q4_matmul runs on the GEMV: on B200 the tcgen05 GEMM at
+// m = 16 beat two m = 8 GEMV launches on four of the decoder's five shapes.
+constexpr int64_t kMatmulGemvMaxM = 8;
+
+size_t vox_q4_matmul_workspace(const vox_q4_weight* w, int64_t m, const vox_epilogue* ep)
+{
+    if (!w || w->n < 1 || w->k < 32 || m < 1) return 0;
+    const size_t g = (vox_q4_gemv_workspace(w, m < kMatmulGemvMaxM ? m : kMatmulGemvMaxM, ep) + 255) & ~(size_t)255;
+    if (m <= kMatmulGemvMaxM) return g;
+    return g + (((size_t)m * (size_t)w->k * 2 + 255) & ~(size_t)255);
+}
+
+vox_status vox_q4_matmul(const vox_q4_weight* w, const float* x, int64_t m, int64_t ldx, float* y, int64_t ldy,
+                         const vox_epilogue* ep, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (m >= 1 && m <= kMatmulGemvMaxM) return vox_q4_gemv(w, x, m, ldx, y, ldy, ep, workspace, ws_bytes, stream);
+    vox_status st = check_weight(w);
+    if (st) return st;
+    if (!x || !y) return VOX_ERR_NULL;
+    if (m < 1 || m > (1LL << 30) || w->k % 64 || ldx < w->k) return VOX_ERR_SHAPE;
+    const int op = ep ? ep->op : VOX_EP_NONE;
+    if (op != VOX_EP_NONE && op != VOX_EP_RESIDUAL && op != VOX_EP_GELU) return VOX_ERR_RANGE;
+    if (ep && ep->rmsnorm && !(ep->eps >= 0.f)) return VOX_ERR_RANGE;
+    if (!workspace) return VOX_ERR_WORKSPACE;
+    if (ws_bytes < vox_q4_matmul_workspace(w, m, ep)) return VOX_ERR_WORKSPACE;
+    if (!al16(workspace)) return VOX_ERR_ALIGN;
+    if ((st = check_epilogue(ep, w->n, w->k, m, ldy, true, true))) return st;
+    // x (normalised first if asked) -> bf16 rows in the workspace, then the GEMM
+    uint8_t* xb = static_cast<uint8_t*>(workspace) + ((vox_q4_gemv_workspace(w, kMatmulGemvMaxM, ep) + 255) & ~(size_t)255);
+    st = (ep && ep->rmsnorm) ? launch_rmsnorm(x, m, w->k, ldx, ep->eps, ep->norm_weight, xb, VOX_BF16, w->k, S(stream))
+                             : launch_cast_rows(x, m, w->k, ldx, xb, VOX_BF16, w->k, S(stream));
+    if (st) return st;
+    vox_epilogue e2 = {};
+    if (ep) {
+        e2 = *ep;
+        e2.rmsnorm = 0;
+    }
+    return launch_q4_gemm(static_cast<const uint8_t*>(w->data), w->n, w->k, xb, m, w->k, y, VOX_F32, ldy,
+                          ep ? &e2 : nullptr, S(stream));
 }
 
 vox_status vox_kv_append_rolling(void* k_cache, void* v_cache, const void* k_new, const void* v_new,

@@ -18,8 +18,8 @@
 // 750; readings: RMSNorm pre-norm, ungated GELU FFN):
 //   xn = RMSNorm(x) (bf16) -> QKV GEMM -> window attention -> O GEMM + x
 //   -> RMSNorm -> up GEMM + GELU -> down GEMM + x.  Then the 4x downsample
-//   (rows 4r..4r+3 side by side = a [rows/4][4 dim] view) and the adapter's
-//   first GEMM 5120 -> 3072.
+//   (rows 4r..4r+3 side by side = a [rows/4][4 dim] view) and the adapter:
+//   GEMM 5120 -> 3072 + GELU (bf16), GEMM 3072 -> 3072.
 #include "vox_internal.cuh"
 
 namespace vox {
@@ -208,13 +208,15 @@ vox_status vox_encoder_chunk(const vox_encoder* e, void* stream)
 {
     if (!e) return VOX_ERR_NULL;
     if (!e->wqkv || !e->wo || !e->wup || !e->wdown || !e->k_hist || !e->v_hist || !e->x || !e->xn || !e->qkv ||
-        !e->att || !e->up || !e->adapter_out_buf)
+        !e->att || !e->up || !e->adapter_mid || !e->adapter_out_buf)
         return VOX_ERR_NULL;
     if (e->n_layers < 1 || e->n_heads < 1 || e->head_dim < 1 || e->head_dim > 64 || e->rows < 4 || e->rows % 4 ||
         e->dim != e->n_heads * e->head_dim || e->dim % 64 || e->ffn % 64)
         return VOX_ERR_SHAPE;
     if (e->window < 1) return VOX_ERR_RANGE;
-    if (!al16(e->xn) || !al16(e->qkv) || !al16(e->att) || !al16(e->up)) return VOX_ERR_ALIGN;
+    if (!al16(e->xn) || !al16(e->qkv) || !al16(e->att) || !al16(e->up) || !al16(e->adapter_mid))
+        return VOX_ERR_ALIGN;
+    if (e->adapter_out % 64) return VOX_ERR_SHAPE;
     const int64_t D = e->dim, F = e->ffn, R = e->rows;
     vox_status st;
     for (int l = 0; l < e->n_layers; ++l) {
@@ -225,6 +227,7 @@ vox_status vox_encoder_chunk(const vox_encoder* e, void* stream)
         if (!e->k_hist[l] || !e->v_hist[l]) return VOX_ERR_NULL;
     }
     if ((st = check_w(e->adapter, e->adapter_out, 4 * D))) return st;
+    if ((st = check_w(e->adapter2, e->adapter_out, e->adapter_out))) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const float scale = 1.0f / sqrtf((float)e->head_dim);
     for (int l = 0; l < e->n_layers; ++l) {
@@ -258,8 +261,14 @@ vox_status vox_encoder_chunk(const vox_encoder* e, void* stream)
     }
     // 4x downsample: bf16 copy of the rows, read as [R/4][4D]
     if ((st = launch_cast_rows(e->x, R, D, D, e->xn, VOX_BF16, D, s))) return st;
-    return launch_q4_gemm(static_cast<const uint8_t*>(e->adapter.data), e->adapter_out, 4 * D, e->xn, R / 4, 4 * D,
-                          e->adapter_out_buf, VOX_F32, e->adapter_out, nullptr, s);
+    vox_epilogue gl = {};
+    gl.op = VOX_EP_GELU;
+    if ((st = launch_q4_gemm(static_cast<const uint8_t*>(e->adapter.data), e->adapter_out, 4 * D, e->xn, R / 4,
+                             4 * D, e->adapter_mid, VOX_BF16, e->adapter_out, &gl, s)))
+        return st;
+    return launch_q4_gemm(static_cast<const uint8_t*>(e->adapter2.data), e->adapter_out, e->adapter_out,
+                          e->adapter_mid, R / 4, e->adapter_out, e->adapter_out_buf, VOX_F32, e->adapter_out, nullptr,
+                          s);
 }
 
 }  // extern "C"

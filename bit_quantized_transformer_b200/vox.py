@@ -61,10 +61,10 @@ class vox_encoder(ctypes.Structure):
                 ("ffn", _I32), ("window", _I32), ("rows", _I32), ("adapter_out", _I32), ("eps", _F),
                 ("wqkv", ctypes.POINTER(vox_q4_weight)), ("wo", ctypes.POINTER(vox_q4_weight)),
                 ("wup", ctypes.POINTER(vox_q4_weight)), ("wdown", ctypes.POINTER(vox_q4_weight)),
-                ("adapter", vox_q4_weight),
+                ("adapter", vox_q4_weight), ("adapter2", vox_q4_weight),
                 ("k_hist", ctypes.POINTER(_P)), ("v_hist", ctypes.POINTER(_P)),
-                ("x", _P), ("xn", _P), ("qkv", _P), ("att", _P), ("up", _P), ("adapter_out_buf", _P),
-                ("tap", _P)]
+                ("x", _P), ("xn", _P), ("qkv", _P), ("att", _P), ("up", _P), ("adapter_mid", _P),
+                ("adapter_out_buf", _P), ("tap", _P)]
 
 
 _W = ctypes.POINTER(vox_q4_weight)
@@ -79,6 +79,8 @@ _SIGS = {
     "vox_q4_gemv": (_I32, [_W, _P, _I64, _I64, _P, _I64, _E, _P, _SZ, _P]),
     "vox_q4_gemv_workspace": (_SZ, [_W, _I64, _E]),
     "vox_q4_gemm": (_I32, [_W, _P, _I32, _I64, _I64, _P, _I32, _I64, _E, _P]),
+    "vox_q4_matmul": (_I32, [_W, _P, _I64, _I64, _P, _I64, _E, _P, _SZ, _P]),
+    "vox_q4_matmul_workspace": (_SZ, [_W, _I64, _E]),
     "vox_kv_append_rolling": (_I32, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _P]),
     "vox_gqa_decode_attn": (_I32, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _F, _P, _SZ, _P]),
     "vox_gqa_decode_attn_workspace": (_SZ, [_I32, _I32, _I32, _I32]),
@@ -158,6 +160,16 @@ def vox_q4_gemv(w: vox_q4_weight, x, m, ldx, y, ldy, ep=None, workspace=None, ws
 def vox_q4_gemm(w: vox_q4_weight, x, x_dtype, m, ldx, y, y_dtype, ldy, ep=None, stream=None):
     _check(lib.vox_q4_gemm(ctypes.byref(w), ptr(x), x_dtype, m, ldx, ptr(y), y_dtype, ldy,
                            ctypes.byref(ep) if ep is not None else None, stream_ptr(stream)), "vox_q4_gemm")
+
+
+def vox_q4_matmul_workspace(w: vox_q4_weight, m: int, ep: vox_epilogue | None = None) -> int:
+    return lib.vox_q4_matmul_workspace(ctypes.byref(w), m, ctypes.byref(ep) if ep is not None else None)
+
+
+def vox_q4_matmul(w: vox_q4_weight, x, m, ldx, y, ldy, ep=None, workspace=None, ws_bytes=0, stream=None):
+    _check(lib.vox_q4_matmul(ctypes.byref(w), ptr(x), m, ldx, ptr(y), ldy,
+                             ctypes.byref(ep) if ep is not None else None, ptr(workspace), ws_bytes,
+                             stream_ptr(stream)), "vox_q4_matmul")
 
 
 def vox_kv_append_rolling(k_cache, v_cache, k_new, v_new, new_dtype, n_kv_heads, head_dim, window, pos,

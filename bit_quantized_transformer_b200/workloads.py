@@ -211,6 +211,8 @@ class EncoderModel:
             kh.append(kt.data_ptr()); vh.append(vt.data_ptr())
         self.ad_t, ad = pack_q4(*synth.q4_blocks(shape.adapter_out, shape.downsample * D, seed, synth.ADAPTER_ID),
                                 device)
+        self.ad2_t, ad2 = pack_q4(*synth.q4_blocks(shape.adapter_out, shape.adapter_out, seed, synth.ADAPTER2_ID),
+                                  device)
         self._keep = keep
         self.wqkv, self.wo, self.wup, self.wdown = wqkv, wo, wup, wdown
         self.k_hist = [keep[6 * l + 4] for l in range(self.L)]
@@ -222,6 +224,7 @@ class EncoderModel:
         self.qkv = torch.zeros(R, 3 * D, **bf)
         self.att = torch.zeros(R, D, **bf)
         self.up = torch.zeros(R, F, **bf)
+        self.mid = torch.zeros(R // shape.downsample, shape.adapter_out, **bf)
         self.out = torch.zeros(R // shape.downsample, shape.adapter_out, dtype=torch.float32, device=device)
         Arr = V.vox_q4_weight * self.L
         Ptr = ctypes.c_void_p * self.L
@@ -230,7 +233,8 @@ class EncoderModel:
         e.n_layers, e.dim, e.n_heads, e.head_dim = self.L, D, shape.n_heads, shape.head_dim
         e.ffn, e.window, e.rows, e.adapter_out, e.eps = F, shape.window, R, shape.adapter_out, eps
         e.wqkv, e.wo, e.wup, e.wdown = [ctypes.cast(a, ctypes.POINTER(V.vox_q4_weight)) for a in self._arrs[:4]]
-        e.adapter = ad
+        e.adapter, e.adapter2 = ad, ad2
+        e.adapter_mid = self.mid.data_ptr()
         e.k_hist = ctypes.cast(self._arrs[4], ctypes.POINTER(ctypes.c_void_p))
         e.v_hist = ctypes.cast(self._arrs[5], ctypes.POINTER(ctypes.c_void_p))
         for name in ("x", "xn", "qkv", "att", "up"):
@@ -240,7 +244,7 @@ class EncoderModel:
         self.tap = torch.zeros(2, R, D, dtype=torch.float32, device=device) if tap else None
         e.tap = self.tap.data_ptr() if tap else None
         self.enc = e
-        self.adapter = ad
+        self.adapter, self.adapter2 = ad, ad2
 
     def reset(self):
         self.x.copy_(self.x0)
@@ -252,4 +256,5 @@ class EncoderModel:
         s = self.shape
         R, D, F = s.rows, s.dim, s.ffn
         per_layer = 2 * R * D * (3 * D + D + F) + 2 * R * F * D
-        return self.L * per_layer + 2 * (R // s.downsample) * (s.downsample * D) * s.adapter_out
+        rd = R // s.downsample
+        return self.L * per_layer + 2 * rd * (s.downsample * D) * s.adapter_out + 2 * rd * s.adapter_out ** 2

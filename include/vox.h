@@ -189,6 +189,23 @@ vox_status vox_q4_gemm(const vox_q4_weight *w, const void *x, int32_t x_dtype, i
                        int64_t ldx, void *y, int32_t y_dtype, int64_t ldy,
                        const vox_epilogue *ep, void *stream);
 
+/* ------------------------------------------------- Q4_0 matmul, any M
+ * vox_q4_matmul -- [Q4], [FUSE]: y = x W^T for m rows of fp32 activations,
+ * choosing the kernel by m at the crossover measured on B200 (the batched
+ * sweep over the decoder's shapes): m <= 8 runs the register-dequantising
+ * GEMV (vox_q4_gemv), m > 8 rounds x (after the optional RMSNorm) to bf16
+ * into the workspace and runs the tcgen05 GEMM (vox_q4_gemm).  x: device fp32
+ * [m][ldx]; y: device fp32 [m][ldy].  Epilogues: every vox_q4_gemv epilogue
+ * at m <= 8; NONE, RESIDUAL and GELU (with or without the RMSNorm prologue)
+ * at m > 8, other ones -> VOX_ERR_RANGE.  workspace: device,
+ * vox_q4_matmul_workspace() bytes, 16-byte aligned; its first 256 bytes
+ * must be zero before the first use (the GEMV's argmax state, left zero by
+ * every call).  Calls that share a workspace must not overlap on the GPU.
+ * Errors as vox_q4_gemv and vox_q4_gemm. */
+vox_status vox_q4_matmul(const vox_q4_weight *w, const float *x, int64_t m, int64_t ldx, float *y, int64_t ldy,
+                         const vox_epilogue *ep, void *workspace, size_t ws_bytes, void *stream);
+size_t vox_q4_matmul_workspace(const vox_q4_weight *w, int64_t m, const vox_epilogue *ep);
+
 /* ------------------------------------------------------------ rolling cache
  * vox_kv_append_rolling -- [ROLL].  Stores one position: k_new and v_new
  * (device [n_kv_heads][head_dim] of new_dtype VOX_F32 or VOX_BF16) are
@@ -340,7 +357,8 @@ typedef struct {
     const vox_q4_weight *wo;     /* dim x dim                                           */
     const vox_q4_weight *wup;    /* ffn x dim                                           */
     const vox_q4_weight *wdown;  /* dim x ffn                                           */
-    vox_q4_weight adapter;       /* adapter_out x 4dim                                   */
+    vox_q4_weight adapter;       /* adapter_out x 4dim: the adapter's first Linear        */
+    vox_q4_weight adapter2;      /* adapter_out x adapter_out: its second Linear          */
     const void *const *k_hist;   /* host array [n_layers] of device bf16 [window][dim]  */
     const void *const *v_hist;
     float *x;                    /* device fp32 [rows][dim]: chunk input, updated in place */
@@ -348,6 +366,7 @@ typedef struct {
     void *qkv;                   /* device bf16 [rows][3dim] scratch                    */
     void *att;                   /* device bf16 [rows][dim] scratch                     */
     void *up;                    /* device bf16 [rows][ffn] scratch                     */
+    void *adapter_mid;           /* device bf16 [rows/4][adapter_out] scratch: GELU output */
     float *adapter_out_buf;      /* device fp32 [rows/4][adapter_out]                   */
     float *tap;                  /* device fp32 [2][rows][dim], or NULL: receives the last
                                     layer's input x (tap[0]) and its residual stream h
@@ -357,7 +376,9 @@ typedef struct {
 
 /* One encoder chunk: 32 x {RMSNorm, QKV GEMM, window attention, O GEMM +
  * residual, RMSNorm, up GEMM + GELU, down GEMM + residual}, then the 4x
- * downsample (rows 4r..4r+3 concatenated) and the adapter's first GEMM. */
+ * downsample (rows 4r..4r+3 concatenated) and the adapter ([ARCH]: Linear
+ * 4dim -> adapter_out, exact-erf GELU, Linear adapter_out -> adapter_out;
+ * the GELU output is rounded to bf16 in adapter_mid). */
 vox_status vox_encoder_chunk(const vox_encoder *enc, void *stream);
 
 #ifdef __cplusplus

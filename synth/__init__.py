@@ -32,6 +32,7 @@ ENC_BASE = 2_000_000
 E_QKV, E_O, E_UP, E_DOWN, E_KHIST, E_VHIST = range(6)
 ADAPTER_ID = 3_000_000      # adapter first Linear, Q4_0 3072 x 5120
 ENC_X_ID = 3_000_001        # encoder chunk input rows
+ADAPTER2_ID = 3_000_002     # adapter second Linear, Q4_0 3072 x 3072
 SWEEP_BASE = 4_000_000      # batched-shape sweep tensors
 
 D_SCALE = 0.002

@@ -138,6 +138,30 @@ def test_gemm_validation(V):
                          None) == V.VOX_ERR_SHAPE
 
 
+def test_matmul_validation(V):
+    """vox_q4_matmul checks the GEMM side's arguments on the host (m > 8);
+    m <= 8 takes the GEMV's checks."""
+    L = V.lib
+    w = V.vox_q4_weight(FAKE, 128, 128)
+    ws = V.vox_q4_matmul_workspace(w, 16, None)
+    assert ws >= 256 + 16 * 128 * 2
+    assert V.vox_q4_matmul_workspace(w, 8, None) == V.vox_q4_gemv_workspace(w, 8, None)
+    mm = lambda m=16, ldx=128, ep=None, wsp=FAKE, wsb=ws, x=FAKE: L.vox_q4_matmul(
+        ctypes.byref(w), x, m, ldx, FAKE, 128, ctypes.byref(ep) if ep else None, wsp, wsb, None)
+    assert mm(x=None) == V.VOX_ERR_NULL
+    assert mm(m=0) == V.VOX_ERR_SHAPE
+    assert mm(ldx=100) == V.VOX_ERR_SHAPE
+    assert mm(wsp=None) == V.VOX_ERR_WORKSPACE
+    assert mm(wsb=ws - 16) == V.VOX_ERR_WORKSPACE
+    assert mm(wsp=FAKE + 8) == V.VOX_ERR_ALIGN
+    assert mm(ep=V.vox_epilogue(op=V.VOX_EP_SILU_MUL)) == V.VOX_ERR_RANGE
+    assert mm(ep=V.vox_epilogue(op=V.VOX_EP_ARGMAX, argmax=FAKE)) == V.VOX_ERR_RANGE
+    assert mm(ep=V.vox_epilogue(op=V.VOX_EP_GELU, rmsnorm=1, eps=-1.0)) == V.VOX_ERR_RANGE
+    assert mm(m=4, x=None) == V.VOX_ERR_NULL            # the GEMV's own checks
+    w96 = V.vox_q4_weight(FAKE, 128, 96)
+    assert L.vox_q4_matmul(ctypes.byref(w96), FAKE, 16, 96, FAKE, 128, None, FAKE, ws, None) == V.VOX_ERR_SHAPE
+
+
 def test_kv_and_attention_validation(V):
     L = V.lib
     assert L.vox_kv_append_rolling(None, FAKE, FAKE, FAKE, 0, 8, 128, 16, 0, None) == V.VOX_ERR_NULL

@@ -315,6 +315,45 @@ def test_kv_append_bitexact(env, dtype):
         assert np.array_equal(bf16_bits(kc), kc_ref) and np.array_equal(bf16_bits(vc), vc_ref)
 
 
+# ------------------------------------------------------- matmul dispatch
+@pytest.mark.parametrize("m", [1, 8, 9, 16, 64])
+@pytest.mark.parametrize("epi", ["none", "rms_gelu", "residual"])
+def test_matmul_dispatch(env, m, epi):
+    """vox_q4_matmul at either side of the GEMV / GEMM crossover, fp32 in and
+    out, with the epilogues both kernels share; checked against the oracle on
+    the fp32 input (the GEMM side's bf16 rounding of x is the kernel's error)."""
+    torch, V, WL = env
+    n, k = 384, 1280
+    qs, d = synth.q4_blocks(n, k, 0, 9500 + m)
+    x = synth.activations(m, k, 0, 9600 + m) * 3.0
+    res = synth.activations(m, n, 0, 9700 + m)
+    packed, w = WL.pack_q4(qs, d, "cuda")
+    W = ref.q4_weights(qs, d)
+    ep = None
+    xr = x.astype(np.float64)
+    if epi == "rms_gelu":
+        ep = V.vox_epilogue(op=V.VOX_EP_GELU, rmsnorm=1, eps=1e-5)
+        xr = ref.rmsnorm(xr)
+    elif epi == "residual":
+        rt = WL.to_dev(res, "cuda")
+        ep = V.vox_epilogue(op=V.VOX_EP_RESIDUAL, residual=rt.data_ptr(), ldr=n)
+    y = torch.full((m, n), float("nan"), device="cuda")
+    wsb = V.vox_q4_matmul_workspace(w, m, ep)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    V.vox_q4_matmul(w, WL.to_dev(x, "cuda"), m, k, y, n, ep, ws, wsb)
+    check_status(V)
+    got = np_of(y).astype(np.float64)
+    want = xr @ W.T
+    if epi == "rms_gelu":
+        got_lin, want = got, ref.gelu(want)
+        err = ref.gemv_error(got_lin, want, xr, W)
+    elif epi == "residual":
+        err = ref.gemv_error(got - res, want, xr, W)
+    else:
+        err = ref.gemv_error(got, want, xr, W)
+    assert err <= TOL, err
+
+
 # -------------------------------------------------------------- attention
 def attn_case(env, n_q, n_kv, hd, W, pos, seed=0, nan_fill=False):
     torch, V, WL = env

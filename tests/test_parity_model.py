@@ -337,11 +337,25 @@ def test_encoder_layer_and_adapter(env):
     x0 = synth.activations(R, D, 0, synth.ENC_X_ID)
     assert np.array_equal(np_of(em.tap[0]), x0)                 # layer 0's input is the chunk input
     x1 = check_encoder_layer(shape, em, 0, 0)
-    # adapter on the downsampled bf16 rows of x1
-    aq, ad = synth.q4_blocks(shape.adapter_out, 4 * D, 0, synth.ADAPTER_ID)
-    xd = ref.downsample_rows(ref.bf16_to_f64(ref.f32_to_bf16(x1.astype(np.float32))), 4)
-    err_ad = gemv_err(np_of(em.out), xd, aq, ad)
-    assert err_ad <= TOL, err_ad
+    check_adapter(shape, em, x1, 0)
+
+
+def check_adapter(shape, em, x_out, seed):
+    """The adapter on the downsampled bf16 rows of the chunk output: the first
+    Linear + GELU (stored as bf16) on the GPU's input, the second Linear on the
+    GPU's GELU output; the oracle's whole adapter is reported."""
+    aq, ad = synth.q4_blocks(shape.adapter_out, 4 * shape.dim, seed, synth.ADAPTER_ID)
+    a2q, a2d = synth.q4_blocks(shape.adapter_out, shape.adapter_out, seed, synth.ADAPTER2_ID)
+    xd = ref.downsample_rows(ref.bf16_to_f64(ref.f32_to_bf16(x_out.astype(np.float32))), 4)
+    W1 = ref.q4_weights(aq, ad)
+    mid = ref.bf16_to_f64(bits(em.mid))
+    err1 = ref.gemv_error(mid, ref.gelu(xd @ W1.T), xd, W1)
+    assert err1 <= TOL, ("adapter linear 1 + gelu", err1)
+    err2 = gemv_err(np_of(em.out), mid, a2q, a2d)
+    assert err2 <= TOL, ("adapter linear 2", err2)
+    full = ref.adapter(xd, W1, ref.q4_weights(a2q, a2d))
+    e2e = np.max(np.abs(np_of(em.out) - full)) / np.max(np.abs(full))
+    print(f"adapter end-to-end max rel error {e2e:.3e}")
 
 
 def test_encoder_chunk_last_layer(env):
@@ -355,7 +369,4 @@ def test_encoder_chunk_last_layer(env):
     assert V.vox_device_status(True) == 0
     x_out = check_encoder_layer(shape, em, shape.n_layers - 1, 0)
     assert np.all(np.isfinite(x_out))
-    aq, ad = synth.q4_blocks(shape.adapter_out, 4 * shape.dim, 0, synth.ADAPTER_ID)
-    xd = ref.downsample_rows(ref.bf16_to_f64(ref.f32_to_bf16(x_out.astype(np.float32))), 4)
-    err_ad = gemv_err(np_of(em.out), xd, aq, ad)
-    assert err_ad <= TOL, err_ad
+    check_adapter(shape, em, x_out, 0)
