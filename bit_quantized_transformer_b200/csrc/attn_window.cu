@@ -5,9 +5,12 @@
 // n_hist + i and sees key position p iff pos_i - window < p <= pos_i; keys
 // before n_hist come from the history rows, the rest from the chunk itself.
 //
-// One CTA per (64 query rows, head); four warps of 16 query rows each.
-// Per 64-key tile (K and V staged in shared memory, 80-byte rows, which
-// ldmatrix reads without bank conflicts):
+// One CTA per (32 query rows, head): two warps of 16 query rows each, so
+// the 256-row chunk x 32 heads gives 256 CTAs.  The keys a CTA needs (its
+// 32 rows' windows, 781 positions at window 750) stream through a 3-stage
+// ring of 64-key K and V tiles filled with 16-byte cp.async copies, so the
+// loads of tile i + 2 overlap the math of tile i.  Per tile (80-byte rows,
+// which ldmatrix reads without bank conflicts):
 //   S = Q K^T        mma m16n8k16 bf16, head_dim padded to 48 with zeros
 //   online softmax in the exp2 domain, masked by position
 //   O += P V         P split into bf16 hi + lo parts (two MMAs)
@@ -15,10 +18,14 @@
 
 namespace vox {
 
-constexpr int kWinQ = 64;       // query rows per CTA
+constexpr int kWinQ = 32;       // query rows per CTA
+constexpr int kWinWarps = kWinQ / 16;
+constexpr int kWinThreads = 32 * kWinWarps;
 constexpr int kWinK = 64;       // keys per tile
+constexpr int kWinStages = 3;
 constexpr int kWinHd = 40;
 constexpr int kWinRow = kWinHd * 2;   // 80 bytes
+constexpr int kWinTile = kWinK * kWinRow;   // one K or V tile
 
 struct WinArgs {
     const uint16_t* q;
@@ -53,10 +60,38 @@ __device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], uint32_t addr)
                  : "r"(addr) : "memory");
 }
 
-__global__ void __launch_bounds__(128) window_attn_kernel(const WinArgs a)
+// 16-byte asynchronous global -> shared copy; src_bytes 0 writes zeros.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes)
 {
-    __shared__ __align__(128) uint8_t sK[kWinK * kWinRow];
-    __shared__ __align__(128) uint8_t sV[kWinK * kWinRow];
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Copies of key tile [j0, j0 + 64) of head h (K and V) into one ring stage;
+// rows at or past j_end are zero-filled.
+__device__ __forceinline__ void win_load_tile(const WinArgs& a, int h, int64_t j0, int64_t j_end, uint8_t* sK,
+                                              uint8_t* sV, int tid)
+{
+    for (int i = tid; i < kWinK * 5 * 2; i += kWinThreads) {
+        const int mat = i / (kWinK * 5), rem = i - mat * (kWinK * 5), kr = rem / 5, u = rem - kr * 5;
+        const int64_t j = j0 + kr;
+        const bool in = j < j_end;
+        const int64_t jj = in ? j : j_end - 1;                 // a valid address; nothing is read when !in
+        const uint16_t* src = jj < a.n_hist ? (mat ? a.vh : a.kh) + jj * a.ld_hist
+                                            : (mat ? a.vn : a.kn) + (jj - a.n_hist) * a.ld_new;
+        cp_async16((mat ? sV : sK) + kr * kWinRow + u * 16, src + h * kWinHd + u * 8, in ? 16u : 0u);
+    }
+}
+
+__global__ void __launch_bounds__(kWinThreads) window_attn_kernel(const WinArgs a)
+{
+    __shared__ __align__(128) uint8_t sKs[kWinStages][kWinTile];
+    __shared__ __align__(128) uint8_t sVs[kWinStages][kWinTile];
     pdl_wait();
     pdl_launch_dependents();
 
@@ -102,22 +137,26 @@ __global__ void __launch_bounds__(128) window_attn_kernel(const WinArgs a)
     const int64_t p_hi = a.n_hist + q_last;
     const int64_t j_begin = p_lo - W + 1 > 0 ? p_lo - W + 1 : 0;
     const int64_t j_end = p_hi + 1 < n_keys ? p_hi + 1 : n_keys;
-    const uint32_t sKa = smem_addr(sK), sVa = smem_addr(sV);
+    const int64_t ntiles = j_end > j_begin ? (j_end - j_begin + kWinK - 1) / kWinK : 0;
 
-    for (int64_t j0 = j_begin; j0 < j_end; j0 += kWinK) {
-        __syncthreads();
-        for (int i = tid; i < kWinK * 5 * 2; i += 128) {
-            const int mat = i / (kWinK * 5), rem = i % (kWinK * 5), kr = rem / 5, u = rem % 5;
-            const int64_t j = j0 + kr;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (j < j_end) {
-                const uint16_t* src = j < a.n_hist ? (mat ? a.vh : a.kh) + j * a.ld_hist
-                                                   : (mat ? a.vn : a.kn) + (j - a.n_hist) * a.ld_new;
-                v = *reinterpret_cast<const uint4*>(src + h * kWinHd + u * 8);
-            }
-            *reinterpret_cast<uint4*>((mat ? sV : sK) + kr * kWinRow + u * 16) = v;
+    // prologue: the first two tiles in flight
+#pragma unroll
+    for (int st = 0; st < kWinStages - 1; ++st) {
+        if (st < ntiles) win_load_tile(a, h, j_begin + (int64_t)st * kWinK, j_end, sKs[st], sVs[st], tid);
+        cp_async_commit();
+    }
+    for (int64_t it = 0; it < ntiles; ++it) {
+        const int64_t j0 = j_begin + it * kWinK;
+        cp_async_wait<kWinStages - 2>();                     // tile `it` has landed (this thread's copies)
+        __syncthreads();                                     // ... everyone's; and stage it-1 is free
+        {
+            const int64_t nx = it + kWinStages - 1;
+            const int sn = (int)(nx % kWinStages);
+            if (nx < ntiles) win_load_tile(a, h, j_begin + nx * kWinK, j_end, sKs[sn], sVs[sn], tid);
+            cp_async_commit();
         }
-        __syncthreads();
+        const int sc = (int)(it % kWinStages);
+        const uint32_t sKa = smem_addr(sKs[sc]), sVa = smem_addr(sVs[sc]);
 
         // ---- S = Q K^T : 8 n-tiles of 8 keys
         float s[8][4];
@@ -273,7 +312,7 @@ vox_status launch_window_attn(const void* q, int64_t ldq, const void* k_hist, co
     a.window = window;
     a.sl2 = scale * 1.4426950408889634f;
     dim3 grid((unsigned)ceil_div(n_q, kWinQ), (unsigned)n_heads);
-    return launch_pdl(window_attn_kernel, grid, dim3(128), 0, s, a);
+    return launch_pdl(window_attn_kernel, grid, dim3(kWinThreads), 0, s, a);
 }
 
 }  // namespace vox

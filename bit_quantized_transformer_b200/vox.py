@@ -92,6 +92,17 @@ _SIGS = {
     "vox_decoder_step": (_I32, [ctypes.POINTER(vox_decoder), _P]),
     "vox_decoder_step_kernels": (_I32, [ctypes.POINTER(vox_decoder), _P]),
     "vox_encoder_chunk": (_I32, [ctypes.POINTER(vox_encoder), _P]),
+    "vox_gguf_open": (_I32, [ctypes.c_char_p, ctypes.POINTER(_P)]),
+    "vox_gguf_close": (None, [_P]),
+    "vox_gguf_tensor_count": (_I64, [_P]),
+    "vox_gguf_find_tensor": (_I64, [_P, ctypes.c_char_p]),
+    "vox_gguf_tensor_info": (_I32, [_P, _I64, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I32),
+                                    ctypes.POINTER(_I32), ctypes.POINTER(_I64), ctypes.POINTER(ctypes.c_uint64)]),
+    "vox_gguf_tensor_data": (_P, [_P, _I64]),
+    "vox_gguf_get_int": (_I32, [_P, ctypes.c_char_p, ctypes.POINTER(_I64)]),
+    "vox_gguf_get_float": (_I32, [_P, ctypes.c_char_p, ctypes.POINTER(ctypes.c_double)]),
+    "vox_gguf_get_string": (ctypes.c_char_p, [_P, ctypes.c_char_p]),
+    "vox_gguf_upload_q4": (_I32, [_P, _I64, _P, _SZ, _I32, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -227,3 +238,58 @@ def vox_encoder_chunk(enc: vox_encoder, stream=None):
 
 def vox_device_status(clear: bool = True) -> int:
     return lib.vox_device_status(1 if clear else 0)
+
+
+# ------------------------------------------------------------ GGUF files
+class GGUF:
+    """A GGUF file opened through vox_gguf_open (the handle is closed with
+    close() or when the object is collected)."""
+
+    def __init__(self, path: str):
+        h = _P()
+        _check(lib.vox_gguf_open(str(path).encode(), ctypes.byref(h)), "vox_gguf_open")
+        self.h = h
+
+    def close(self):
+        if self.h:
+            lib.vox_gguf_close(self.h)
+            self.h = None
+
+    def __del__(self):
+        self.close()
+
+    def tensor_count(self) -> int:
+        return lib.vox_gguf_tensor_count(self.h)
+
+    def find(self, name: str) -> int:
+        return lib.vox_gguf_find_tensor(self.h, name.encode())
+
+    def info(self, i: int):
+        """(name, type, dims innermost first, nbytes) of tensor i."""
+        name, typ, nd = ctypes.c_char_p(), _I32(), _I32()
+        dims, nb = (_I64 * 4)(), ctypes.c_uint64()
+        _check(lib.vox_gguf_tensor_info(self.h, i, ctypes.byref(name), ctypes.byref(typ), ctypes.byref(nd), dims,
+                                        ctypes.byref(nb)), "vox_gguf_tensor_info")
+        return name.value.decode(), typ.value, list(dims)[:nd.value], nb.value
+
+    def data(self, i: int) -> bytes:
+        p = lib.vox_gguf_tensor_data(self.h, i)
+        return ctypes.string_at(p, self.info(i)[3]) if p else b""
+
+    def get_int(self, key: str) -> int:
+        v = _I64()
+        _check(lib.vox_gguf_get_int(self.h, key.encode(), ctypes.byref(v)), "vox_gguf_get_int")
+        return v.value
+
+    def get_float(self, key: str) -> float:
+        v = ctypes.c_double()
+        _check(lib.vox_gguf_get_float(self.h, key.encode(), ctypes.byref(v)), "vox_gguf_get_float")
+        return v.value
+
+    def get_string(self, key: str):
+        v = lib.vox_gguf_get_string(self.h, key.encode())
+        return None if v is None else v.decode()
+
+    def upload_q4(self, i: int, scratch, packed, flags: int = VOX_PACK_PLAIN, stream=None):
+        _check(lib.vox_gguf_upload_q4(self.h, i, ptr(scratch), scratch.numel() * scratch.element_size(), flags,
+                                      ptr(packed), stream_ptr(stream)), "vox_gguf_upload_q4")

@@ -288,6 +288,43 @@ vox_status vox_window_attn(const void *q, int64_t ldq, const void *k_hist, const
 vox_status vox_rmsnorm(const float *x, int64_t m, int64_t n, int64_t ldx, float eps,
                        const float *g, void *out, int32_t out_dtype, int64_t ldo, void *stream);
 
+/* ------------------------------------------------------------ GGUF files
+ * [Q4]: the pages' quantised weights ship as a GGUF file with Q4_0 tensors.
+ * vox_gguf_open reads a GGUF (version 2 or 3) file into host memory and
+ * indexes its metadata and tensors; the handle owns that copy until
+ * vox_gguf_close.  Bounds are checked against the file size: a truncated or
+ * malformed file -> VOX_ERR_SHAPE (bad magic, version, counts or tensor
+ * infos), VOX_ERR_ALIGN (a tensor offset off the file's alignment) or
+ * VOX_ERR_RANGE (a tensor past the end, or the file cannot be read).
+ * Tensor dims are innermost first: a weight of n rows x k columns has
+ * dims = {k, n}.  Element types: 0 f32, 1 f16, 2 Q4_0; tensors of other
+ * types are listed with nbytes = 0 and no data pointer. */
+typedef struct vox_gguf vox_gguf;
+vox_status vox_gguf_open(const char *path, vox_gguf **out);
+void vox_gguf_close(vox_gguf *g);
+int64_t vox_gguf_tensor_count(const vox_gguf *g);                 /* -1 for NULL          */
+int64_t vox_gguf_find_tensor(const vox_gguf *g, const char *name); /* index, or -1         */
+/* name, element type, dimension count, dims[4] (unused ones 1) and data bytes
+ * of tensor i; any output pointer may be NULL.  i out of range ->
+ * VOX_ERR_RANGE. */
+vox_status vox_gguf_tensor_info(const vox_gguf *g, int64_t i, const char **name, int32_t *type,
+                                int32_t *n_dims, int64_t *dims, uint64_t *nbytes);
+/* Host pointer to tensor i's bytes inside the handle, or NULL. */
+const void *vox_gguf_tensor_data(const vox_gguf *g, int64_t i);
+/* Metadata by key: integers and bools, floats, strings (NULL if absent or
+ * not a string).  Missing key -> VOX_ERR_RANGE, other type -> VOX_ERR_DTYPE. */
+vox_status vox_gguf_get_int(const vox_gguf *g, const char *key, int64_t *value);
+vox_status vox_gguf_get_float(const vox_gguf *g, const char *key, double *value);
+const char *vox_gguf_get_string(const vox_gguf *g, const char *key);
+/* Upload Q4_0 tensor i (dims {k, n}) and repack it like vox_q4_pack: its
+ * GGUF blocks are copied host -> device into scratch (device, at least the
+ * tensor's nbytes; the call returns once the host bytes are staged), then
+ * packed into `packed` (device, vox_q4_packed_bytes(n, k) bytes, 16-byte
+ * aligned) on `stream`.  Not Q4_0 -> VOX_ERR_DTYPE; more than 2 dims ->
+ * VOX_ERR_SHAPE; short scratch -> VOX_ERR_WORKSPACE; flags as vox_q4_pack. */
+vox_status vox_gguf_upload_q4(const vox_gguf *g, int64_t i, void *scratch, size_t scratch_bytes, int32_t flags,
+                              void *packed, void *stream);
+
 /* ------------------------------------------------------------ composed path
  * The decoder token step and the encoder chunk, built from the calls above
  * and launched back to back on one stream (the pages' "one submission per
