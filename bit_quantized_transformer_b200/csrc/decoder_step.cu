@@ -86,7 +86,7 @@ struct PsArgs {
     int32_t n_layers, dim, q_dim, kv_dim, ffn, vocab, n_kv, group, window;
     float eps, qscale;
     uint32_t act_bytes;                      // shared bytes of the activation / merge region
-    int32_t test_withhold;                   // test hook: warp 0 of CTA 0 waits for a stage never issued
+    int32_t test_withhold;                   // test hook: warp 0 of CTA 0 first waits on a barrier nothing completes
 };
 
 // ------------------------------------------------------------ workspace
@@ -145,16 +145,24 @@ __host__ __device__ inline PsSmem ps_smem_layout(uint32_t act_bytes)
 }
 
 // ------------------------------------------------------------ helpers
+// floor(num / den) for non-negative operands, in 32 bits when they fit
+// (64-bit division is a long software sequence on the GPU).
+__device__ __forceinline__ int64_t udiv(uint64_t num, uint64_t den)
+{
+    if (num < (1ull << 32) && den < (1ull << 32)) return (int64_t)((uint32_t)num / (uint32_t)den);
+    return (int64_t)(num / den);
+}
+
 __device__ __forceinline__ int64_t split_begin(int64_t b, int64_t total, int64_t parts)
 {
-    return b * total / parts;
+    return udiv((uint64_t)b * (uint64_t)total, (uint64_t)parts);
 }
 
 // Part holding item c when `total` items are split into `parts` ranges
 // [split_begin(b), split_begin(b + 1)) (the last non-empty one at or before c).
 __device__ __forceinline__ int64_t split_owner(int64_t c, int64_t total, int64_t parts)
 {
-    return ((c + 1) * parts - 1) / total;
+    return udiv((uint64_t)(c + 1) * (uint64_t)parts - 1, (uint64_t)total);
 }
 
 __device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p)
@@ -309,8 +317,8 @@ __device__ __forceinline__ bool ps_grid_barrier(const PsArgs& P, const PsWs& W, 
         __threadfence();
         const uint64_t old = atomicAdd(reinterpret_cast<unsigned long long*>(ctr), 1ull);
         const uint64_t target = (old / G + 1) * G;
-        int ok = 1;
-        if (ld_acquire_u64(ctr) < target) {
+        int ok = ld_relaxed_s32(abort) ? 0 : 1;               // another CTA already gave up
+        if (ok && ld_acquire_u64(ctr) < target) {
             const uint64_t t0 = global_ns();
             for (;;) {
                 bool done = false;
@@ -502,15 +510,6 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
         float acc0 = 0.f, acc2 = 0.f;
         int64_t r = wb;
         for (int j = 0; j < f.nst; ++j) {
-            if (P.test_withhold && ph == 0 && j == 0 && b == 0 && warp == 0) {
-                // test hook: a wait that can only run out (its stage is never issued)
-                uint64_t* never = reinterpret_cast<uint64_t*>(smem + SL.never);
-                if (!mbar_wait_bounded(never, 0, 0x530)) {
-                    ok = false;
-                    ps_raise(P, W, 0x530);
-                    break;
-                }
-            }
             if (!ps_ring_wait(ring, 0x501)) {
                 ok = false;
                 ps_raise(P, W, 0x501);
@@ -523,7 +522,7 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     const int ri = q0 + u < nrec ? q0 + u : q0;      // a missing second record repeats the first
-                    const int ch = (cin + u) % kc;
+                    const int ch = cin + u < kc ? cin + u : cin + u - kc;
                     const uint4 qv = lds128(base + ri * kChunkBytes + 16 * lane);
                     const uint2 e = lds64(base + ri * kChunkBytes + kChunkQsBytes + 8 * g);
                     p[u][0] = p[u][1] = p[u][2] = p[u][3] = 0.f;
@@ -915,6 +914,13 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
     ps_ring_fill(P, ring, nph, b, G, warp, lane, nch);
 
     bool ok = true;
+    if (P.test_withhold && b == 0 && warp == 0) {
+        // test hook: a wait that can only run out (a barrier nothing completes)
+        if (!mbar_wait_bounded(reinterpret_cast<uint64_t*>(smem + SL.never), 0, 0x530)) {
+            ok = false;
+            ps_raise(P, W, 0x530);
+        }
+    }
     PsBest best = {-INFINITY, 0x7fffffff};
     int ph = 0;
     for (; ph < nph; ++ph) {

@@ -2,10 +2,10 @@
 without faulting or hanging the GPU.
 
 With the test hook VOX_TEST_WITHHOLD_STAGE=1 (read by vox_decoder_step at
-launch), warp 0 of CTA 0 first waits on a ring stage that is never issued.
-That wait gives up after about one second, records 0x530 in the device status
-word and raises the abort flag, so every other CTA leaves its grid barrier
-early; the launch returns and the context stays usable.  After the workspace
+launch), warp 0 of CTA 0 first waits on an mbarrier that nothing ever
+completes.  That wait gives up after about one second, records 0x530 in the
+device status word and raises the abort flag, so every other CTA leaves its
+grid barrier early; the launch returns and the context stays usable.  After the workspace
 is zeroed again and the state restored, the next step is correct."""
 import os
 import time
