@@ -517,19 +517,30 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
             }
             const uint32_t base = smem_addr(ring.base) + (ring.consumed % kPsStages) * kPsStageBytes + smem_token();
             const int nrec = (int)min64(kPsRecs, we - r);
-            for (int q0 = 0; q0 < nrec; q0 += 2) {
-                float p[2][4];
+            for (int q0 = 0; q0 < nrec; q0 += 4) {
+                // four records' MMAs back to back (a missing record repeats the
+                // stage's first; its result is not used), then their bookkeeping
+                float p[4][4];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int ri = q0 + u < nrec ? q0 + u : q0;      // a missing second record repeats the first
-                    const int ch = cin + u < kc ? cin + u : cin + u - kc;
+                for (int u = 0; u < 4; ++u) {
+                    const int ri = q0 + u < nrec ? q0 + u : q0;
+                    int ch = cin + u;
+                    while (ch >= kc) ch -= kc;
                     const uint4 qv = lds128(base + ri * kChunkBytes + 16 * lane);
                     const uint2 e = lds64(base + ri * kChunkBytes + kChunkQsBytes + 8 * g);
                     p[u][0] = p[u][1] = p[u][2] = p[u][3] = 0.f;
                     gemv_record<1>(qv, e, bs_a, cb_a, nblk, ch, 1, 0, t, p[u]);
                 }
+                if (q0 + 4 <= nrec && cin + 4 < kc && r + 4 < we) {
+                    // no tile end and no range end among the four: pairwise sum
+                    acc0 += (p[0][0] + p[1][0]) + (p[2][0] + p[3][0]);
+                    acc2 += (p[0][2] + p[1][2]) + (p[2][2] + p[3][2]);
+                    cin += 4;
+                    r += 4;
+                    continue;
+                }
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
+                for (int u = 0; u < 4; ++u) {
                     if (q0 + u >= nrec) break;
                     acc0 += p[u][0];
                     acc2 += p[u][2];
@@ -845,25 +856,52 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
             }
             named_barrier(1, kPsThreads);
             if (*reinterpret_cast<volatile int32_t*>(s_flag)) {
+                // last CTA of the head: fold the CTAs' records in CTA order.  Pass 1
+                // loads every (record, head) (m, l) pair at once; the factors
+                // exp2(m - M) replace m in shared memory; pass 2 streams the O rows
+                // eight records per round.
                 __threadfence();
                 const float* base = recs + (size_t)hh * W.rmax * W.rec_floats;
+                const int nrec = (int)(lc - fc + 1);
+                float* s_ml = merge;                              // [nrec][group] x (m or factor, l)
+                float* s_L = merge + 2 * nrec * group;
+                for (int i = tid; i < nrec * group; i += kPsThreads) {
+                    const int r = i / group, hi = i - r * group;
+                    float2 ml = make_float2(-INFINITY, 0.f);        // a CTA with no units wrote no record
+                    if (split_begin(fc + r, f.R, G) < split_begin(fc + r + 1, f.R, G))
+                        ml = __ldcg(reinterpret_cast<const float2*>(base + (size_t)r * W.rec_floats + group * kPsHd) + hi);
+                    s_ml[2 * i] = ml.x;
+                    s_ml[2 * i + 1] = ml.y;
+                }
+                named_barrier(1, kPsThreads);
+                if (tid < group) {
+                    float M = -INFINITY, L = 0.f;
+                    for (int r = 0; r < nrec; ++r) M = fmaxf(M, s_ml[2 * (r * group + tid)]);
+                    for (int r = 0; r < nrec; ++r) {
+                        const float mv = s_ml[2 * (r * group + tid)];
+                        const float fct = (mv == -INFINITY) ? 0.f : exp2f(mv - M);
+                        s_ml[2 * (r * group + tid)] = fct;
+                        L += fct * s_ml[2 * (r * group + tid) + 1];
+                    }
+                    s_L[tid] = L;
+                }
+                named_barrier(1, kPsThreads);
                 for (int i = tid; i < group * kPsHd; i += kPsThreads) {
                     const int hi = i / kPsHd, cc = i - hi * kPsHd;
-                    float M = -INFINITY;
-                    for (int64_t c = fc; c <= lc; ++c) {
-                        if (split_begin(c, f.R, G) >= split_begin(c + 1, f.R, G)) continue;
-                        M = fmaxf(M, __ldcg(base + (size_t)(c - fc) * W.rec_floats + group * kPsHd + hi * 2));
+                    float O = 0.f;
+                    for (int r0 = 0; r0 < nrec; r0 += 8) {
+                        float v[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            v[u] = r0 + u < nrec ? __ldcg(base + (size_t)(r0 + u) * W.rec_floats + hi * kPsHd + cc) : 0.f;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            if (r0 + u >= nrec) break;
+                            const float fct = s_ml[2 * ((r0 + u) * group + hi)];
+                            O += fct != 0.f ? fct * v[u] : 0.f;     // an empty CTA's slot may hold anything
+                        }
                     }
-                    float O = 0.f, L = 0.f;
-                    for (int64_t c = fc; c <= lc; ++c) {
-                        if (split_begin(c, f.R, G) >= split_begin(c + 1, f.R, G)) continue;
-                        const float* rc = base + (size_t)(c - fc) * W.rec_floats;
-                        const float mv = __ldcg(rc + group * kPsHd + hi * 2);
-                        const float fct = (mv == -INFINITY) ? 0.f : exp2f(mv - M);
-                        O += fct * __ldcg(rc + hi * kPsHd + cc);
-                        L += fct * __ldcg(rc + group * kPsHd + hi * 2 + 1);
-                    }
-                    P.attn[(hh * group + hi) * kPsHd + cc] = O / L;
+                    P.attn[(hh * group + hi) * kPsHd + cc] = O / s_L[hi];
                 }
             }
         }
@@ -915,8 +953,13 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
 
     bool ok = true;
     if (P.test_withhold && b == 0 && warp == 0) {
-        // test hook: a wait that can only run out (a barrier nothing completes)
-        if (!mbar_wait_bounded(reinterpret_cast<uint64_t*>(smem + SL.never), 0, 0x530)) {
+        // test hook: a wait that can only run out (an mbarrier nothing completes),
+        // bounded at 0.2 s so that it gives up before any grid barrier would
+        uint64_t* never = reinterpret_cast<uint64_t*>(smem + SL.never);
+        const uint64_t t0 = global_ns();
+        bool done = false;
+        while (!done && global_ns() - t0 < 200000000ull) done = mbar_test_wait(never, 0);
+        if (!done) {
             ok = false;
             ps_raise(P, W, 0x530);
         }
