@@ -59,8 +59,9 @@ def parse_args(argv=None):
                         "and its GEMMs; sweep: the decoder shapes at M in {1,4,16,64,256} and the attention at "
                         "KV in {512, 4096, 8192 wrapped}; kernel: a few launches of one kernel on one small "
                         "case (--kernel, --shape, --launches), sized for an ncu capture")
-    p.add_argument("--kernel", choices=["gemv", "attn", "gemm"], default="gemv",
-                   help="kernel workload: gemv N K (M = 1), attn POS (decoder-shaped layer), gemm N K M")
+    p.add_argument("--kernel", choices=["gemv", "attn", "gemm", "step"], default="gemv",
+                   help="kernel workload: gemv N K (M = 1), attn POS (decoder-shaped layer), gemm N K M, "
+                        "step L (the persistent decoder step with L full-size layers, KV 8192 wrapped)")
     p.add_argument("--shape", type=int, nargs="*", default=None)
     p.add_argument("--launches", type=int, default=4)
     return p.parse_args(argv)
@@ -817,8 +818,15 @@ def run_kernel_case(args):
     from bit_quantized_transformer_b200 import vox as V
     from bit_quantized_transformer_b200 import workloads as WL
 
-    shp = args.shape or {"gemv": [4096, 3072], "attn": [8492], "gemm": [131072, 3072, 256]}[args.kernel]
-    if args.kernel == "gemv":
+    shp = args.shape or {"gemv": [4096, 3072], "attn": [8492], "gemm": [131072, 3072, 256], "step": [2]}[args.kernel]
+    if args.kernel == "step":
+        shape = synth.DecoderShape(n_layers=shp[0])
+        dm = WL.DecoderModel(shape, seed=0, filled=FILLED, token=17)
+        for _ in range(args.launches):
+            dm.step()
+        what = {"kernel": "decoder_step_kernel", "layers": shp[0],
+                "bytes_per_launch": dm.weight_bytes() + dm.kv_bytes(FILLED)}
+    elif args.kernel == "gemv":
         n, k = shp[0], shp[1]
         qs, d = synth.q4_blocks(n, k, 0, 77)
         packed, w = WL.pack_q4(qs, d, "cuda")

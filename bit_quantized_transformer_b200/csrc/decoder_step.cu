@@ -517,30 +517,21 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
             }
             const uint32_t base = smem_addr(ring.base) + (ring.consumed % kPsStages) * kPsStageBytes + smem_token();
             const int nrec = (int)min64(kPsRecs, we - r);
-            for (int q0 = 0; q0 < nrec; q0 += 4) {
-                // four records' MMAs back to back (a missing record repeats the
-                // stage's first; its result is not used), then their bookkeeping
-                float p[4][4];
+            for (int q0 = 0; q0 < nrec; q0 += 2) {
+                // two records' MMAs back to back (a missing second record repeats
+                // the first; its result is not used), then their bookkeeping
+                float p[2][4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     const int ri = q0 + u < nrec ? q0 + u : q0;
-                    int ch = cin + u;
-                    while (ch >= kc) ch -= kc;
+                    const int ch = cin + u < kc ? cin + u : cin + u - kc;
                     const uint4 qv = lds128(base + ri * kChunkBytes + 16 * lane);
                     const uint2 e = lds64(base + ri * kChunkBytes + kChunkQsBytes + 8 * g);
                     p[u][0] = p[u][1] = p[u][2] = p[u][3] = 0.f;
                     gemv_record<1>(qv, e, bs_a, cb_a, nblk, ch, 1, 0, t, p[u]);
                 }
-                if (q0 + 4 <= nrec && cin + 4 < kc && r + 4 < we) {
-                    // no tile end and no range end among the four: pairwise sum
-                    acc0 += (p[0][0] + p[1][0]) + (p[2][0] + p[3][0]);
-                    acc2 += (p[0][2] + p[1][2]) + (p[2][2] + p[3][2]);
-                    cin += 4;
-                    r += 4;
-                    continue;
-                }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     if (q0 + u >= nrec) break;
                     acc0 += p[u][0];
                     acc2 += p[u][2];
