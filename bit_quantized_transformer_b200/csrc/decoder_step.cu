@@ -54,11 +54,17 @@
 
 namespace vox {
 
-constexpr int kPsWarps = 8;
+#ifndef VOX_PS_WARPS
+#define VOX_PS_WARPS 12
+#endif
+#ifndef VOX_PS_STAGES
+#define VOX_PS_STAGES 4
+#endif
+constexpr int kPsWarps = VOX_PS_WARPS;
 constexpr int kPsThreads = 32 * kPsWarps;
-constexpr int kPsStages = 3;
-constexpr int kPsStageBytes = 8192;
-constexpr int kPsRecs = kPsStageBytes / kChunkBytes;       // 14 records per GEMV stage
+constexpr int kPsStages = VOX_PS_STAGES;
+constexpr int kPsStageBytes = 4096;                          // one K or V half of an attention unit
+constexpr int kPsRecs = kPsStageBytes / kChunkBytes;       // 7 records per GEMV stage
 constexpr int kPsMaxLayers = 32;
 constexpr int kPsUnit = 16;                                  // cache slots per attention unit
 constexpr int kPsHd = 128;
@@ -220,8 +226,8 @@ __device__ __forceinline__ PsPhase ps_phase(const PsArgs& P, int ph, int64_t b, 
         f.cb = split_begin(b, f.R, G);
         f.ce = split_begin(b + 1, f.R, G);
         f.wb = f.we = 0;
-        const int64_t mine = f.ce - f.cb - warp;               // units cb + warp + 8j
-        f.nst = mine > 0 ? (int32_t)((mine + kPsWarps - 1) / kPsWarps) : 0;
+        const int64_t mine = f.ce - f.cb - warp;               // units cb + warp + kPsWarps * j
+        f.nst = mine > 0 ? 2 * (int32_t)((mine + kPsWarps - 1) / kPsWarps) : 0;   // a K and a V stage each
     } else {
         f.kc = (int32_t)((f.k + 63) / 64);
         f.R = ((f.n + 15) / 16) * f.kc;
@@ -258,14 +264,14 @@ __device__ __forceinline__ void ps_issue(const PsArgs& P, const PsCursor& c, int
 {
     const PsPhase& f = c.f;
     if (f.kind == PS_ATTN) {
-        const int64_t unit = f.cb + warp + (int64_t)kPsWarps * c.idx;
+        // stage 2u: the K rows of the warp's unit u, stage 2u + 1: its V rows
+        const int64_t unit = f.cb + warp + (int64_t)kPsWarps * (c.idx >> 1);
         const int64_t hh = unit / nch, ci = unit - hh * nch;
         const int32_t row = (int32_t)(hh * P.window + ci * kPsUnit);
+        const CUtensorMap* map = (c.idx & 1) ? &P.vmap[f.layer] : &P.kmap[f.layer];
         mbar_arrive_expect_tx(bar, kPsStageBytes);
-        tma_load_2d(dst + 0, &P.kmap[f.layer], 0, row, bar);
-        tma_load_2d(dst + 2048, &P.kmap[f.layer], 64, row, bar);
-        tma_load_2d(dst + 4096, &P.vmap[f.layer], 0, row, bar);
-        tma_load_2d(dst + 6144, &P.vmap[f.layer], 64, row, bar);
+        tma_load_2d(dst + 0, map, 0, row, bar);
+        tma_load_2d(dst + 2048, map, 64, row, bar);
     } else {
         const int64_t r0 = f.wb + (int64_t)kPsRecs * c.idx;
         const uint32_t bytes = (uint32_t)min64(kPsRecs, f.we - r0) * kChunkBytes;
@@ -295,11 +301,11 @@ __device__ __forceinline__ void ps_ring_fill(const PsArgs& P, PsRing& r, int nph
     }
 }
 
-// Wait for the next stage of the ring; returns its shared address (0 on failure).
-__device__ __forceinline__ bool ps_ring_wait(PsRing& r, int32_t where)
+// Wait for stage consumed + ahead of the ring; false if the wait gave up.
+__device__ __forceinline__ bool ps_ring_wait(PsRing& r, int32_t where, uint32_t ahead = 0)
 {
-    const uint32_t slot = r.consumed % kPsStages;
-    const uint32_t parity = (r.consumed / kPsStages) & 1u;
+    const uint32_t slot = (r.consumed + ahead) % kPsStages;
+    const uint32_t parity = ((r.consumed + ahead) / kPsStages) & 1u;
     return mbar_wait_bounded(&r.bars[slot], parity, where);
 }
 
@@ -645,7 +651,7 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
         for (int jj = 0; jj < 8; ++jj) o[jj][0] = o[jj][1] = o[jj][2] = o[jj][3] = 0.f;
         uint32_t qh[8][2], ql[8][2];
         bool have_q = false;
-        while (ok && j < f.nst) {
+        while (ok && j < f.nst / 2) {
             const int64_t unit = f.cb + warp + (int64_t)kPsWarps * j;
             if (unit / nch != hh) break;
             if (!have_q) {
@@ -666,14 +672,14 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
                 }
                 have_q = true;
             }
-            if (!ps_ring_wait(ring, 0x502)) {
+            if (!ps_ring_wait(ring, 0x502) || !ps_ring_wait(ring, 0x502, 1)) {
                 ok = false;
                 ps_raise(P, W, 0x502);
                 break;
             }
-            const uint32_t slot_s = ring.consumed % kPsStages;
-            uint8_t* stp = ring.base + slot_s * kPsStageBytes;
-            const uint32_t st = smem_addr(stp);
+            uint8_t* stK = ring.base + (ring.consumed % kPsStages) * kPsStageBytes;
+            uint8_t* stV = ring.base + ((ring.consumed + 1) % kPsStages) * kPsStageBytes;
+            const uint32_t sK = smem_addr(stK), sV = smem_addr(stV);
             const int64_t slot0 = (unit - hh * nch) * kPsUnit;   // first cache slot of the unit
 
             // generic-proxy fix-ups of the TMA-written stage
@@ -685,15 +691,16 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
                 const uint16_t* src = (part < 2 ? P.kc[l] : P.vc[l]) + (hh * Wn + new_slot) * kPsHd + (part & 1) * 64 +
                                       u8 * 8;
                 const uint4 v = __ldcg(reinterpret_cast<const uint4*>(src));
-                *reinterpret_cast<uint4*>(stp + part * 2048 + sw128_offset(rr, (uint32_t)u8)) = v;
+                *reinterpret_cast<uint4*>((part < 2 ? stK : stV) + (part & 1) * 2048 + sw128_offset(rr, (uint32_t)u8)) =
+                    v;
                 touched = true;
             }
             if (slot0 + kPsUnit > n_valid) {
                 // slots past the valid range may hold anything (NaN included): zero their V rows
                 for (int i = lane; i < 16 * 16; i += 32) {
-                    const int rr = i >> 4, part = 2 + ((i >> 3) & 1), u8 = i & 7;
+                    const int rr = i >> 4, half = (i >> 3) & 1, u8 = i & 7;
                     if (slot0 + rr >= n_valid)
-                        *reinterpret_cast<uint4*>(stp + part * 2048 + sw128_offset((uint32_t)rr, (uint32_t)u8)) =
+                        *reinterpret_cast<uint4*>(stV + half * 2048 + sw128_offset((uint32_t)rr, (uint32_t)u8)) =
                             make_uint4(0u, 0u, 0u, 0u);
                 }
                 touched = true;
@@ -709,7 +716,7 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
                 const uint32_t rr = (uint32_t)(8 * (mi & 1) + (lane & 7));
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t tile = st + (kk >> 2) * 2048;
+                    const uint32_t tile = sK + (kk >> 2) * 2048;
                     uint32_t ak[4];
                     ldsm_x4(ak, tile + sw128_offset(rr, (uint32_t)(2 * (kk & 3) + (mi >> 1))));
                     mma_bf16_16816(sa[(kk & 1) * 2 + 0], ak, qh[kk][0], qh[kk][1], sa[(kk & 1) * 2 + 0]);
@@ -764,7 +771,7 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
                 const uint32_t rr = (uint32_t)(8 * (mi >> 1) + (lane & 7));
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
-                    const uint32_t tile = st + (2 + (jj >> 2)) * 2048;
+                    const uint32_t tile = sV + (jj >> 2) * 2048;
                     uint32_t av[4];
                     ldsm_x4_trans(av, tile + sw128_offset(rr, (uint32_t)(2 * (jj & 3) + (mi & 1))));
                     float c[4] = {o[jj][0] * corr[0], o[jj][1] * corr[1], o[jj][2] * corr[0], o[jj][3] * corr[1]};
@@ -779,7 +786,7 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
             // generic writes into a buffer the async proxy refills next: order them first
             if (touched) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
-            ++ring.consumed;
+            ring.consumed += 2;
             ++j;
             ps_ring_fill(P, ring, nph, b, G, warp, lane, nch);
         }

@@ -20,8 +20,11 @@
 //               (g, t) its 16 bytes of codes (rows g and g+8, both 32-column
 //               blocks); each 32-bit word gives four bf16 pairs 128 + q by
 //               OR-ing the nibble into the fraction of 128.0 (exact), then
-//               one exact subtraction of 136 and one multiply by d (one
-//               rounding to bf16), stored in the canonical K-major
+//               an exact subtraction of 136 gives q - 8, which is widened to
+//               fp32 and multiplied by d in fp32 (exact: 4 x 11 significant
+//               bits), and the product is rounded to bf16 once (nearest
+//               even) -- the same bits vox_q4_dequant returns -- and stored
+//               in the canonical K-major
 //               128-byte-swizzled layout the MMA reads (4-byte stores, free of
 //               bank conflicts); after the last chunk they read the
 //               accumulator with tcgen05.ld and run the epilogue (residual
@@ -98,18 +101,11 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8])
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// bf16x2 a - b and a * b, one rounding each (b exact in the subtraction here).
+// bf16x2 a - b (exact here: both are small integers).
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b)
 {
     uint32_t d;
     asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
@@ -212,11 +208,10 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
                 const uint8_t* rec = st + C::xbytes + kGemmABytes + dw * kChunkBytes;
                 const uint4 qv = *reinterpret_cast<const uint4*>(rec + 16 * lane);
                 const uint2 dd = *reinterpret_cast<const uint2*>(rec + kChunkQsBytes + 8 * g);
-                // scales as bf16 pairs: d(row g, block 0), d(row g+8, block 0), d(g, 1), d(g+8, 1)
+                // scales in fp32 (exact): d(row g, block 0), d(row g+8, block 0), d(g, 1), d(g+8, 1)
                 const float2 d0 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
                 const float2 d1 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
-                const uint32_t D[4] = {pack_bf16x2(d0.x, d0.x), pack_bf16x2(d0.y, d0.y), pack_bf16x2(d1.x, d1.x),
-                                       pack_bf16x2(d1.y, d1.y)};
+                const float D[4] = {d0.x, d0.y, d1.x, d1.y};
 #pragma unroll
                 for (int bb = 0; bb < 2; ++bb) {
 #pragma unroll
@@ -227,7 +222,10 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
 #pragma unroll
                         for (int h = 0; h < 4; ++h) {
                             const uint32_t raw = lop3_and_or(src[h], M_L, C_B);            // 128 + q, exact
-                            const uint32_t v = bf16x2_mul(bf16x2_sub(raw, B136), D[bb * 2 + (h & 1)]);
+                            const uint32_t qm = bf16x2_sub(raw, B136);          // q - 8, exact
+                            const float dd_ = D[bb * 2 + (h & 1)];
+                            const uint32_t v = pack_bf16x2(__uint_as_float(qm << 16) * dd_,
+                                                           __uint_as_float(qm & 0xFFFF0000u) * dd_);
                             const uint32_t row = (h & 1) ? row_g8 : row_g;
                             // columns 32 bb + 16 (h >> 1) + 8 wi + 2t, +1: unit 4 bb + 2 (h >> 1) + wi
                             const uint32_t unit = (uint32_t)(bb * 4 + (h >> 1) * 2 + wi);

@@ -472,6 +472,29 @@ def test_gemm_parity(env, n, k, m):
     assert err <= TOL, err
 
 
+def test_gemm_weights_round_once(env):
+    """With one-hot activation rows (X = I), the GEMM's output is the bf16
+    weight tile the kernel staged in shared memory, widened exactly: it must
+    equal vox_q4_dequant's bf16 weights (round-to-nearest-even of the exact
+    (q - 8) d) bit for bit, including scales whose products need rounding."""
+    torch, V, WL = env
+    n, k = 256, 128
+    qs, d = synth.q4_blocks(n, k, 0, 9901)
+    d = d.copy()
+    d[::3] = synth.fp16_bits(np.linspace(0.0011, 0.0117, d[::3].size)).reshape(d[::3].shape)   # 11-bit scales
+    packed, w = WL.pack_q4(qs, d, "cuda")
+    X = torch.eye(k, dtype=torch.bfloat16, device="cuda")
+    Y = torch.full((k, n), float("nan"), dtype=torch.float32, device="cuda")
+    V.vox_q4_gemm(w, X, V.VOX_BF16, k, k, Y, V.VOX_F32, n)
+    Wb = torch.empty(n, k, dtype=torch.bfloat16, device="cuda")
+    V.vox_q4_dequant(w, 0, n, Wb, V.VOX_BF16, k)
+    check_status(V)
+    got = Y.cpu().numpy().T                                  # [n][k]
+    want = ref.bf16_to_f64(bf16_bits(Wb)).astype(np.float32)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    assert np.array_equal(bf16_bits(Wb), ref.c_dequant_bf16(qs, d))
+
+
 def test_gemm_epilogues(env):
     torch, V, WL = env
     n, k, m = 1280, 5120, 256
