@@ -537,6 +537,25 @@ def run_encoder(args):
     peak = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
         os.path.join(ROOT, "MEASURED_PEAKS.json")) else {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
     tf_g = flops / (ms_g / 1e3) / 1e12
+    cpu = None
+    if not args.no_cpu_baseline:
+        import numpy as np
+
+        from oracle import ref
+
+        w0 = synth.encoder_layer_weights(shape, 0, 0)
+        mats = [ref.q4_weights(*w0[k]) for k in ("wqkv", "wo", "wup", "wdown")]
+        xs = [np.asarray(synth.activations(R, m.shape[1], 0, 90 + i), np.float64) for i, m in enumerate(mats)]
+        t0 = time.perf_counter()
+        fl = 0
+        while time.perf_counter() - t0 < min(args.cpu_seconds, 10.0):
+            for x_, m_ in zip(xs, mats):
+                x_ @ m_.T
+                fl += 2 * x_.shape[0] * m_.shape[0] * m_.shape[1]
+        dt = time.perf_counter() - t0
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": omp_threads(), "kind": "oracle",
+               "sample": f"encoder layer 0's four GEMMs at M = {R} (fp64 numpy matmul on the exactly dequantised "
+                         f"weights, the oracle's route), {fl / 1e9:.0f} GFLOP in {dt:.1f} s"}
     line = {"metric": "encoder chunk Q4_0 GEMM TFLOP/s (bf16 tensor cores)", "value": tf_g, "unit": "TFLOP/s",
             "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": ms_g,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 MMA, f32 accumulate",
@@ -547,7 +566,7 @@ def run_encoder(args):
                          "frac": tf_g / peak["bf16_tflops"], "frac_of_sustained": tf_g / peak["bf16_tflops_sustained"],
                          "traffic": None},
             "chunk_ms": ms, "chunk_tflops_gemm_only_numerator": flops / (ms / 1e3) / 1e12,
-            "gpu_launches": len(calls) * steps}
+            "gpu_launches": len(calls) * steps, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -586,8 +605,15 @@ def run_sweep(args):
         keep = [packed] + [packed.clone() for _ in range(copies - 1)]
         wts = [V.weight(t, n, k) for t in keep]
         res = {}
-        for M in Ms + ["16_gemv"]:
-            if M == "16_gemv":
+        for M in Ms + ["16_gemv"] + [f"matmul_{mm}" for mm in Ms]:
+            if isinstance(M, str) and M.startswith("matmul_"):
+                mm = int(M.split("_")[1])
+                wsm = torch.zeros(V.vox_q4_matmul_workspace(wts[0], mm, None), dtype=torch.uint8, device="cuda")
+
+                def fn(mm=mm, wsm=wsm):
+                    for w in wts:
+                        V.vox_q4_matmul(w, x32, mm, 9216, y, n, None, wsm, wsm.numel())
+            elif M == "16_gemv":
                 def fn():
                     for w in wts:
                         for h in range(2):
@@ -603,7 +629,7 @@ def run_sweep(args):
             g = graph_of(fn)
             g.replay()
             us = time_replays(g, reps, 1) / (reps * copies) * 1e3
-            m = 16 if M == "16_gemv" else M
+            m = 16 if M == "16_gemv" else (int(M.split("_")[1]) if isinstance(M, str) else M)
             res[str(M)] = {"us": us, "weight_gbs": nbytes / us / 1e3, "tflops": 2 * m * n * k / us / 1e6}
             del g
         out[f"{n}x{k}"] = res
@@ -633,13 +659,18 @@ def run_sweep(args):
         attn[str(min(pos + 1, W)) + (" wrapped" if pos >= W else "")] = {"us_per_layer": us, "gbs": nb / us / 1e3}
         del g
     assert V.vox_device_status(True) == 0
+    peak, peak_src = measured_peaks()
+    lm1 = out["131072x3072"]["1"]["weight_gbs"]
     line = {"metric": "decoder-shape sweep: weight GB/s and TFLOP/s per M; attention GB/s per KV length",
             "value": out["131072x3072"]["1"]["weight_gbs"], "unit": "GB/s", "n_gpus": 1, "steps": reps,
             "warmup": 1, "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "q4_0 weights; fp16 (K1) / bf16 (K2) tensor-core inputs; f32 accumulate", "data": "synthetic",
             "config": {"workload": "decoder_shapes_M_sweep_and_attention_kv_sweep", "M": Ms,
                        "l2": "weight copies > 2x L2 per shape"},
-            "sweep": out, "crossover": cross, "attention": attn}
+            "sweep": out, "crossover": cross, "attention": attn,
+            "roofline": {"bound": "hbm", "kernel": "q4_gemv_kernel (LM head, M = 1)", "achieved": lm1, "peak": peak,
+                         "unit": "GB/s", "frac": lm1 / peak, "traffic": None, "peak_source": peak_src},
+            "dispatch": "vox_q4_matmul: the GEMV for M <= 8, the tcgen05 GEMM above (entries matmul_M)"}
     print(json.dumps(line), flush=True)
     return 0
 

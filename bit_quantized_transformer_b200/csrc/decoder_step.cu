@@ -19,24 +19,25 @@
 // "Arquitetura") is dequantised in registers inside the products.
 //
 // Design (B200, HBM-bound at M = 1):
-//  * One CTA per SM, 8 warps.  Every warp owns a ring of 3 shared-memory
-//    stages of 8 KB in which its lane 0 keeps bulk (TMA) copies in flight.
+//  * One CTA per SM, 12 warps.  Every warp owns a ring of 4 shared-memory
+//    stages of 4 KB in which its lane 0 keeps bulk (TMA) copies in flight.
 //    The ring is one continuous stream across phases: once a warp has
 //    consumed its last stage of a phase it immediately issues the first
 //    stages of the next phase (weights and old cache rows never depend on
 //    this step's activations), so HBM stays busy while the CTA waits at the
 //    grid barrier.
-//  * GEMV phases: the (16-row tile, 64-column chunk) records of the packed
-//    matrix are split evenly over CTAs and, inside a CTA, over warps
-//    (stream-K); a GEMV stage is up to 14 records (8064 bytes).  A tile a
-//    warp covers alone is finished from its registers; a tile cut between
-//    warps is summed in warp order from shared memory; a tile cut between
-//    CTAs is summed in CTA order from global memory by the last CTA to
-//    arrive (per-tile arrival counter).  All sums have a fixed order: the
-//    result does not depend on timing.
+//  * GEMV phases: every CTA owns a contiguous run of whole 16-row tiles of
+//    the packed matrix (at most one tile more than another), and inside a
+//    CTA the run's (tile, 64-column chunk) records are split evenly over the
+//    warps (stream-K); a GEMV stage is up to 7 records (4032 bytes).  A tile
+//    a warp covers alone is finished from its registers; a tile cut between
+//    warps is summed in warp order from shared memory.  Residuals are loaded
+//    before the main loop.  All sums have a fixed order: the result does not
+//    depend on timing.
 //  * ATTN phases: 16-slot units (kv head, slots) are split evenly over CTAs;
-//    inside a CTA the warps take units round robin, each unit one stage of
-//    four 2-D TMA boxes (K and V, 64 columns x 16 rows, 128-byte swizzle).
+//    inside a CTA the warps take units round robin, each unit two stages
+//    (its K rows, then its V rows) of two 2-D TMA boxes each (64 columns x
+//    16 rows, 128-byte swizzle).
 //    Per unit a warp runs S = K q'^T and O^T += V^T P on mma.sync with an
 //    online softmax in the exp2 domain (q' = q * scale * log2 e split into
 //    bf16 hi + lo).  At the end of each kv head the warps' states are merged
@@ -99,7 +100,7 @@ struct PsArgs {
 // All counters are zero between steps (the finisher of each count resets
 // it); the barrier counter only grows, by a multiple of the grid per step.
 struct PsWs {
-    size_t bar, abort, amax_key, amax_cnt, tilecnt, attncnt, pieces, recs, total;
+    size_t bar, abort, amax_key, amax_cnt, attncnt, recs, total;
     int32_t rmax, rec_floats;
 };
 
@@ -108,7 +109,6 @@ __host__ __device__ inline int ps_rec_floats(int group) { return (group * (kPsHd
 __host__ __device__ inline PsWs ps_ws_layout(int G, int n_layers, int n_kv, int group)
 {
     PsWs L;
-    const int nph = 5 * n_layers + 1;
     L.rmax = (G + n_kv - 1) / n_kv + 2;
     L.rec_floats = ps_rec_floats(group);
     L.bar = 0;
@@ -116,12 +116,8 @@ __host__ __device__ inline PsWs ps_ws_layout(int G, int n_layers, int n_kv, int 
     L.amax_key = 256;
     L.amax_cnt = 264;
     size_t off = 512;
-    L.tilecnt = off;
-    off += ((size_t)nph * G * 4 + 255) & ~(size_t)255;
     L.attncnt = off;
     off += ((size_t)n_layers * n_kv * 4 + 255) & ~(size_t)255;
-    L.pieces = off;
-    off += (size_t)G * 2 * 16 * 4;
     L.recs = off;
     off += ((size_t)n_kv * L.rmax * L.rec_floats * 4 + 255) & ~(size_t)255;
     L.total = off;
@@ -201,6 +197,7 @@ struct PsPhase {
     int64_t cb, ce;            // this CTA's range
     int64_t wb, we;            // GEMV: this warp's record range
     int32_t nst;               // this warp's stages in the phase
+    int64_t hfirst, hcnt;      // ATTN: the first CTA of this CTA's kv head and the head's CTA count
 };
 
 __device__ __forceinline__ PsPhase ps_phase(const PsArgs& P, int ph, int64_t b, int64_t G, int warp, int64_t nch)
@@ -221,18 +218,27 @@ __device__ __forceinline__ PsPhase ps_phase(const PsArgs& P, int ph, int64_t b, 
     default: break;
     }
     if (f.kind == PS_ATTN) {
+        // every CTA works on one kv head: head h has CTAs [h G / n_kv, (h + 1) G / n_kv),
+        // which split its nch units evenly
         f.kc = 0;
         f.R = (int64_t)P.n_kv * nch;
-        f.cb = split_begin(b, f.R, G);
-        f.ce = split_begin(b + 1, f.R, G);
+        const int64_t h = split_owner(b, G, P.n_kv);
+        f.hfirst = split_begin(h, G, P.n_kv);
+        f.hcnt = split_begin(h + 1, G, P.n_kv) - f.hfirst;
+        f.cb = h * nch + split_begin(b - f.hfirst, nch, f.hcnt);
+        f.ce = h * nch + split_begin(b - f.hfirst + 1, nch, f.hcnt);
         f.wb = f.we = 0;
         const int64_t mine = f.ce - f.cb - warp;               // units cb + warp + kPsWarps * j
         f.nst = mine > 0 ? 2 * (int32_t)((mine + kPsWarps - 1) / kPsWarps) : 0;   // a K and a V stage each
     } else {
+        // whole 16-row tiles per CTA (a tile is never cut between CTAs), the
+        // CTA's records split evenly over its warps
+        f.hfirst = f.hcnt = 0;
         f.kc = (int32_t)((f.k + 63) / 64);
-        f.R = ((f.n + 15) / 16) * f.kc;
-        f.cb = split_begin(b, f.R, G);
-        f.ce = split_begin(b + 1, f.R, G);
+        const int64_t T = (f.n + 15) / 16;
+        f.R = T * f.kc;
+        f.cb = split_begin(b, T, G) * f.kc;
+        f.ce = split_begin(b + 1, T, G) * f.kc;
         const int64_t Rb = f.ce - f.cb;
         f.wb = f.cb + Rb * warp / kPsWarps;
         f.we = f.cb + Rb * (warp + 1) / kPsWarps;
@@ -439,8 +445,9 @@ struct PsBest {
     int32_t i;
 };
 
+// res0 / res1: the residual of rows g and g + 8 (WO, W2), loaded ahead.
 __device__ __forceinline__ void ps_epilogue(const PsArgs& P, const PsPhase& f, int64_t tile, float v0, float v1,
-                                            float rr, int64_t pos, PsBest& best)
+                                            float rr, int64_t pos, PsBest& best, float res0, float res1)
 {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const float val[2] = {v0 * rr, v1 * rr};
@@ -485,30 +492,58 @@ __device__ __forceinline__ void ps_epilogue(const PsArgs& P, const PsPhase& f, i
                 cache[(head * P.window + pos % P.window) * kPsHd + col] = f32_to_bf16_bits(val[hh]);
             }
         } else if (f.kind == PS_WO) {
-            P.h[row] = __ldcg(P.x + row) + val[hh];
+            P.h[row] = (hh ? res1 : res0) + val[hh];
         } else {                                             // PS_W2
-            P.x[row] = __ldcg(P.h + row) + val[hh];
+            P.x[row] = (hh ? res1 : res0) + val[hh];
         }
     }
 }
 
 // ------------------------------------------------------------ GEMV phase
-// The warp's stages of one GEMV phase, then the merges of the tiles it
-// shares with other warps or CTAs.  `ok` turns false when a wait gave up;
-// the warp then skips work but still reaches every CTA barrier.
-__device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, const PsPhase& f, int ph, PsRing& ring, int nph,
-                              int64_t b, int64_t G, int64_t nch, int64_t pos, uint8_t* smem, const PsSmem& SL,
-                              PsBest& best, float rr, bool& ok)
+// The warp's stages of one GEMV phase, then the tiles it shares with other
+// warps of the CTA (summed in warp order from shared memory by the warp that
+// holds the tile's first record).  A CTA owns whole tiles, so no tile is
+// ever split between CTAs.  `ok` turns false when a wait gave up; the warp
+// then skips work but still reaches every CTA barrier.
+__device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, const PsPhase& f, int ph,
+                                              PsRing& ring, int nph, int64_t b, int64_t G, int64_t nch, int64_t pos,
+                                              uint8_t* smem, const PsSmem& SL, PsBest& best, float rr, bool& ok)
 {
+    (void)W;
+    (void)ph;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
     const int kc = f.kc, nblk = 2 * kc;
     float* s_piece = reinterpret_cast<float*>(smem + SL.piece);
     const uint32_t tk = smem_token();
     const uint32_t bs_a = smem_addr(smem + SL.act) + tk;
     const uint32_t cb_a = bs_a + (uint32_t)kc * 128u;
+    const int64_t wb = f.wb, we = f.we;
+
+    // The residual of the first two tiles that start in this warp's range
+    // (the tiles it finishes), loaded before the main loop.
+    const float* res_src = f.kind == PS_WO ? P.x : f.kind == PS_W2 ? P.h : nullptr;
+    const int64_t t_a = (wb + kc - 1) / kc;
+    float res[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    if (res_src && we > wb) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            if ((t_a + i) * kc >= we) break;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int64_t row = (t_a + i) * 16 + g + 8 * hh;
+                if (row < f.n) res[i][hh] = __ldcg(res_src + row);
+            }
+        }
+    }
+    auto res_of = [&](int64_t tile, int hh) -> float {
+        if (!res_src) return 0.f;
+        if (tile == t_a) return res[0][hh];
+        if (tile == t_a + 1) return res[1][hh];
+        const int64_t row = tile * 16 + g + 8 * hh;
+        return row < f.n ? __ldcg(res_src + row) : 0.f;
+    };
 
     // ---- main loop: this warp's records, two at a time
-    const int64_t wb = f.wb, we = f.we;
     if (we > wb && ok) {
         int64_t tile = wb / kc;
         int cin = (int)(wb - tile * kc);
@@ -544,7 +579,7 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
                     ++r;
                     if (++cin == kc || r == we) {
                         if (whole && cin == kc) {
-                            ps_epilogue(P, f, tile, acc0, acc2, rr, pos, best);
+                            ps_epilogue(P, f, tile, acc0, acc2, rr, pos, best, res_of(tile, 0), res_of(tile, 1));
                         } else if (t == 0) {
                             // a piece of a tile shared with other warps: slot 0 is the warp's first tile
                             const int slot = (tile == wb / kc) ? 0 : 1;
@@ -566,62 +601,22 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
     named_barrier(1, kPsThreads);
     if (!ok || we <= wb) return;
 
-    // ---- tiles cut between warps or CTAs: the warp holding the tile's first
-    // record inside this CTA sums the pieces in warp order
+    // ---- tiles cut between warps: the warp holding the tile's first record
+    // sums the pieces in warp order and finishes the tile
     const int64_t cb = f.cb, ce = f.ce, Rb = ce - cb;
-    const int64_t ft = wb / kc, lt = (we - 1) / kc;
-    for (int which = 0; which < 2; ++which) {
-        if (which == 1 && lt == ft) break;
-        const int64_t tl = which == 0 ? ft : lt;
-        const int64_t t0 = tl * kc, t1 = t0 + kc;
-        if (t0 >= wb && t1 <= we) continue;                     // finished in the main loop
-        if (which == 0 && t0 < wb && wb != cb) continue;        // an earlier warp of this CTA handles it
-        const int64_t last_in = (t1 < ce ? t1 : ce) - 1;
-        const int wl = (int)(((last_in - cb + 1) * kPsWarps - 1) / Rb);
+    const int64_t lt = (we - 1) / kc;
+    const int64_t t0 = lt * kc, t1 = t0 + kc;
+    if (t0 >= wb && t1 > we) {
+        const int wl = (int)(((t1 - cb) * kPsWarps - 1) / Rb);       // warp holding the tile's last record
         float s0 = 0.f, s2 = 0.f;
         for (int w2 = warp; w2 <= wl; ++w2) {
             const int64_t b2 = cb + Rb * w2 / kPsWarps, e2 = cb + Rb * (w2 + 1) / kPsWarps;
             if (e2 <= b2) continue;
-            const int slot = (w2 == warp) ? which : 0;
+            const int slot = (w2 == warp) ? (lt == wb / kc ? 0 : 1) : 0;
             s0 += s_piece[(w2 * 2 + slot) * 16 + g];
             s2 += s_piece[(w2 * 2 + slot) * 16 + g + 8];
         }
-        if (t0 >= cb && t1 <= ce) {
-            ps_epilogue(P, f, tl, s0, s2, rr, pos, best);
-            continue;
-        }
-        // cut between CTAs: publish this CTA's piece; the last CTA to arrive
-        // sums all pieces in CTA order and runs the epilogue
-        float* gp = reinterpret_cast<float*>(P.ws + W.pieces);
-        const int cslot = (tl == cb / kc) ? 0 : 1;
-        if (t == 0) {
-            __stcg(gp + (b * 2 + cslot) * 16 + g, s0);
-            __stcg(gp + (b * 2 + cslot) * 16 + g + 8, s2);
-            __threadfence();
-        }
-        __syncwarp();
-        const int64_t fc = split_owner(t0, f.R, G), lc = split_owner(t1 - 1, f.R, G);
-        int is_last = 0;
-        if (lane == 0) {
-            uint32_t ncon = 0;
-            for (int64_t c = fc; c <= lc; ++c) ncon += split_begin(c, f.R, G) < split_begin(c + 1, f.R, G) ? 1u : 0u;
-            uint32_t* ctr = reinterpret_cast<uint32_t*>(P.ws + W.tilecnt) + (size_t)ph * G + fc;
-            const uint32_t old = atom_add_acq_rel_gpu(ctr, 1u);
-            is_last = old + 1u == ncon;
-            if (is_last) atomicExch(ctr, 0u);
-        }
-        is_last = __shfl_sync(0xffffffffu, is_last, 0);
-        if (!is_last) continue;
-        __threadfence();
-        float a0 = 0.f, a2 = 0.f;
-        for (int64_t c = fc; c <= lc; ++c) {
-            const int64_t c0 = split_begin(c, f.R, G), c1 = split_begin(c + 1, f.R, G);
-            if (c1 <= c0) continue;
-            const int sl = (tl == c0 / kc) ? 0 : 1;
-            a0 += __ldcg(gp + (c * 2 + sl) * 16 + g);
-            a2 += __ldcg(gp + (c * 2 + sl) * 16 + g + 8);
-        }
-        ps_epilogue(P, f, tl, a0, a2, rr, pos, best);
+        ps_epilogue(P, f, lt, s0, s2, rr, pos, best, res_of(lt, 0), res_of(lt, 1));
     }
 }
 
@@ -816,7 +811,7 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
 
         // ---- merge the warps (warp order), then finish the head or publish the CTA's record
         const bool inside = hh * nch >= f.cb && (hh + 1) * nch <= f.ce;
-        const int64_t fc = split_owner(hh * nch, f.R, G), lc = split_owner(hh * nch + nch - 1, f.R, G);
+        const int64_t fc = f.hfirst, lc = f.hfirst + f.hcnt - 1;   // the CTAs of this kv head
         float* rec = recs + ((size_t)hh * W.rmax + (size_t)(b - fc)) * W.rec_floats;
         for (int i = tid; i < group * kPsHd; i += kPsThreads) {
             const int hi = i / kPsHd, cc = i - hi * kPsHd;
@@ -841,11 +836,12 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
             }
         }
         if (!inside) {
-            __threadfence();
-            named_barrier(1, kPsThreads);
+            named_barrier(1, kPsThreads);                 // every record store of the CTA is issued
             if (tid == 0) {
+                __threadfence();                          // ... and published before the arrival
                 uint32_t ncon = 0;
-                for (int64_t c = fc; c <= lc; ++c) ncon += split_begin(c, f.R, G) < split_begin(c + 1, f.R, G) ? 1u : 0u;
+                for (int64_t c = 0; c < f.hcnt; ++c)
+                    ncon += split_begin(c, nch, f.hcnt) < split_begin(c + 1, nch, f.hcnt) ? 1u : 0u;
                 uint32_t* ctr = reinterpret_cast<uint32_t*>(P.ws + W.attncnt) + (size_t)l * P.n_kv + hh;
                 const uint32_t old = atom_add_acq_rel_gpu(ctr, 1u);
                 const int last = old + 1u == ncon;
@@ -866,7 +862,7 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
                 for (int i = tid; i < nrec * group; i += kPsThreads) {
                     const int r = i / group, hi = i - r * group;
                     float2 ml = make_float2(-INFINITY, 0.f);        // a CTA with no units wrote no record
-                    if (split_begin(fc + r, f.R, G) < split_begin(fc + r + 1, f.R, G))
+                    if (split_begin(r, nch, f.hcnt) < split_begin(r + 1, nch, f.hcnt))
                         ml = __ldcg(reinterpret_cast<const float2*>(base + (size_t)r * W.rec_floats + group * kPsHd) + hi);
                     s_ml[2 * i] = ml.x;
                     s_ml[2 * i + 1] = ml.y;
@@ -1036,6 +1032,7 @@ const char* decoder_step_unsupported(const vox_decoder* d)
     if (d->n_layers > kPsMaxLayers) return "more than 32 layers";
     if (d->head_dim != kPsHd) return "head_dim is not 128";
     if (d->n_q_heads / d->n_kv_heads > kPsMaxGroup) return "more than 4 query heads per kv head";
+    if (d->n_kv_heads > device_sm_count()) return "more kv heads than SMs";
     if (d->dim % 4 || d->ffn % 8) return "dim not a multiple of 4 or ffn not a multiple of 8";
     return nullptr;
 }

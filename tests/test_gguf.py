@@ -7,7 +7,7 @@ import pytest
 
 import synth
 from oracle import ref
-from tests import gguf_writer as GW
+import gguf_writer as GW
 
 
 @pytest.fixture(scope="module")
