@@ -446,15 +446,12 @@ struct PsBest {
 };
 
 // res0 / res1: the residual of rows g and g + 8 (WO, W2), loaded ahead.
-// KIND is the phase kind, a template parameter so that each GEMV phase's
-// loop holds only its own epilogue.
-template <int KIND>
 __device__ __forceinline__ void ps_epilogue(const PsArgs& P, const PsPhase& f, int64_t tile, float v0, float v1,
                                             float rr, int64_t pos, PsBest& best, float res0, float res1)
 {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const float val[2] = {v0 * rr, v1 * rr};
-    if (KIND == PS_LM) {
+    if (f.kind == PS_LM) {
         float bv = -INFINITY;
         int32_t bi = 0x7fffffff;
 #pragma unroll
@@ -475,7 +472,7 @@ __device__ __forceinline__ void ps_epilogue(const PsArgs& P, const PsPhase& f, i
         return;
     }
     if (t != 0) return;
-    if (KIND == PS_W13) {
+    if (f.kind == PS_W13) {
         const int64_t row = tile * 16 + g;                   // gate row g pairs with up row g + 8
         if (row < f.n) P.act[tile * 8 + g] = silu_f(val[0]) * val[1];
         return;
@@ -484,7 +481,7 @@ __device__ __forceinline__ void ps_epilogue(const PsArgs& P, const PsPhase& f, i
     for (int hh = 0; hh < 2; ++hh) {
         const int64_t row = tile * 16 + g + 8 * hh;
         if (row >= f.n) continue;
-        if (KIND == PS_QKV) {
+        if (f.kind == PS_QKV) {
             P.qkv[row] = val[hh];
             const int64_t rel = row - P.q_dim;
             if (rel >= 0) {
@@ -494,7 +491,7 @@ __device__ __forceinline__ void ps_epilogue(const PsArgs& P, const PsPhase& f, i
                 uint16_t* cache = is_v ? P.vc[f.layer] : P.kc[f.layer];
                 cache[(head * P.window + pos % P.window) * kPsHd + col] = f32_to_bf16_bits(val[hh]);
             }
-        } else if (KIND == PS_WO) {
+        } else if (f.kind == PS_WO) {
             P.h[row] = (hh ? res1 : res0) + val[hh];
         } else {                                             // PS_W2
             P.x[row] = (hh ? res1 : res0) + val[hh];
@@ -508,7 +505,6 @@ __device__ __forceinline__ void ps_epilogue(const PsArgs& P, const PsPhase& f, i
 // holds the tile's first record).  A CTA owns whole tiles, so no tile is
 // ever split between CTAs.  `ok` turns false when a wait gave up; the warp
 // then skips work but still reaches every CTA barrier.
-template <int KIND>
 __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, const PsPhase& f, int ph,
                                               PsRing& ring, int nph, int64_t b, int64_t G, int64_t nch, int64_t pos,
                                               uint8_t* smem, const PsSmem& SL, PsBest& best, float rr, bool& ok)
@@ -525,7 +521,7 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
 
     // The residual of the first two tiles that start in this warp's range
     // (the tiles it finishes), loaded before the main loop.
-    const float* res_src = KIND == PS_WO ? P.x : KIND == PS_W2 ? P.h : nullptr;
+    const float* res_src = f.kind == PS_WO ? P.x : f.kind == PS_W2 ? P.h : nullptr;
     const int64_t t_a = (wb + kc - 1) / kc;
     float res[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
     if (res_src && we > wb) {
@@ -583,7 +579,7 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
                     ++r;
                     if (++cin == kc || r == we) {
                         if (whole && cin == kc) {
-                            ps_epilogue<KIND>(P, f, tile, acc0, acc2, rr, pos, best, res_of(tile, 0), res_of(tile, 1));
+                            ps_epilogue(P, f, tile, acc0, acc2, rr, pos, best, res_of(tile, 0), res_of(tile, 1));
                         } else if (t == 0) {
                             // a piece of a tile shared with other warps: slot 0 is the warp's first tile
                             const int slot = (tile == wb / kc) ? 0 : 1;
@@ -620,7 +616,7 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
             s0 += s_piece[(w2 * 2 + slot) * 16 + g];
             s2 += s_piece[(w2 * 2 + slot) * 16 + g + 8];
         }
-        ps_epilogue<KIND>(P, f, lt, s0, s2, rr, pos, best, res_of(lt, 0), res_of(lt, 1));
+        ps_epilogue(P, f, lt, s0, s2, rr, pos, best, res_of(lt, 0), res_of(lt, 1));
     }
 }
 
@@ -986,13 +982,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
             for (int w = 0; w < kPsWarps; ++w) ssq += s_sq[w];
             rr = 1.0f / sqrtf(ssq / (float)f.k + P.eps);
         }
-        switch (f.kind) {
-        case PS_QKV: ps_gemv_phase<PS_QKV>(P, W, f, ph, ring, nph, b, G, nch, pos, smem, SL, best, rr, ok); break;
-        case PS_WO:  ps_gemv_phase<PS_WO>(P, W, f, ph, ring, nph, b, G, nch, pos, smem, SL, best, rr, ok); break;
-        case PS_W13: ps_gemv_phase<PS_W13>(P, W, f, ph, ring, nph, b, G, nch, pos, smem, SL, best, rr, ok); break;
-        case PS_W2:  ps_gemv_phase<PS_W2>(P, W, f, ph, ring, nph, b, G, nch, pos, smem, SL, best, rr, ok); break;
-        default:     ps_gemv_phase<PS_LM>(P, W, f, ph, ring, nph, b, G, nch, pos, smem, SL, best, rr, ok); break;
-        }
+        ps_gemv_phase(P, W, f, ph, ring, nph, b, G, nch, pos, smem, SL, best, rr, ok);
     }
 
     // ---- greedy argmax: warps -> CTA -> one 64-bit atomic max; the last CTA
