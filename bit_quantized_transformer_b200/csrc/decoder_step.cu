@@ -294,12 +294,20 @@ struct PsRing {
     PsCursor cur;
 };
 
+#ifndef VOX_PS_PREFETCH
+#define VOX_PS_PREFETCH VOX_PS_STAGES
+#endif
+constexpr int kPsPrefetch = VOX_PS_PREFETCH;                 // stages of a later phase in flight at most
+
+// Top the warp's ring up to kPsStages stages in flight; stages of a phase
+// after ph_now count against the smaller kPsPrefetch.
 __device__ __forceinline__ void ps_ring_fill(const PsArgs& P, PsRing& r, int nph, int64_t b, int64_t G, int warp,
-                                             int lane, int64_t nch)
+                                             int lane, int64_t nch, int ph_now)
 {
     while (r.issued - r.consumed < (uint32_t)kPsStages) {
         ps_cursor_settle(P, r.cur, nph, b, G, warp, nch);
         if (r.cur.ph >= nph) break;
+        if (kPsPrefetch < kPsStages && r.cur.ph > ph_now && r.issued - r.consumed >= (uint32_t)kPsPrefetch) break;
         const uint32_t slot = r.issued % kPsStages;
         if (lane == 0) ps_issue(P, r.cur, warp, nch, r.base + slot * kPsStageBytes, &r.bars[slot]);
         ++r.issued;
@@ -319,10 +327,14 @@ __device__ __forceinline__ bool ps_ring_wait(PsRing& r, int32_t where, uint32_t 
 // One arrival per CTA on a monotonically growing counter; the target is the
 // next multiple of the grid size above the arrival's old value.  Bounded:
 // gives up after about one second or when another CTA raised the abort flag.
+// The arriving thread is lane 1 of warp 0, which issues no bulk copies: a
+// fence waits for the memory operations of its own thread only.
+constexpr int kPsSyncThread = 1;
+
 __device__ __forceinline__ bool ps_grid_barrier(const PsArgs& P, const PsWs& W, int32_t* s_flag, int32_t where)
 {
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == kPsSyncThread) {
         uint64_t* ctr = reinterpret_cast<uint64_t*>(P.ws + W.bar);
         const int32_t* abort = reinterpret_cast<const int32_t*>(P.ws + W.abort);
         const uint64_t G = gridDim.x;
@@ -595,7 +607,7 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
             }
             __syncwarp();
             ++ring.consumed;
-            ps_ring_fill(P, ring, nph, b, G, warp, lane, nch);
+            ps_ring_fill(P, ring, nph, b, G, warp, lane, nch, ph);
         }
     }
     named_barrier(1, kPsThreads);
@@ -783,7 +795,7 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
             __syncwarp();
             ring.consumed += 2;
             ++j;
-            ps_ring_fill(P, ring, nph, b, G, warp, lane, nch);
+            ps_ring_fill(P, ring, nph, b, G, warp, lane, nch, (int)f.layer * 5 + 1);
         }
 
         // ---- this warp's state for head hh -> merge buffer
@@ -837,7 +849,7 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
         }
         if (!inside) {
             named_barrier(1, kPsThreads);                 // every record store of the CTA is issued
-            if (tid == 0) {
+            if (tid == kPsSyncThread) {
                 __threadfence();                          // ... and published before the arrival
                 uint32_t ncon = 0;
                 for (int64_t c = 0; c < f.hcnt; ++c)
@@ -943,7 +955,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
     ring.cur.ph = 0;
     ring.cur.idx = 0;
     ring.cur.f = ps_phase(P, 0, b, G, warp, nch);
-    ps_ring_fill(P, ring, nph, b, G, warp, lane, nch);
+    ps_ring_fill(P, ring, nph, b, G, warp, lane, nch, 0);
 
     bool ok = true;
     if (P.test_withhold && b == 0 && warp == 0) {
@@ -964,6 +976,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
         if (ph > 0 && !ps_grid_barrier(P, W, s_flag, 0x510)) break;
         const PsPhase f = ps_phase(P, ph, b, G, warp, nch);
         if (f.kind == PS_ATTN) {
+            if (kPsPrefetch < kPsStages) ps_ring_fill(P, ring, nph, b, G, warp, lane, nch, ph);
             ps_attn_phase(P, W, f, ring, nph, b, G, nch, pos, n_valid, smem, SL, ok);
             continue;
         }
@@ -976,6 +989,8 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
         for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
         if (lane == 0) s_sq[warp] = sq;
         __syncthreads();
+        // the rest of this phase's stages, once the activation loads are done
+        if (kPsPrefetch < kPsStages) ps_ring_fill(P, ring, nph, b, G, warp, lane, nch, ph);
         float rr = 1.0f;
         if (f.kind == PS_QKV || f.kind == PS_W13 || f.kind == PS_LM) {
             float ssq = 0.f;
@@ -993,7 +1008,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
             s_best_i[warp] = best.i;
         }
         __syncthreads();
-        if (tid == 0 && !ld_relaxed_s32(reinterpret_cast<const int32_t*>(P.ws + W.abort))) {
+        if (tid == kPsSyncThread && !ld_relaxed_s32(reinterpret_cast<const int32_t*>(P.ws + W.abort))) {
             float bv = -INFINITY;
             int32_t bi = 0x7fffffff;
             for (int w = 0; w < kPsWarps; ++w)
