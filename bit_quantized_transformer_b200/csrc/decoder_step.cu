@@ -126,7 +126,7 @@ __host__ __device__ inline PsWs ps_ws_layout(int G, int n_layers, int n_kv, int 
 
 // ------------------------------------------------------- shared memory
 struct PsSmem {
-    uint32_t ring, bars, act, piece, sq, best_v, best_i, flags, never, total;
+    uint32_t ring, bars, act, piece, q, sq, best_v, best_i, flags, never, total;
 };
 
 __host__ __device__ inline PsSmem ps_smem_layout(uint32_t act_bytes)
@@ -137,6 +137,7 @@ __host__ __device__ inline PsSmem ps_smem_layout(uint32_t act_bytes)
     L.bars = off;   off += kPsWarps * kPsStages * 8;
     L.act = off;    off += (act_bytes + 15u) & ~15u;
     L.piece = off;  off += kPsWarps * 2 * 16 * 4;
+    L.q = off;      off += kPsMaxGroup * kPsHd * 4;             // the query heads of the CTA's kv head
     L.sq = off;     off += kPsWarps * 4;
     L.best_v = off; off += kPsWarps * 4;
     L.best_i = off; off += kPsWarps * 4;
@@ -658,21 +659,28 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
         for (int jj = 0; jj < 8; ++jj) o[jj][0] = o[jj][1] = o[jj][2] = o[jj][3] = 0.f;
         uint32_t qh[8][2], ql[8][2];
         bool have_q = false;
+        // the head's queries, written by the QKV phase of other CTAs: one round
+        // of loads for the whole CTA into shared memory
+        float* s_q = reinterpret_cast<float*>(smem + SL.q);
+        for (int i = tid; i < group * kPsHd; i += kPsThreads) s_q[i] = __ldcg(P.qkv + hh * group * kPsHd + i);
+        named_barrier(1, kPsThreads);
         while (ok && j < f.nst / 2) {
             const int64_t unit = f.cb + warp + (int64_t)kPsWarps * j;
             if (unit / nch != hh) break;
             if (!have_q) {
                 // q' = q * scale * log2(e), split into bf16 hi + lo B fragments (heads >= group are zero)
                 const bool okq = g < group;
-                const float* qr = P.qkv + (hh * group + (okq ? g : 0)) * kPsHd;
+                const float* qr = s_q + (okq ? g : 0) * kPsHd;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
                     if (okq) {
-                        v0 = __ldcg(qr + 16 * kk + 2 * t) * P.qscale;
-                        v1 = __ldcg(qr + 16 * kk + 2 * t + 1) * P.qscale;
-                        v2 = __ldcg(qr + 16 * kk + 2 * t + 8) * P.qscale;
-                        v3 = __ldcg(qr + 16 * kk + 2 * t + 9) * P.qscale;
+                        const float2 a0 = *reinterpret_cast<const float2*>(qr + 16 * kk + 2 * t);
+                        const float2 a1 = *reinterpret_cast<const float2*>(qr + 16 * kk + 2 * t + 8);
+                        v0 = a0.x * P.qscale;
+                        v1 = a0.y * P.qscale;
+                        v2 = a1.x * P.qscale;
+                        v3 = a1.y * P.qscale;
                     }
                     split_bf16x2(v0, v1, qh[kk][0], ql[kk][0]);
                     split_bf16x2(v2, v3, qh[kk][1], ql[kk][1]);
@@ -862,52 +870,41 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
             }
             named_barrier(1, kPsThreads);
             if (*reinterpret_cast<volatile int32_t*>(s_flag)) {
-                // last CTA of the head: fold the CTAs' records in CTA order.  Pass 1
-                // loads every (record, head) (m, l) pair at once; the factors
-                // exp2(m - M) replace m in shared memory; pass 2 streams the O rows
-                // eight records per round.
+                // last CTA of the head: fold the CTAs' records in CTA order, every
+                // record's (m, l, O) of an output loaded in one round per 16
+                // records (a CTA with no units wrote no record and is skipped)
                 __threadfence();
                 const float* base = recs + (size_t)hh * W.rmax * W.rec_floats;
                 const int nrec = (int)(lc - fc + 1);
-                float* s_ml = merge;                              // [nrec][group] x (m or factor, l)
-                float* s_L = merge + 2 * nrec * group;
-                for (int i = tid; i < nrec * group; i += kPsThreads) {
-                    const int r = i / group, hi = i - r * group;
-                    float2 ml = make_float2(-INFINITY, 0.f);        // a CTA with no units wrote no record
-                    if (split_begin(r, nch, f.hcnt) < split_begin(r + 1, nch, f.hcnt))
-                        ml = __ldcg(reinterpret_cast<const float2*>(base + (size_t)r * W.rec_floats + group * kPsHd) + hi);
-                    s_ml[2 * i] = ml.x;
-                    s_ml[2 * i + 1] = ml.y;
-                }
-                named_barrier(1, kPsThreads);
-                if (tid < group) {
-                    float M = -INFINITY, L = 0.f;
-                    for (int r = 0; r < nrec; ++r) M = fmaxf(M, s_ml[2 * (r * group + tid)]);
-                    for (int r = 0; r < nrec; ++r) {
-                        const float mv = s_ml[2 * (r * group + tid)];
-                        const float fct = (mv == -INFINITY) ? 0.f : exp2f(mv - M);
-                        s_ml[2 * (r * group + tid)] = fct;
-                        L += fct * s_ml[2 * (r * group + tid) + 1];
-                    }
-                    s_L[tid] = L;
-                }
-                named_barrier(1, kPsThreads);
                 for (int i = tid; i < group * kPsHd; i += kPsThreads) {
                     const int hi = i / kPsHd, cc = i - hi * kPsHd;
-                    float O = 0.f;
-                    for (int r0 = 0; r0 < nrec; r0 += 8) {
-                        float v[8];
+                    float M = -INFINITY, O = 0.f, L = 0.f;
+                    for (int r0 = 0; r0 < nrec; r0 += 16) {
+                        float mv[16], lv[16], ov[16];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            v[u] = r0 + u < nrec ? __ldcg(base + (size_t)(r0 + u) * W.rec_floats + hi * kPsHd + cc) : 0.f;
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            if (r0 + u >= nrec) break;
-                            const float fct = s_ml[2 * ((r0 + u) * group + hi)];
-                            O += fct != 0.f ? fct * v[u] : 0.f;     // an empty CTA's slot may hold anything
+                        for (int u = 0; u < 16; ++u) {
+                            const int r = r0 + u;
+                            const bool have = r < nrec && split_begin(r, nch, f.hcnt) < split_begin(r + 1, nch, f.hcnt);
+                            const float* rc = base + (size_t)(have ? r : 0) * W.rec_floats;
+                            mv[u] = have ? __ldcg(rc + group * kPsHd + hi * 2) : -INFINITY;
+                            lv[u] = have ? __ldcg(rc + group * kPsHd + hi * 2 + 1) : 0.f;
+                            ov[u] = have ? __ldcg(rc + hi * kPsHd + cc) : 0.f;
                         }
+                        float Mb = M;
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) Mb = fmaxf(Mb, mv[u]);
+                        const float fo = (M == -INFINITY) ? 0.f : exp2f(M - Mb);
+                        O *= fo;
+                        L *= fo;
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) {
+                            const float fct = (mv[u] == -INFINITY) ? 0.f : exp2f(mv[u] - Mb);
+                            O = fmaf(fct, ov[u], O);
+                            L = fmaf(fct, lv[u], L);
+                        }
+                        M = Mb;
                     }
-                    P.attn[(hh * group + hi) * kPsHd + cc] = O / s_L[hi];
+                    P.attn[(hh * group + hi) * kPsHd + cc] = O / L;
                 }
             }
         }
