@@ -870,41 +870,58 @@ __device__ __forceinline__ void ps_attn_phase(const PsArgs& P, const PsWs& W, co
             }
             named_barrier(1, kPsThreads);
             if (*reinterpret_cast<volatile int32_t*>(s_flag)) {
-                // last CTA of the head: fold the CTAs' records in CTA order, every
-                // record's (m, l, O) of an output loaded in one round per 16
-                // records (a CTA with no units wrote no record and is skipped)
+                // last CTA of the head: fold the CTAs' records in CTA order.  Each
+                // thread first issues the loads of its outputs' O values of every
+                // record (they do not depend on m), then the (m, l) pairs go
+                // through shared memory, where the factors exp2(m - M) replace m.
                 __threadfence();
                 const float* base = recs + (size_t)hh * W.rmax * W.rec_floats;
                 const int nrec = (int)(lc - fc + 1);
-                for (int i = tid; i < group * kPsHd; i += kPsThreads) {
-                    const int hi = i / kPsHd, cc = i - hi * kPsHd;
-                    float M = -INFINITY, O = 0.f, L = 0.f;
-                    for (int r0 = 0; r0 < nrec; r0 += 16) {
-                        float mv[16], lv[16], ov[16];
+                float* s_ml = merge;                              // [nrec][group] x (m or factor, l)
+                float* s_L = merge + 2 * nrec * group;
+                constexpr int kFold = 24;                          // records of one round of O loads
+                for (int i0 = 0; i0 < group * kPsHd; i0 += kPsThreads) {
+                    const int i = i0 + tid;
+                    const int hi = i < group * kPsHd ? i / kPsHd : 0, cc = i - hi * kPsHd;
+                    float O = 0.f;
+                    for (int r0 = 0; r0 < nrec; r0 += kFold) {
+                        float ov[kFold];
 #pragma unroll
-                        for (int u = 0; u < 16; ++u) {
-                            const int r = r0 + u;
-                            const bool have = r < nrec && split_begin(r, nch, f.hcnt) < split_begin(r + 1, nch, f.hcnt);
-                            const float* rc = base + (size_t)(have ? r : 0) * W.rec_floats;
-                            mv[u] = have ? __ldcg(rc + group * kPsHd + hi * 2) : -INFINITY;
-                            lv[u] = have ? __ldcg(rc + group * kPsHd + hi * 2 + 1) : 0.f;
-                            ov[u] = have ? __ldcg(rc + hi * kPsHd + cc) : 0.f;
+                        for (int u = 0; u < kFold; ++u)
+                            ov[u] = (i < group * kPsHd && r0 + u < nrec)
+                                        ? __ldcg(base + (size_t)(r0 + u) * W.rec_floats + hi * kPsHd + cc) : 0.f;
+                        if (i0 == 0 && r0 == 0) {
+                            for (int q = tid; q < nrec * group; q += kPsThreads) {
+                                const int r = q / group, h2 = q - r * group;
+                                float2 ml = make_float2(-INFINITY, 0.f);   // a CTA with no units wrote no record
+                                if (split_begin(r, nch, f.hcnt) < split_begin(r + 1, nch, f.hcnt))
+                                    ml = __ldcg(reinterpret_cast<const float2*>(base + (size_t)r * W.rec_floats +
+                                                                               group * kPsHd) + h2);
+                                s_ml[2 * q] = ml.x;
+                                s_ml[2 * q + 1] = ml.y;
+                            }
+                            named_barrier(1, kPsThreads);
+                            if (tid < group) {
+                                float M = -INFINITY, L = 0.f;
+                                for (int r = 0; r < nrec; ++r) M = fmaxf(M, s_ml[2 * (r * group + tid)]);
+                                for (int r = 0; r < nrec; ++r) {
+                                    const float mv = s_ml[2 * (r * group + tid)];
+                                    const float fct = (mv == -INFINITY) ? 0.f : exp2f(mv - M);
+                                    s_ml[2 * (r * group + tid)] = fct;
+                                    L += fct * s_ml[2 * (r * group + tid) + 1];
+                                }
+                                s_L[tid] = L;
+                            }
+                            named_barrier(1, kPsThreads);
                         }
-                        float Mb = M;
 #pragma unroll
-                        for (int u = 0; u < 16; ++u) Mb = fmaxf(Mb, mv[u]);
-                        const float fo = (M == -INFINITY) ? 0.f : exp2f(M - Mb);
-                        O *= fo;
-                        L *= fo;
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) {
-                            const float fct = (mv[u] == -INFINITY) ? 0.f : exp2f(mv[u] - Mb);
-                            O = fmaf(fct, ov[u], O);
-                            L = fmaf(fct, lv[u], L);
+                        for (int u = 0; u < kFold; ++u) {
+                            if (r0 + u >= nrec) break;
+                            const float fct = s_ml[2 * ((r0 + u) * group + hi)];
+                            O += fct != 0.f ? fct * ov[u] : 0.f;   // an empty CTA's slot may hold anything
                         }
-                        M = Mb;
                     }
-                    P.attn[(hh * group + hi) * kPsHd + cc] = O / L;
+                    if (i < group * kPsHd) P.attn[(hh * group + hi) * kPsHd + cc] = O / s_L[hi];
                 }
             }
         }
