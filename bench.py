@@ -453,7 +453,7 @@ def run_ours(args):
             "k1_gemv": {"kernel": "q4_gemv_kernel", "launches": dm.gemv_chain_launches(),
                         "us_per_launch": ms_g / dm.gemv_chain_launches() * 1e3, "gbs": k1_gbs,
                         "frac": k1_gbs / peak},
-            "k4_attention": {"kernel": "gqa_decode_attn_kernel", "gbs":
+            "k4_attention": {"kernel": "gqa_decode_attn_kernel+attn_combine_kernel", "gbs":
                              attn_bytes / (ms_a / 1e3) / 1e9, "us_per_layer": ms_a / dm.L * 1e3},
             "gpu_launches": (dm.step_launches() if form == "persistent" else dm.step_kernels_launches()) * args.steps,
             "clocks": clk,

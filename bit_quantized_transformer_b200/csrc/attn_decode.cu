@@ -1,5 +1,5 @@
-// Rolling KV cache append (K3) and split-KV GQA decode attention (K4), whose
-// last CTA per kv head merges that head's partials by a log-sum-exp combine.
+// Rolling KV cache append (K3), split-KV GQA decode attention (K4) and the
+// log-sum-exp combine of its partials (K5).
 //
 // Sources: "Mistral Voxtral Realtime 4B ... 순수 C 기반 CPU 전용 추론 구현",
 // "주요 기능" (rolling KV cache over an 8192-position sliding window; fused
@@ -21,10 +21,9 @@
 // q' and P are split into bf16 hi + lo parts (two MMAs each), so the
 // tensor-core inputs carry about 16 significant bits; K and V are the cache's
 // own bf16 values.  Each CTA writes one (m, l, O) partial per kv head it
-// touched, into that head's contiguous run of records, then arrives on the
-// head's counter; the last CTA to arrive merges the head's run in CTA order
-// (deterministic), one warp per query head, all of a head's records loaded in
-// one round before the arithmetic.
+// touched, into that head's contiguous run of records; K5 merges each head's
+// run in CTA order (deterministic), one small CTA per query head, all of a
+// head's records loaded in one round before the arithmetic.
 //
 // Programmatic dependent launch: the producer starts streaming before the
 // upstream kernel (the QKV projection that appends this step's k, v) has
@@ -80,11 +79,10 @@ constexpr int kAttnMaxStages = 6;
 constexpr int kAttnTileBytes = kAttnChunk * 128;            // one 64 x 64 bf16 box
 constexpr int kAttnStageBytes = 4 * kAttnTileBytes;         // K lo/hi, V lo/hi
 constexpr int kAttnMaxCtas = 592;
-constexpr int kCombineBatch = 20;                  // records of a head loaded per round of the merge
+constexpr int kCombineBatch = 20;                  // records of a head loaded per round in K5
 constexpr int kAttnMaxGroup = 8;
 
 struct AttnArgs {
-    uint32_t* cnt;                             // per kv head arrival counters (zero between calls)
     const float* q;
     const uint16_t* kcache;
     const uint16_t* vcache;
@@ -122,15 +120,12 @@ static int64_t attn_grid(int n_kv, int window)
     return G;
 }
 
-// Workspace: the per-head arrival counters (a 256-byte aligned region),
-// then rmax partial records per kv head (room for the largest group).
-__host__ __device__ constexpr size_t attn_cnt_bytes(int n_kv) { return ((size_t)n_kv * 4 + 255) & ~(size_t)255; }
-
+// Workspace: rmax partial records per kv head (room for the largest group).
 size_t attn_workspace_bytes(int n_kv, int hd, int window)
 {
     (void)window;
-    return attn_cnt_bytes(n_kv) +
-           (((size_t)n_kv * attn_rmax(n_kv) * attn_rec_floats(kAttnMaxGroup, hd) * sizeof(float) + 255) & ~(size_t)255);
+    return ((size_t)n_kv * attn_rmax(n_kv) * attn_rec_floats(kAttnMaxGroup, hd) * sizeof(float) + 255) &
+           ~(size_t)255;
 }
 
 __host__ __device__ inline int64_t attn_begin(int64_t b, int64_t total, int64_t G) { return b * total / G; }
@@ -150,69 +145,6 @@ __host__ __device__ inline AttnSmem attn_smem_layout(int stages)
     L.flags = L.bars + 2u * (uint32_t)stages * 8u;
     L.total = L.flags + 16 + 1024;             // + alignment slack
     return L;
-}
-
-// ------------------------------------------------------------------ merge
-// The merge of one query head's records, run by the last CTA to finish the
-// kv head (one warp per query head; lane l covers dims 4l .. 4l+3).  The
-// head's records sit in one contiguous run; a CTA in the head's range that
-// owned no chunk (possible when the grid outnumbers the chunks) wrote
-// nothing and is skipped.  Each round loads up to kCombineBatch records,
-// then folds them max-first in CTA order.
-__device__ __forceinline__ bool attn_cta_nonempty(int64_t bo, int64_t total, int64_t G)
-{
-    if (total < (1 << 20) && G < (1 << 11)) {
-        const uint32_t t32 = (uint32_t)total, g32 = (uint32_t)G, b32 = (uint32_t)bo;
-        return (b32 * t32) / g32 != ((b32 + 1) * t32) / g32;
-    }
-    return attn_begin(bo, total, G) != attn_begin(bo + 1, total, G);
-}
-
-__device__ void attn_fold(const AttnArgs& a, int kh, int gi, int lane, int64_t G, int64_t nch, int64_t total)
-{
-    const int group = a.group;
-    const int64_t bf = attn_owner((int64_t)kh * nch, total, G), bl = attn_owner((int64_t)kh * nch + nch - 1, total, G);
-    const int nrec = (int)(bl - bf + 1);
-    const float* recs = a.ws + (size_t)kh * a.rmax * a.rec_floats;
-    float M = -INFINITY, L = 0.f;
-    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int r0 = 0; r0 < nrec; r0 += kCombineBatch) {
-        // lane i decides whether record r0 + i exists
-        const bool mine = r0 + lane < nrec && lane < kCombineBatch && attn_cta_nonempty(bf + r0 + lane, total, G);
-        const uint32_t mask = __ballot_sync(0xffffffffu, mine);
-        float2 ml[kCombineBatch];
-        float4 ov[kCombineBatch];
-#pragma unroll
-        for (int u = 0; u < kCombineBatch; ++u) {
-            ml[u] = make_float2(-INFINITY, 0.f);
-            ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if ((mask >> u) & 1u) {
-                const float* rec = recs + (size_t)(r0 + u) * a.rec_floats;
-                ml[u] = __ldcg(reinterpret_cast<const float2*>(rec + group * kAttnHd) + gi);
-                ov[u] = __ldcg(reinterpret_cast<const float4*>(rec + gi * kAttnHd) + lane);
-            }
-        }
-        float mb = M;
-#pragma unroll
-        for (int u = 0; u < kCombineBatch; ++u) mb = fmaxf(mb, ml[u].x);
-        const float fo = M == -INFINITY ? 0.f : exp2f(M - mb);
-        O = make_float4(O.x * fo, O.y * fo, O.z * fo, O.w * fo);
-        L *= fo;
-#pragma unroll
-        for (int u = 0; u < kCombineBatch; ++u) {
-            if (ml[u].x == -INFINITY) continue;
-            const float f = exp2f(ml[u].x - mb);
-            O.x = fmaf(f, ov[u].x, O.x);
-            O.y = fmaf(f, ov[u].y, O.y);
-            O.z = fmaf(f, ov[u].z, O.z);
-            O.w = fmaf(f, ov[u].w, O.w);
-            L = fmaf(f, ml[u].y, L);
-        }
-        M = mb;
-    }
-    const float inv = 1.0f / L;
-    *reinterpret_cast<float4*>(a.out + ((int64_t)kh * group + gi) * kAttnHd + 4 * lane) =
-        make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 2)
@@ -336,24 +268,6 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
                 rec[group * kAttnHd + hh * 2 + 0] = M;
                 rec[group * kAttnHd + hh * 2 + 1] = Lsum;
             }
-        }
-        named_barrier(1, 32 * kAttnWarps);
-        // arrive on the head's counter; the last CTA of the head merges its records
-        if (tid == 0) {
-            const int64_t bl_seg = attn_owner(kh_seg * nch + nch - 1, total, G);
-            uint32_t ncon = 0;
-            for (int64_t c = bf_seg; c <= bl_seg; ++c) ncon += attn_cta_nonempty(c, total, G) ? 1u : 0u;
-            __threadfence();
-            uint32_t old;
-            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(a.cnt + kh_seg) : "memory");
-            const int last = old + 1u == ncon;
-            if (last) atomicExch(a.cnt + kh_seg, 0u);
-            s_fail[1] = last;
-        }
-        named_barrier(1, 32 * kAttnWarps);
-        if (s_fail[1]) {
-            __threadfence();
-            for (int gi = warp; gi < group; gi += kAttnWarps) attn_fold(a, (int)kh_seg, gi, lane, G, nch, total);
         }
         named_barrier(1, 32 * kAttnWarps);
     };
@@ -507,6 +421,76 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     if (seg_head >= 0) flush(seg_idx, seg_head);
 }
 
+// ------------------------------------------------------------------ K5
+// One 32-thread CTA per (kv head, query head of its group); lane l covers
+// dims 4l .. 4l+3.  The head's records sit in one contiguous run; a CTA in
+// the head's range that owned no chunk (possible when the grid outnumbers
+// the chunks) wrote nothing and is skipped.  Each round loads up to
+// kCombineBatch records, then folds them max-first in CTA order.
+__device__ __forceinline__ bool attn_cta_nonempty(int64_t bo, int64_t total, int64_t G)
+{
+    if (total < (1 << 20) && G < (1 << 11)) {
+        const uint32_t t32 = (uint32_t)total, g32 = (uint32_t)G, b32 = (uint32_t)bo;
+        return (b32 * t32) / g32 != ((b32 + 1) * t32) / g32;
+    }
+    return attn_begin(bo, total, G) != attn_begin(bo + 1, total, G);
+}
+
+__global__ void __launch_bounds__(32) attn_combine_kernel(const AttnArgs a, int64_t G)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int group = a.group;
+    const int kh = blockIdx.x / group, gi = blockIdx.x - kh * group, lane = threadIdx.x;
+    const int W = a.window;
+    const int64_t pos = a.pos_dev ? *a.pos_dev : a.pos;
+    const int64_t n_valid = pos + 1 < W ? pos + 1 : W;
+    const int64_t nch = (n_valid + kAttnChunk - 1) / kAttnChunk;
+    const int64_t total = (int64_t)a.n_kv * nch;
+    const int64_t bf = attn_owner((int64_t)kh * nch, total, G), bl = attn_owner((int64_t)kh * nch + nch - 1, total, G);
+    const int nrec = (int)(bl - bf + 1);
+    const float* recs = a.ws + (size_t)kh * a.rmax * a.rec_floats;
+    float M = -INFINITY, L = 0.f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r0 = 0; r0 < nrec; r0 += kCombineBatch) {
+        // lane i decides whether record r0 + i exists
+        const bool mine = r0 + lane < nrec && lane < kCombineBatch && attn_cta_nonempty(bf + r0 + lane, total, G);
+        const uint32_t mask = __ballot_sync(0xffffffffu, mine);
+        float2 ml[kCombineBatch];
+        float4 ov[kCombineBatch];
+#pragma unroll
+        for (int u = 0; u < kCombineBatch; ++u) {
+            ml[u] = make_float2(-INFINITY, 0.f);
+            ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if ((mask >> u) & 1u) {
+                const float* rec = recs + (size_t)(r0 + u) * a.rec_floats;
+                ml[u] = __ldcg(reinterpret_cast<const float2*>(rec + group * kAttnHd) + gi);
+                ov[u] = __ldcg(reinterpret_cast<const float4*>(rec + gi * kAttnHd) + lane);
+            }
+        }
+        float mb = M;
+#pragma unroll
+        for (int u = 0; u < kCombineBatch; ++u) mb = fmaxf(mb, ml[u].x);
+        const float fo = M == -INFINITY ? 0.f : exp2f(M - mb);
+        O = make_float4(O.x * fo, O.y * fo, O.z * fo, O.w * fo);
+        L *= fo;
+#pragma unroll
+        for (int u = 0; u < kCombineBatch; ++u) {
+            if (ml[u].x == -INFINITY) continue;
+            const float f = exp2f(ml[u].x - mb);
+            O.x = fmaf(f, ov[u].x, O.x);
+            O.y = fmaf(f, ov[u].y, O.y);
+            O.z = fmaf(f, ov[u].z, O.z);
+            O.w = fmaf(f, ov[u].w, O.w);
+            L = fmaf(f, ml[u].y, L);
+        }
+        M = mb;
+    }
+    const float inv = 1.0f / L;
+    *reinterpret_cast<float4*>(a.out + ((int64_t)kh * group + gi) * kAttnHd + 4 * lane) =
+        make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+}
+
 vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc, float* out, int n_q, int n_kv,
                                   int hd, int window, int64_t pos, const int64_t* pos_dev, float scale, void* ws,
                                   cudaStream_t s)
@@ -533,8 +517,7 @@ vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc
     a.pos = pos;
     a.pos_dev = pos_dev;
     a.qscale = scale * 1.4426950408889634f;
-    a.cnt = static_cast<uint32_t*>(ws);
-    a.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + attn_cnt_bytes(n_kv));
+    a.ws = static_cast<float*>(ws);
     a.rec_floats = attn_rec_floats(a.group, hd);
     a.rmax = attn_rmax(n_kv);
     a.stages = env_int_attn("VOX_ATTN_STAGES", 3, 2, kAttnMaxStages);
@@ -545,12 +528,14 @@ vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc
                               (int)attn_smem_layout(kAttnMaxStages).total, attr_done);
     if (st != VOX_OK) return st;
     const int64_t G = attn_grid(n_kv, window);
-    return launch_pdl(gqa_decode_attn_kernel, dim3((unsigned)G), dim3(kAttnThreads), SL.total, s, kmap, vmap, a);
+    st = launch_pdl(gqa_decode_attn_kernel, dim3((unsigned)G), dim3(kAttnThreads), SL.total, s, kmap, vmap, a);
+    if (st != VOX_OK) return st;
+    return launch_pdl(attn_combine_kernel, dim3((unsigned)(n_kv * a.group)), dim3(32), 0, s, a, G);
 }
 
 // --------------------------------------------- allocation-free entry point
 // vox_gqa_decode_attn needs the caller to hand in device scratch for the
-// split-KV partial records and the per-head arrival counters.  Some callers cannot: a host program that links
+// split-KV partial records.  Some callers cannot: a host program that links
 // only this C library and owns no device allocator, or a real-time audio
 // thread that must not call cudaMalloc (it can block and synchronise the
 // device).  vox_gqa_decode_attn_static serves them from one fixed scratch
@@ -570,7 +555,6 @@ constexpr int attn_static_max_records(int n)
                                                                         : attn_static_max_records(n - 1));
 }
 constexpr size_t kStaticScratchBytes =
-    attn_cnt_bytes(kStaticMaxKv) +
     (size_t)attn_static_max_records(kStaticMaxKv) * attn_rec_floats(kStaticMaxGroup, kAttnHd) * sizeof(float);
 
 static __device__ __align__(256) uint8_t g_attn_static_scratch[kStaticScratchBytes];
@@ -632,9 +616,8 @@ extern "C" vox_status vox_gqa_decode_attn_static(const float* q, const void* k_c
     if (((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache) |
           reinterpret_cast<uintptr_t>(out)) & 15u) != 0)
         return VOX_ERR_ALIGN;
-    // the counters and the records this call uses: n_kv runs of rmax records of the group's size
-    const size_t need = attn_cnt_bytes(n_kv_heads) +
-                        (size_t)n_kv_heads * attn_rmax(n_kv_heads) * attn_rec_floats(group, kAttnHd) * sizeof(float);
+    // the records this call writes: n_kv runs of rmax records of the group's size
+    const size_t need = (size_t)n_kv_heads * attn_rmax(n_kv_heads) * attn_rec_floats(group, kAttnHd) * sizeof(float);
     if (need > kStaticScratchBytes) {
         set_error_text("vox_gqa_decode_attn_static: shape needs more than the static scratch");
         return VOX_ERR_RANGE;

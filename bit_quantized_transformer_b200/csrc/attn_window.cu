@@ -60,18 +60,6 @@ __device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], uint32_t addr)
                  : "r"(addr) : "memory");
 }
 
-// 16-byte asynchronous global -> shared copy; src_bytes 0 writes zeros.
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
 // Copies of key tile [j0, j0 + 64) of head h (K and V) into one ring stage;
 // rows at or past j_end are zero-filled.
 __device__ __forceinline__ void win_load_tile(const WinArgs& a, int h, int64_t j0, int64_t j_end, uint8_t* sK,

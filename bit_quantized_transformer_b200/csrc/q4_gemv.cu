@@ -89,6 +89,7 @@ struct GemvArgs {
     uint8_t* ws;
     int32_t stages;
     int32_t pre;                             // ring stages issued before griddepcontrol.wait
+    int32_t evict_first;                     // 1: weight copies marked evict-first in L2
 };
 
 // Shared-memory carve-up, computed identically on host and device.
@@ -129,12 +130,15 @@ size_t gemv_workspace_bytes(int64_t n, int64_t k, int op)
 // Issue ring batch j of a warp's range [wb, we): up to kGemvRecs records
 // in one bulk copy, completing on `bar`.
 __device__ __forceinline__ void gemv_issue(const uint8_t* w, int64_t wb, int64_t we, int j, uint8_t* dst,
-                                           uint64_t* bar)
+                                           uint64_t* bar, int evict_first)
 {
     const int64_t r0 = wb + (int64_t)j * kGemvRecs;
     const uint32_t bytes = (uint32_t)min64(kGemvRecs, we - r0) * kChunkBytes;
     mbar_arrive_expect_tx(bar, bytes);
-    bulk_g2s(dst, w + r0 * kChunkBytes, bytes, bar);
+    if (evict_first)
+        bulk_g2s_stream(dst, w + r0 * kChunkBytes, bytes, bar);
+    else
+        bulk_g2s(dst, w + r0 * kChunkBytes, bytes, bar);
 }
 
 // Running greedy-argmax candidates of one lane, for its tokens 2t and 2t + 1.
@@ -311,7 +315,7 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
         fence_mbar_init();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         for (int j = 0; j < a.pre && j < nbatch; ++j)
-            gemv_issue(a.w, wb, we, j, ring + j * kGemvStageBytes, &bars[j]);
+            gemv_issue(a.w, wb, we, j, ring + j * kGemvStageBytes, &bars[j], a.evict_first);
         s_ptile[warp] = -1;
     }
 
@@ -333,7 +337,7 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
     // the rest of the ring, issued once the activations are in
     if (lane == 0)
         for (int j = a.pre; j < stages && j < nbatch; ++j)
-            gemv_issue(a.w, wb, we, j, ring + j * kGemvStageBytes, &bars[j]);
+            gemv_issue(a.w, wb, we, j, ring + j * kGemvStageBytes, &bars[j], a.evict_first);
 
     // RMSNorm factors of this lane's tokens 2t, 2t+1 (zero for tokens past m)
     float rr[2];
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
             }
             __syncwarp();
             if (lane == 0 && j + stages < nbatch)
-                gemv_issue(a.w, wb, we, j + stages, ring + s * kGemvStageBytes, &bars[s]);
+                gemv_issue(a.w, wb, we, j + stages, ring + s * kGemvStageBytes, &bars[s], a.evict_first);
             if (++s == stages) s = 0;
         }
         if (fail_j >= 0 && lane == 0) {
@@ -566,6 +570,7 @@ vox_status launch_q4_gemv(const uint8_t* w, int64_t n, int64_t k, const float* x
     if (L.total > 227 * 1024) return VOX_ERR_SHAPE;            // activations do not fit shared memory
     a.stages = stages;
     a.pre = env_int("VOX_GEMV_PREFETCH", 1, 0, stages);
+    a.evict_first = env_int("VOX_GEMV_EVICT_FIRST", 1, 0, 1);
 
     void (*kern)(GemvArgs) = m == 1 ? q4_gemv_kernel<1> : q4_gemv_kernel<8>;
     static std::atomic<unsigned long long> attr_done1{0}, attr_done8{0};

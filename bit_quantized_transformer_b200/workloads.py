@@ -161,7 +161,7 @@ class DecoderModel:
             self.shape.vocab * self.shape.dim * 18 // 32
 
     def attn_chain(self, pos: int):
-        """The step's attention launches alone (one split-KV launch per layer, merge included),
+        """The step's attention launches alone (per layer: split-KV + combine),
         at a host-given position."""
         wsb = V.vox_gqa_decode_attn_workspace(self.shape.n_q_heads, self.shape.n_kv_heads, self.shape.head_dim,
                                               self.W)
@@ -177,7 +177,7 @@ class DecoderModel:
 
     def step_kernels_launches(self) -> int:
         """Kernels one vox_decoder_step_kernels launches."""
-        return 1 + self.L * 5 + 1 + 1
+        return 1 + self.L * 6 + 1 + 1
 
     def weight_bytes(self) -> int:
         """Packed Q4 bytes streamed per step (all layers + LM head + one embedding row)."""

@@ -226,13 +226,9 @@ vox_status vox_kv_append_rolling(void *k_cache, void *v_cache, const void *k_new
  * 16-byte aligned; out: device fp32 [n_q_heads][head_dim], 16-byte aligned
  * (it is written with 16-byte stores).  Split-KV: slot
  * ranges are reduced independently into the workspace (device, at least
- * vox_gqa_decode_attn_workspace() bytes, 16-byte aligned), then the last
- * CTA to finish a kv head merges that head's partials by a log-sum-exp
- * combine.  The workspace starts with the per-kv-head arrival counters,
- * ((4 n_kv_heads + 255) / 256) * 256 bytes that must be zero before the
- * first call (every call leaves them zero again); the partial records after
- * them need no initial contents.  Calls sharing a workspace must not overlap
- * on the GPU.  head_dim must be
+ * vox_gqa_decode_attn_workspace() bytes, 16-byte aligned, no initial contents
+ * needed) and merged by a log-sum-exp combine (a second, small kernel).
+ * Calls sharing a workspace must not overlap on the GPU.  head_dim must be
  * 128 (the decoder's).
  * Errors: NULL -> VOX_ERR_NULL; pos < 0, window <= 0, n_q % n_kv != 0, a
  * group above 8 or more than 512 kv heads -> VOX_ERR_RANGE; other head_dim
@@ -252,14 +248,11 @@ size_t vox_gqa_decode_attn_workspace(int32_t n_q_heads, int32_t n_kv_heads, int3
  * audio thread that must not call cudaMalloc, which can block and
  * synchronise the device).  Same arguments, result and precision as
  * vox_gqa_decode_attn.  It allocates nothing: the split-KV partial records
- * and the per-head arrival counters go to one fixed array in device memory
- * that is part of the loaded library (about 1.2 MiB), sized for at most 8 kv
- * heads with at most 4 query heads per kv head at head_dim 128 (the
- * decoder's 32 / 8 fits); larger shapes return VOX_ERR_RANGE with a message
- * in vox_last_error().  The array starts at zero when the library is loaded;
- * every call writes each record it reads and leaves the counters at zero
- * again (a call whose bounded wait gave up -- a non-zero
- * vox_device_status -- may leave them set: reload the library then).
+ * go to one fixed array in device memory that is part of the loaded library
+ * (about 1.2 MiB), sized for at most 8 kv heads with at most 4 query heads
+ * per kv head at head_dim 128 (the decoder's 32 / 8 fits); larger shapes
+ * return VOX_ERR_RANGE with a message in vox_last_error().  Nothing in the
+ * array needs to start at zero: every call writes each record it reads.
  * All calls on one device share the array, so two calls that overlap on the
  * GPU (other streams, concurrent graph replays) corrupt each other's
  * results: order them on one stream.  The first call on each device looks
@@ -385,7 +378,7 @@ vox_status vox_decoder_step(const vox_decoder *dec, void *stream);
 
 /* vox_decoder_step_kernels -- the same step as a sequence of launches of the
  * library's kernels on one stream (embedding row, per layer the QKV GEMV with
- * rolling append, attention (with its merge), Wo, W1||W3 and W2 GEMVs, then the LM
+ * rolling append, attention + combine, Wo, W1||W3 and W2 GEMVs, then the LM
  * head with argmax and the position advance), each with programmatic
  * dependent launch; the sequence can be captured in a CUDA graph.  Errors:
  * NULL fields -> VOX_ERR_NULL; shapes that do not match the weights, a group

@@ -367,8 +367,7 @@ def attn_case(env, n_q, n_kv, hd, W, pos, seed=0, nan_fill=False):
     kc, vc = WL.bf16_dev(kb, "cuda"), WL.bf16_dev(vb, "cuda")
     out = torch.full((n_q, hd), float("nan"), device="cuda")
     wsb = V.vox_gqa_decode_attn_workspace(n_q, n_kv, hd, W)
-    ws = torch.full((wsb,), 0xFF, dtype=torch.uint8, device="cuda")    # the records need no initial contents
-    ws[:(4 * n_kv + 255) // 256 * 256] = 0                              # the arrival counters start at zero
+    ws = torch.full((wsb,), 0xFF, dtype=torch.uint8, device="cuda")    # no initial contents needed
     V.vox_gqa_decode_attn(WL.to_dev(q, "cuda"), kc, vc, out, n_q, n_kv, hd, W, pos, 1.0 / math.sqrt(hd), ws, wsb)
     check_status(V)
     o = np_of(out)
