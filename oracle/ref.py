@@ -293,6 +293,37 @@ def kv_append(k_cache, v_cache, k_new, v_new, pos):
     v_cache[:, s, :] = f32_to_bf16(np.asarray(v_new, np.float32))
 
 
+# ------------------------------------------------------------ paged caches
+# Batched decode (voxtral.c page, "주요 기능": a rolling cache per stream and
+# batched attention).  Reading R16: each sequence of a batch keeps its own
+# rolling cache of W slots, stored in pages of PAGE_SLOTS consecutive slots
+# of every kv head, drawn from a pool [n_pages][n_kv][PAGE_SLOTS][hd]; its
+# table row names the page of each run of PAGE_SLOTS slots.  The paging only
+# decides where a slot is stored: every sequence then follows the
+# single-sequence definitions above unchanged.
+PAGE_SLOTS = 64
+
+
+def paged_to_cache(pool, table_row):
+    """The logical rolling cache [n_kv][W][hd] (W = len(table_row) * 64) of
+    one sequence: slot p is row p mod 64 of page table_row[p // 64]."""
+    n_pages, n_kv, ps, hd = pool.shape
+    W = len(table_row) * ps
+    out = np.empty((n_kv, W, hd), pool.dtype)
+    for c, page in enumerate(table_row):
+        out[:, c * ps:(c + 1) * ps, :] = pool[page]
+    return out
+
+
+def paged_append(k_pool, v_pool, table_row, k_new, v_new, pos):
+    """kv_append for a paged sequence: the slot pos mod W, in its page."""
+    W = len(table_row) * PAGE_SLOTS
+    s = kv_slot(pos, W)
+    page, row = table_row[s // PAGE_SLOTS], s % PAGE_SLOTS
+    k_pool[page, :, row, :] = f32_to_bf16(np.asarray(k_new, np.float32))
+    v_pool[page, :, row, :] = f32_to_bf16(np.asarray(v_new, np.float32))
+
+
 def argmax_lowest(v):
     """Greedy argmax, lowest index on ties (R11); numpy's argmax does this."""
     return int(np.argmax(np.asarray(v)))

@@ -34,6 +34,9 @@ ADAPTER_ID = 3_000_000      # adapter first Linear, Q4_0 3072 x 5120
 ENC_X_ID = 3_000_001        # encoder chunk input rows
 ADAPTER2_ID = 3_000_002     # adapter second Linear, Q4_0 3072 x 3072
 SWEEP_BASE = 4_000_000      # batched-shape sweep tensors
+# batched decode: layer l's page pools use ids BATCH_BASE + 16*l + {0: K, 1: V}
+BATCH_BASE = 5_000_000
+BATCH_TABLE_ID = 5_999_999  # page assignment of the batch's sequences
 
 D_SCALE = 0.002
 
@@ -166,3 +169,24 @@ def encoder_layer_history(shape: EncoderShape, layer: int, seed: int = 0):
     base = ENC_BASE + DEC_STRIDE * layer
     shp = (shape.window, shape.dim)
     return bf16_normal(shp, seed, base + E_KHIST), bf16_normal(shp, seed, base + E_VHIST)
+
+
+# --------------------------------------------------------- batched decode
+PAGE_SLOTS = 64
+
+
+def page_pool(shape: DecoderShape, layer: int, n_pages: int, seed: int = 0):
+    """bf16 K and V page pools [n_pages, n_kv_heads, 64, head_dim] of one layer."""
+    base = BATCH_BASE + DEC_STRIDE * layer
+    shp = (n_pages, shape.n_kv_heads, PAGE_SLOTS, shape.head_dim)
+    return bf16_normal(shp, seed, base), bf16_normal(shp, seed, base + 1)
+
+
+def page_table(n_seq: int, window: int, n_pages: int, seed: int = 0) -> np.ndarray:
+    """int32 [n_seq, window / 64]: distinct pages in a random order (every
+    sequence owns window / 64 pages of the pool)."""
+    pps = window // PAGE_SLOTS
+    if n_seq * pps > n_pages:
+        raise ValueError("pool too small for the batch")
+    perm = rng_for(seed, BATCH_TABLE_ID).permutation(n_pages)[:n_seq * pps]
+    return perm.astype(np.int32).reshape(n_seq, pps)

@@ -741,3 +741,85 @@ def test_planted_mistakes_in_metric_and_layers_are_caught():
     for bad in (enc_residual_from_norm, enc_gelu_after_down, enc_window_one_wider):
         with pytest.raises(AssertionError):
             pin_encoder_layer(bad)
+
+
+# ------------------------------------------------------------ paged caches
+def pin_paged(to_cache, append):
+    """Brute force on a tiny pool whose every element holds a code of its own
+    (page, head, row, col): the gathered cache and the appended slot must sit
+    exactly where the page table says (reading R16), and appending through
+    the pages must equal appending to the gathered cache."""
+    P, n_kv, hd = 7, 2, 3
+    pool = np.zeros((P, n_kv, ref.PAGE_SLOTS, hd), np.uint16)
+    for p in range(P):
+        for h in range(n_kv):
+            for r in range(ref.PAGE_SLOTS):
+                for c in range(hd):
+                    pool[p, h, r, c] = ((p * n_kv + h) * ref.PAGE_SLOTS + r) * hd + c
+    table = np.array([5, 0, 3], np.int32)                  # W = 192 slots in pages 5, 0, 3
+    W = len(table) * ref.PAGE_SLOTS
+    cache = to_cache(pool, table)
+    assert cache.shape == (n_kv, W, hd)
+    for h in range(n_kv):
+        for slot in range(W):
+            for c in range(hd):
+                page, row = int(table[slot // ref.PAGE_SLOTS]), slot % ref.PAGE_SLOTS
+                assert cache[h, slot, c] == ((page * n_kv + h) * ref.PAGE_SLOTS + row) * hd + c
+    rng = np.random.default_rng(11)
+    kp, vp = pool.copy(), pool.copy()
+    kc, vc = to_cache(kp, table), to_cache(vp, table)
+    for pos in (0, 1, 63, 64, 191, 192, 200, 3 * W + 70):
+        k = rng.standard_normal((n_kv, hd)).astype(np.float32)
+        v = rng.standard_normal((n_kv, hd)).astype(np.float32)
+        before_k = kp.copy()
+        append(kp, vp, table, k, v, pos)
+        ref.kv_append(kc, vc, k, v, pos)
+        assert np.array_equal(to_cache(kp, table), kc) and np.array_equal(to_cache(vp, table), vc)
+        changed = np.argwhere(kp != before_k)
+        slot = pos % W
+        assert all(int(p) == table[slot // ref.PAGE_SLOTS] and int(r) == slot % ref.PAGE_SLOTS
+                   for p, _, r, _ in changed)
+    assert np.array_equal(kp[[1, 2, 4, 6]], pool[[1, 2, 4, 6]])   # pages nobody owns stay untouched
+
+
+def test_paged_cache_bruteforce():
+    pin_paged(ref.paged_to_cache, ref.paged_append)
+
+
+def test_paged_attention_equals_contiguous():
+    """A batch of sequences on one pool: each sequence's attention is the
+    single-sequence attention of its gathered cache; identity tables reduce to
+    a plain reshape of the pool."""
+    import synth
+
+    shape = synth.DecoderShape(n_layers=1, n_q_heads=4, n_kv_heads=2, head_dim=16, window=128)
+    kp, vp = synth.page_pool(shape, 0, 5, 3)
+    ident = np.array([0, 1], np.int32)
+    assert np.array_equal(ref.paged_to_cache(kp, ident), kp[:2].transpose(1, 0, 2, 3).reshape(2, 128, 16))
+    table = synth.page_table(2, 128, 5, 3)
+    q = np.random.default_rng(4).standard_normal((2, 4, 16)).astype(np.float32)
+    for s, pos in enumerate((40, 300)):
+        kc, vc = ref.paged_to_cache(kp, table[s]), ref.paged_to_cache(vp, table[s])
+        o = ref.gqa_attn(q[s], kc, vc, pos)
+        assert np.allclose(o, ref.c_gqa_attn(q[s], kc, vc, pos), rtol=0, atol=1e-12)
+
+
+def test_planted_mistakes_in_paging_are_caught():
+    def row_major_pages(pool, table_row):             # page and row swapped
+        n_pages, n_kv, ps, hd = pool.shape
+        out = np.empty((n_kv, len(table_row) * ps, hd), pool.dtype)
+        for slot in range(len(table_row) * ps):
+            out[:, slot] = pool[table_row[slot % len(table_row)], :, slot // len(table_row)]
+        return out
+
+    def ignores_table(pool, table_row):
+        return ref.paged_to_cache(pool, np.arange(len(table_row)))
+
+    def append_wrong_row(k_pool, v_pool, table_row, k_new, v_new, pos):
+        ref.paged_append(k_pool, v_pool, table_row, k_new, v_new, pos + 1)
+
+    for bad in (row_major_pages, ignores_table):
+        with pytest.raises(AssertionError):
+            pin_paged(bad, ref.paged_append)
+    with pytest.raises(AssertionError):
+        pin_paged(ref.paged_to_cache, append_wrong_row)
