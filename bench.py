@@ -55,13 +55,15 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
-    p.add_argument("--workload", choices=["decoder", "gemv", "layer", "encoder", "sweep", "kernel"],
+    p.add_argument("--workload", choices=["decoder", "gemv", "layer", "encoder", "sweep", "kernel", "batch"],
                    default="decoder",
                    help="decoder: the headline line (default); gemv: the single 4096x3072 GEMV; layer: one "
                         "decoder layer at KV 1024; encoder: the 32-layer encoder chunk at M=256 "
                         "and its GEMMs; sweep: the decoder shapes at M in {1,4,16,64,256} and the attention at "
                         "KV in {512, 4096, 8192 wrapped}; kernel: a few launches of one kernel on one small "
-                        "case (--kernel, --shape, --launches), sized for an ncu capture")
+                        "case (--kernel, --shape, --launches), sized for an ncu capture; batch: --seqs "
+                        "sequences stepped together over paged caches (26 layers, KV 8192 wrapped)")
+    p.add_argument("--seqs", type=int, default=8, help="batch workload: sequences (1..8)")
     p.add_argument("--kernel", choices=["gemv", "attn", "gemm", "step"], default="gemv",
                    help="kernel workload: gemv N K (M = 1), attn POS (decoder-shaped layer), gemm N K M, "
                         "step L (the persistent decoder step with L full-size layers, KV 8192 wrapped)")
@@ -852,6 +854,80 @@ def run_layer(args):
     return 0
 
 
+def run_batch(args):
+    """Batched decode: --seqs sequences, each with its own 8192-slot rolling
+    cache in 64-slot pages (filled past one wrap, positions 8192 + 300 + 37 s),
+    stepped together through the 26-layer decoder: every weight is streamed
+    once per step for all sequences (the GEMV at m = seqs rows), the
+    attention reads every sequence's cache.  One step = one replay of the
+    captured vox_decoder_batch_step graph.  Reports tokens/s and the step's
+    algorithmic GB/s (weights once + every sequence's cache)."""
+    import torch
+
+    import synth
+    from bit_quantized_transformer_b200 import build
+
+    build.build()
+    from bit_quantized_transformer_b200 import vox as V
+    from bit_quantized_transformer_b200 import workloads as WL
+
+    n = max(1, min(8, args.seqs))
+    shape = synth.DecoderShape()
+    positions = [FILLED + 37 * s for s in range(n)]
+    tokens = [(17 + 7919 * s) % shape.vocab for s in range(n)]
+    bm = WL.BatchDecoderModel(shape, n, positions, tokens, device_fill=True)
+    step_bytes = bm.weight_bytes() + bm.kv_bytes(positions)
+    g = bm.capture()
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    reps = max(3, args.steps)
+    clocks = ClockSampler(0)
+    clocks.start()
+    ms = time_fn(g.replay, reps, 1)
+    clk = clocks.stop()
+    assert V.vox_device_status(True) == 0
+    ms_step = ms / reps
+    gbs = step_bytes / (ms_step / 1e3) / 1e9
+    peak, peak_src = measured_peaks()
+    # end to end through the API: tokens in from pinned host memory, next tokens out, every step
+    tok_h = torch.tensor(tokens, dtype=torch.int32).pin_memory()
+    out_h = torch.empty(n, dtype=torch.int32).pin_memory()
+
+    def e2e_step():
+        bm.token.copy_(tok_h, non_blocking=True)
+        g.replay()
+        out_h.copy_(bm.token, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    e2e_n = max(3, min(reps, 50))
+    t0 = time.perf_counter()
+    for _ in range(e2e_n):
+        e2e_step()
+    e2e_ms = (time.perf_counter() - t0) * 1e3 / e2e_n
+    assert V.vox_device_status(True) == 0
+    del g
+    line = {"metric": "batched decode tokens/s (sequences x steps / s), paged per-sequence caches",
+            "value": n * 1e3 / ms_step, "unit": "tokens/s", "n_gpus": 1, "steps": reps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "q4_0 weights, fp16/bf16 tensor-core inputs, f32 accumulate",
+            "data": "synthetic (pools drawn on the device)",
+            "config": {"workload": f"decoder_batch_q4_26L_kv8192wrapped_{n}seq_paged", "sequences": n,
+                       "positions": positions, "page_slots": 64, "pages": bm.n_pages,
+                       "bytes_per_step": step_bytes, "l2": "inputs larger than L2 (no flush)"},
+            "gbs": gbs, "hbm_frac": gbs / peak,
+            "roofline": {"bound": "hbm", "kernel": "the batched step's kernel sequence", "achieved": gbs,
+                         "peak": peak, "unit": "GB/s", "frac": gbs / peak, "traffic": None,
+                         "peak_source": peak_src},
+            "gpu_launches": reps * bm.launches(), "clocks": clk,
+            "e2e": {"value": n * 1e3 / e2e_ms, "unit": "tokens/s", "h2d_bytes_per_step": 4 * n,
+                    "d2h_bytes_per_step": 4 * n, "ms_per_step": e2e_ms,
+                    "api": "vox_decoder_batch_step graph replay, tokens H2D before and D2H after every step"}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def omp_threads():
     return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
@@ -936,6 +1012,8 @@ def main(argv=None):
         return run_gemv(args)
     if args.workload == "layer":
         return run_layer(args)
+    if args.workload == "batch":
+        return run_batch(args)
     return run_ours(args)
 
 

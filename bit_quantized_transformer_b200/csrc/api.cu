@@ -8,7 +8,7 @@ namespace vox {
 const char* last_error_text();
 vox_status launch_q4_pack(const uint8_t*, int64_t, int64_t, int, uint8_t*, cudaStream_t);
 vox_status launch_q4_dequant(const uint8_t*, int64_t, int64_t, int64_t, const int32_t*, int64_t, void*, int,
-                             int64_t, cudaStream_t);
+                             int64_t, cudaStream_t, int gather = 0);
 vox_status launch_q4_gemv(const uint8_t*, int64_t, int64_t, const float*, int64_t, int64_t, float*, int64_t,
                           const vox_epilogue*, void*, cudaStream_t);
 size_t gemv_workspace_bytes(int64_t n, int64_t k, int op);
@@ -18,7 +18,10 @@ vox_status launch_kv_append(void*, void*, const void*, const void*, int, int, in
                             cudaStream_t);
 vox_status launch_gqa_decode_attn(const float*, const void*, const void*, float*, int, int, int, int, int64_t,
                                   const int64_t*, float, void*, cudaStream_t);
-size_t attn_workspace_bytes(int n_kv, int hd, int window);
+size_t attn_workspace_bytes(int n_kv, int hd, int window, int n_seq = 1);
+vox_status launch_gqa_decode_attn_seqs(const float*, const void*, const void*, float*, int, int, int, int, int64_t,
+                                       const int64_t*, float, void*, cudaStream_t, int, const int32_t*, int64_t,
+                                       int64_t);
 vox_status launch_window_attn(const void*, int64_t, const void*, const void*, int64_t, int64_t, const void*,
                               const void*, int64_t, int64_t, void*, int, int64_t, int, int, int, float,
                               cudaStream_t);
@@ -98,7 +101,7 @@ static vox_status check_epilogue(const vox_epilogue* ep, int64_t n, int64_t k, i
                                  bool allow_rms, bool gemm)
 {
     int op = ep ? ep->op : VOX_EP_NONE;
-    if (op < VOX_EP_NONE || op > VOX_EP_ARGMAX) return VOX_ERR_RANGE;
+    if (op < VOX_EP_NONE || op > VOX_EP_KV_APPEND_PAGED) return VOX_ERR_RANGE;
     if (ep && ep->rmsnorm && !allow_rms) return VOX_ERR_RANGE;
     if (ep && ep->rmsnorm && !(ep->eps >= 0.f)) return VOX_ERR_RANGE;
     int64_t ncols = op == VOX_EP_SILU_MUL ? n / 2 : n;
@@ -118,6 +121,13 @@ static vox_status check_epilogue(const vox_epilogue* ep, int64_t n, int64_t k, i
         if (ep->n_kv_heads < 1 || ep->head_dim < 1 || ep->q_rows < 0) return VOX_ERR_SHAPE;
         if ((int64_t)ep->q_rows + 2LL * ep->n_kv_heads * ep->head_dim > n) return VOX_ERR_SHAPE;
         if (ep->window < 1 || (!ep->pos_dev && ep->pos < 0)) return VOX_ERR_RANGE;
+        break;
+    case VOX_EP_KV_APPEND_PAGED:
+        if (gemm) return VOX_ERR_RANGE;
+        if (!ep->k_cache || !ep->v_cache || !ep->page_table || !ep->pos_dev) return VOX_ERR_NULL;
+        if (ep->n_kv_heads < 1 || ep->head_dim < 1 || ep->q_rows < 0) return VOX_ERR_SHAPE;
+        if ((int64_t)ep->q_rows + 2LL * ep->n_kv_heads * ep->head_dim > n) return VOX_ERR_SHAPE;
+        if (ep->window < 64 || ep->window % 64 || ep->n_pages < 1) return VOX_ERR_RANGE;
         break;
     case VOX_EP_ARGMAX:
         if (gemm) return VOX_ERR_RANGE;
@@ -247,6 +257,33 @@ vox_status vox_gqa_decode_attn(const float* q, const void* k_cache, const void* 
     if (!al16(k_cache) || !al16(v_cache) || !al16(workspace) || !al16(out)) return VOX_ERR_ALIGN;
     return launch_gqa_decode_attn(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_dim, window, pos, nullptr,
                                   scale, workspace, S(stream));
+}
+
+size_t vox_gqa_decode_attn_paged_workspace(int32_t n_seq, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                           int32_t window)
+{
+    if (n_seq < 1 || n_q_heads < 1 || n_kv_heads < 1 || head_dim < 1 || window < 1) return 0;
+    return attn_workspace_bytes(n_kv_heads, head_dim, window, n_seq);
+}
+
+vox_status vox_gqa_decode_attn_paged(const float* q, const void* k_pool, const void* v_pool, int64_t n_pages,
+                                     const int32_t* page_table, const int64_t* pos, int32_t n_seq, float* out,
+                                     int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t window,
+                                     float scale, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!q || !k_pool || !v_pool || !page_table || !pos || !out) return VOX_ERR_NULL;
+    if (n_seq < 1 || n_seq > 64) return VOX_ERR_RANGE;
+    if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return VOX_ERR_RANGE;
+    if (n_q_heads / n_kv_heads > 8 || n_kv_heads > 512) return VOX_ERR_RANGE;
+    if (window < 64 || window % 64 || n_pages < 1) return VOX_ERR_RANGE;
+    if (head_dim != 128) return VOX_ERR_SHAPE;
+    if (n_pages > 0x7fffff00LL / (64LL * n_kv_heads)) return VOX_ERR_SHAPE;
+    if (!workspace) return VOX_ERR_WORKSPACE;
+    if (ws_bytes < vox_gqa_decode_attn_paged_workspace(n_seq, n_q_heads, n_kv_heads, head_dim, window))
+        return VOX_ERR_WORKSPACE;
+    if (!al16(k_pool) || !al16(v_pool) || !al16(workspace) || !al16(out)) return VOX_ERR_ALIGN;
+    return launch_gqa_decode_attn_seqs(q, k_pool, v_pool, out, n_q_heads, n_kv_heads, head_dim, window, 0, pos, scale,
+                                       workspace, S(stream), n_seq, page_table, n_pages, 0);
 }
 
 vox_status vox_window_attn(const void* q, int64_t ldq, const void* k_hist, const void* v_hist, int64_t ld_hist,

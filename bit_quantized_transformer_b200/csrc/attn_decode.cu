@@ -95,7 +95,26 @@ struct AttnArgs {
     int32_t stages;
     int32_t rec_floats;                        // record stride (floats, a multiple of 4)
     int32_t rmax;                              // record slots per kv head
+    // Several sequences (blockIdx.y = sequence s): q, out, the records and
+    // pos_dev advance by one sequence's size.  With a page table the caches
+    // are pools of 64-slot pages [page][n_kv][64][hd]; sequence s's slot p
+    // lives in page pages[s * pps + p / 64] (null: one contiguous cache
+    // [n_kv][window][hd]).
+    const int32_t* pages;
+    int32_t pps;
+    int64_t n_pages;
+    int64_t q_ld;                              // floats from one sequence's q to the next
 };
+
+// First cache row (in the tensor map's rows) of chunk ci of kv head kh of
+// sequence s; -1 for a page index outside the pool.
+__device__ __forceinline__ int64_t attn_chunk_row(const AttnArgs& a, int s, int64_t kh, int64_t ci)
+{
+    if (!a.pages) return kh * a.window + ci * kAttnChunk;
+    const int64_t pg = __ldg(a.pages + (int64_t)s * a.pps + ci);
+    if (pg < 0 || pg >= a.n_pages) return -1;
+    return (pg * a.n_kv + kh) * kAttnChunk;
+}
 
 // Partial record of one CTA for one kv head: O[group][hd], then (m, l) per
 // query head of the group, padded to 16 bytes.  The records of kv head kh
@@ -110,21 +129,23 @@ static int env_int_attn(const char* name, int dflt, int lo, int hi)
     return v < lo ? lo : (v > hi ? hi : v);
 }
 
-static int64_t attn_grid(int n_kv, int window)
+// CTAs per sequence: the SMs (times the knob) shared evenly by the sequences.
+static int64_t attn_grid(int n_kv, int window, int n_seq)
 {
     int64_t chunks = (int64_t)n_kv * ceil_div(window, kAttnChunk);
-    int64_t G = (int64_t)env_int_attn("VOX_ATTN_CTAS_PER_SM", 1, 1, 2) * device_sm_count();
+    int64_t G = (int64_t)env_int_attn("VOX_ATTN_CTAS_PER_SM", 1, 1, 2) * device_sm_count() / n_seq;
     if (G > chunks) G = chunks;
     if (G < n_kv) G = n_kv;                    // then no CTA spans more than two kv heads
     if (G > kAttnMaxCtas) G = kAttnMaxCtas;
     return G;
 }
 
-// Workspace: rmax partial records per kv head (room for the largest group).
-size_t attn_workspace_bytes(int n_kv, int hd, int window)
+// Workspace: rmax partial records per kv head (room for the largest group),
+// per sequence.
+size_t attn_workspace_bytes(int n_kv, int hd, int window, int n_seq)
 {
     (void)window;
-    return ((size_t)n_kv * attn_rmax(n_kv) * attn_rec_floats(kAttnMaxGroup, hd) * sizeof(float) + 255) &
+    return ((size_t)n_seq * n_kv * attn_rmax(n_kv) * attn_rec_floats(kAttnMaxGroup, hd) * sizeof(float) + 255) &
            ~(size_t)255;
 }
 
@@ -163,6 +184,9 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t G = gridDim.x, b = blockIdx.x;
     const int W = a.window;
+    const int seq = blockIdx.y;
+    const float* q_seq = a.q + (int64_t)seq * a.q_ld;
+    float* ws_seq = a.ws + (int64_t)seq * a.n_kv * a.rmax * a.rec_floats;
 
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -178,7 +202,7 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     // step; every kernel here triggers its dependents only after its own
     // griddepcontrol.wait, so when this kernel starts that writer has
     // finished and the early read is safe.
-    const int64_t pos = a.pos_dev ? *a.pos_dev : a.pos;
+    const int64_t pos = a.pos_dev ? a.pos_dev[seq] : a.pos;
     const int64_t n_valid = pos + 1 < W ? pos + 1 : W;
     const int64_t nch = (n_valid + kAttnChunk - 1) / kAttnChunk;      // chunks per kv head
     const int64_t total = (int64_t)a.n_kv * nch;
@@ -195,7 +219,11 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
             for (int64_t c = c_begin; c < c_end; ++c) {
                 if (!s_fail[0] && !mbar_wait_bounded(&empty[slot], ph ^ 1u, 0x201)) s_fail[0] = 1;
                 if (s_fail[0]) break;
-                const int32_t row = (int32_t)(kh * W + ci * kAttnChunk);
+                // a page outside the pool reads the fill value (zeros): the
+                // box starts at the map's row count, wholly past its rows
+                const int64_t crow = attn_chunk_row(a, seq, kh, ci);
+                if (crow < 0) atomicCAS(&g_vox_device_status, 0, 0x203);
+                const int32_t row = (int32_t)(crow < 0 ? a.n_pages * a.n_kv * kAttnChunk : crow);
                 uint8_t* st = smem + SL.ring + slot * kAttnStageBytes;
                 mbar_arrive_expect_tx(&full[slot], kAttnStageBytes);
                 tma_load_2d(st + 0 * kAttnTileBytes, &kmap, 0, row, &full[slot]);
@@ -249,7 +277,7 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         named_barrier(1, 32 * kAttnWarps);
         (void)sidx;
         const int64_t bf_seg = attn_owner(kh_seg * nch, total, G);
-        float* rec = a.ws + ((size_t)kh_seg * a.rmax + (size_t)(b - bf_seg)) * a.rec_floats;
+        float* rec = ws_seq + ((size_t)kh_seg * a.rmax + (size_t)(b - bf_seg)) * a.rec_floats;
         for (int i = tid; i < group * kAttnHd; i += 32 * kAttnWarps) {
             const int hh = i / kAttnHd, cc = i % kAttnHd;
             float M = -INFINITY;
@@ -287,7 +315,7 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
             seg_head = kh;
             // q' = q * scale * log2(e), split into bf16 hi + lo B fragments (heads >= group are zero)
             const bool ok = g < group;
-            const float* qr = a.q + ((int64_t)kh * group + (ok ? g : 0)) * kAttnHd;
+            const float* qr = q_seq + ((int64_t)kh * group + (ok ? g : 0)) * kAttnHd;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
@@ -309,12 +337,13 @@ gqa_decode_attn_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
 
         // Generic-proxy fix-ups of this warp's 16 rows of the TMA-written stage.
         bool touched = false;
-        if (new_slot >= slot0 && new_slot < slot0 + 16) {
+        const int64_t crow = (new_slot >= slot0 && new_slot < slot0 + 16) ? attn_chunk_row(a, seq, kh, ci) : -1;
+        if (crow >= 0) {
             // reload the newest row (K and V, 4 x 128 bytes) written by the upstream kernel
             const uint32_t r = (uint32_t)(new_slot - ci * kAttnChunk);
             const int part = lane >> 3, unit = lane & 7;       // tiles K lo, K hi, V lo, V hi
             const uint16_t* src = (part < 2 ? a.kcache : a.vcache) +
-                                  (kh * W + new_slot) * kAttnHd + (part & 1) * 64 + unit * 8;
+                                  (crow + r) * kAttnHd + (part & 1) * 64 + unit * 8;
             const uint4 v = *reinterpret_cast<const uint4*>(src);
             *reinterpret_cast<uint4*>(stp + part * kAttnTileBytes + sw128_offset(r, (uint32_t)unit)) = v;
             touched = true;
@@ -443,13 +472,14 @@ __global__ void __launch_bounds__(32) attn_combine_kernel(const AttnArgs a, int6
     const int group = a.group;
     const int kh = blockIdx.x / group, gi = blockIdx.x - kh * group, lane = threadIdx.x;
     const int W = a.window;
-    const int64_t pos = a.pos_dev ? *a.pos_dev : a.pos;
+    const int seq = blockIdx.y;
+    const int64_t pos = a.pos_dev ? a.pos_dev[seq] : a.pos;
     const int64_t n_valid = pos + 1 < W ? pos + 1 : W;
     const int64_t nch = (n_valid + kAttnChunk - 1) / kAttnChunk;
     const int64_t total = (int64_t)a.n_kv * nch;
     const int64_t bf = attn_owner((int64_t)kh * nch, total, G), bl = attn_owner((int64_t)kh * nch + nch - 1, total, G);
     const int nrec = (int)(bl - bf + 1);
-    const float* recs = a.ws + (size_t)kh * a.rmax * a.rec_floats;
+    const float* recs = a.ws + ((size_t)seq * a.n_kv + kh) * a.rmax * a.rec_floats;
     float M = -INFINITY, L = 0.f;
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int r0 = 0; r0 < nrec; r0 += kCombineBatch) {
@@ -487,21 +517,23 @@ __global__ void __launch_bounds__(32) attn_combine_kernel(const AttnArgs a, int6
         M = mb;
     }
     const float inv = 1.0f / L;
-    *reinterpret_cast<float4*>(a.out + ((int64_t)kh * group + gi) * kAttnHd + 4 * lane) =
+    *reinterpret_cast<float4*>(a.out + ((int64_t)seq * a.n_q + (int64_t)kh * group + gi) * kAttnHd + 4 * lane) =
         make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
 }
 
-vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc, float* out, int n_q, int n_kv,
-                                  int hd, int window, int64_t pos, const int64_t* pos_dev, float scale, void* ws,
-                                  cudaStream_t s)
+// One sequence with one contiguous cache (n_seq = 1, pages = null) or n_seq
+// sequences over paged pools of n_pages pages.
+vox_status launch_gqa_decode_attn_seqs(const float* q, const void* kc, const void* vc, float* out, int n_q, int n_kv,
+                                       int hd, int window, int64_t pos, const int64_t* pos_dev, float scale, void* ws,
+                                       cudaStream_t s, int n_seq, const int32_t* pages, int64_t n_pages, int64_t q_ld)
 {
+    const uint64_t rows = pages ? (uint64_t)n_pages * n_kv * kAttnChunk : (uint64_t)n_kv * window;
     CUtensorMap kmap, vmap;
-    vox_status st = make_tmap_2d(&kmap, kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)hd,
-                                 (uint64_t)n_kv * window, (uint64_t)hd * 2, 64, kAttnChunk,
-                                 CU_TENSOR_MAP_SWIZZLE_128B);
+    vox_status st = make_tmap_2d(&kmap, kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)hd, rows,
+                                 (uint64_t)hd * 2, 64, kAttnChunk, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != VOX_OK) return st;
-    st = make_tmap_2d(&vmap, vc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)hd, (uint64_t)n_kv * window,
-                      (uint64_t)hd * 2, 64, kAttnChunk, CU_TENSOR_MAP_SWIZZLE_128B);
+    st = make_tmap_2d(&vmap, vc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)hd, rows, (uint64_t)hd * 2, 64,
+                      kAttnChunk, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != VOX_OK) return st;
 
     AttnArgs a = {};
@@ -521,16 +553,29 @@ vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc
     a.rec_floats = attn_rec_floats(a.group, hd);
     a.rmax = attn_rmax(n_kv);
     a.stages = env_int_attn("VOX_ATTN_STAGES", 3, 2, kAttnMaxStages);
+    a.pages = pages;
+    a.q_ld = q_ld > 0 ? q_ld : (int64_t)n_q * hd;
+    a.pps = window / kAttnChunk;
+    a.n_pages = n_pages;
     const AttnSmem SL = attn_smem_layout(a.stages);
 
     static std::atomic<unsigned long long> attr_done{0};
     st = smem_attr_per_device(reinterpret_cast<const void*>(gqa_decode_attn_kernel),
                               (int)attn_smem_layout(kAttnMaxStages).total, attr_done);
     if (st != VOX_OK) return st;
-    const int64_t G = attn_grid(n_kv, window);
-    st = launch_pdl(gqa_decode_attn_kernel, dim3((unsigned)G), dim3(kAttnThreads), SL.total, s, kmap, vmap, a);
+    const int64_t G = attn_grid(n_kv, window, n_seq);
+    st = launch_pdl(gqa_decode_attn_kernel, dim3((unsigned)G, (unsigned)n_seq), dim3(kAttnThreads), SL.total, s,
+                    kmap, vmap, a);
     if (st != VOX_OK) return st;
-    return launch_pdl(attn_combine_kernel, dim3((unsigned)(n_kv * a.group)), dim3(32), 0, s, a, G);
+    return launch_pdl(attn_combine_kernel, dim3((unsigned)(n_kv * a.group), (unsigned)n_seq), dim3(32), 0, s, a, G);
+}
+
+vox_status launch_gqa_decode_attn(const float* q, const void* kc, const void* vc, float* out, int n_q, int n_kv,
+                                  int hd, int window, int64_t pos, const int64_t* pos_dev, float scale, void* ws,
+                                  cudaStream_t s)
+{
+    return launch_gqa_decode_attn_seqs(q, kc, vc, out, n_q, n_kv, hd, window, pos, pos_dev, scale, ws, s, 1,
+                                       nullptr, 0, 0);
 }
 
 // --------------------------------------------- allocation-free entry point

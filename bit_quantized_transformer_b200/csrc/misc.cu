@@ -138,16 +138,17 @@ vox_status launch_cast_rows(const float* x, int64_t m, int64_t n, int64_t ldx, v
 }
 
 // --------------------------------------------------------- position advance
-__global__ void advance_pos_kernel(int64_t* pos)
+__global__ void advance_pos_kernel(int64_t* pos, int n)
 {
     pdl_wait();
     pdl_launch_dependents();
-    if (threadIdx.x == 0) *pos += 1;
+    if ((int)threadIdx.x < n) pos[threadIdx.x] += 1;
 }
 
-vox_status launch_advance_pos(int64_t* pos, cudaStream_t s)
+// Positions pos[0 .. n) advance by one (n <= 32).
+vox_status launch_advance_pos(int64_t* pos, cudaStream_t s, int n)
 {
-    return launch_pdl(advance_pos_kernel, dim3(1), dim3(32), 0, s, pos);
+    return launch_pdl(advance_pos_kernel, dim3(1), dim3(32), 0, s, pos, n);
 }
 
 }  // namespace vox

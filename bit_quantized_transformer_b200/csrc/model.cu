@@ -24,14 +24,17 @@
 
 namespace vox {
 vox_status launch_q4_dequant(const uint8_t*, int64_t, int64_t, int64_t, const int32_t*, int64_t, void*, int,
-                             int64_t, cudaStream_t);
+                             int64_t, cudaStream_t, int gather = 0);
 vox_status launch_q4_gemv(const uint8_t*, int64_t, int64_t, const float*, int64_t, int64_t, float*, int64_t,
                           const vox_epilogue*, void*, cudaStream_t);
 size_t gemv_workspace_bytes(int64_t n, int64_t k, int op);
 vox_status launch_gqa_decode_attn(const float*, const void*, const void*, float*, int, int, int, int, int64_t,
                                   const int64_t*, float, void*, cudaStream_t);
-size_t attn_workspace_bytes(int n_kv, int hd, int window);
-vox_status launch_advance_pos(int64_t*, cudaStream_t);
+size_t attn_workspace_bytes(int n_kv, int hd, int window, int n_seq = 1);
+vox_status launch_gqa_decode_attn_seqs(const float*, const void*, const void*, float*, int, int, int, int, int64_t,
+                                       const int64_t*, float, void*, cudaStream_t, int, const int32_t*, int64_t,
+                                       int64_t);
+vox_status launch_advance_pos(int64_t*, cudaStream_t, int n = 1);
 vox_status launch_rmsnorm(const float*, int64_t, int64_t, int64_t, float, const float*, void*, int, int64_t,
                           cudaStream_t);
 vox_status launch_cast_rows(const float*, int64_t, int64_t, int64_t, void*, int, int64_t, cudaStream_t);
@@ -77,8 +80,9 @@ size_t dec_ps_offset(const vox_decoder* d)
     return g + ((attn_workspace_bytes(d->n_kv_heads, d->head_dim, d->window) + 255) & ~(size_t)255);
 }
 
-// Host-side checks shared by both forms of the decoder step.
-vox_status check_decoder(const vox_decoder* d)
+// Host-side checks shared by both forms of the decoder step (and, without
+// the workspace size, by the batched step).
+vox_status check_decoder(const vox_decoder* d, bool check_ws = true)
 {
     if (!d) return VOX_ERR_NULL;
     if (!d->wqkv || !d->wo || !d->w13 || !d->w2 || !d->k_cache || !d->v_cache || !d->token || !d->pos || !d->x ||
@@ -88,7 +92,7 @@ vox_status check_decoder(const vox_decoder* d)
         d->n_q_heads / d->n_kv_heads > 8 || d->dim % 32 || d->ffn % 32 || d->ffn % 8)
         return VOX_ERR_SHAPE;
     if (d->window < 1) return VOX_ERR_RANGE;
-    if (d->ws_bytes < vox_decoder_workspace(d)) return VOX_ERR_WORKSPACE;
+    if (check_ws && d->ws_bytes < vox_decoder_workspace(d)) return VOX_ERR_WORKSPACE;
     if (!al16(d->workspace)) return VOX_ERR_ALIGN;
     const int64_t D = d->dim, QD = (int64_t)d->n_q_heads * d->head_dim, KVD = (int64_t)d->n_kv_heads * d->head_dim;
     const int64_t F = d->ffn;
@@ -202,6 +206,95 @@ vox_status vox_decoder_step_kernels(const vox_decoder* d, void* stream)
                              d->vocab, &am, ws_g, s)))
         return st;
     return launch_advance_pos(d->pos, s);
+}
+
+// ------------------------------------------------------------ batched step
+static size_t batch_gemv_ws(const vox_decoder_batch* b) { return (dec_gemv_ws(&b->d) + 255) & ~(size_t)255; }
+
+size_t vox_decoder_batch_workspace(const vox_decoder_batch* b)
+{
+    if (!b || b->n_seq < 1 || b->n_seq > 8 || b->d.dim < 32 || b->d.vocab < 1 || b->d.n_kv_heads < 1 ||
+        b->d.window < 1 || b->d.n_layers < 1 || b->d.n_q_heads < b->d.n_kv_heads)
+        return 0;
+    return batch_gemv_ws(b) +
+           ((attn_workspace_bytes(b->d.n_kv_heads, b->d.head_dim, b->d.window, b->n_seq) + 255) & ~(size_t)255);
+}
+
+vox_status vox_decoder_batch_step(const vox_decoder_batch* b, void* stream)
+{
+    if (!b) return VOX_ERR_NULL;
+    const vox_decoder* d = &b->d;
+    vox_status st = check_decoder(d, false);
+    if (st) return st;
+    if (b->n_seq < 1 || b->n_seq > 8) return VOX_ERR_RANGE;
+    if (!b->page_table) return VOX_ERR_NULL;
+    if (d->window < 64 || d->window % 64 || b->n_pages < 1) return VOX_ERR_RANGE;
+    if (b->n_pages > 0x7fffff00LL / (64LL * d->n_kv_heads)) return VOX_ERR_SHAPE;
+    if (d->ws_bytes < vox_decoder_batch_workspace(b)) return VOX_ERR_WORKSPACE;
+    const int64_t m = b->n_seq;
+    const int64_t D = d->dim, QD = (int64_t)d->n_q_heads * d->head_dim, KVD = (int64_t)d->n_kv_heads * d->head_dim;
+    const int64_t F = d->ffn;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws_g = static_cast<uint8_t*>(d->workspace);
+    uint8_t* ws_a = ws_g + batch_gemv_ws(b);
+    const float scale = 1.0f / sqrtf((float)d->head_dim);
+
+    // x[i] = embedding row of sequence i's token (exact fp32 weights)
+    if ((st = launch_q4_dequant(static_cast<const uint8_t*>(d->embedding.data), d->vocab, D, 0, d->token, m, d->x,
+                                VOX_F32, D, s, 1)))
+        return st;
+    for (int l = 0; l < d->n_layers; ++l) {
+        vox_epilogue e = {};
+        e.op = VOX_EP_KV_APPEND_PAGED;
+        e.rmsnorm = 1;
+        e.eps = d->eps;
+        e.k_cache = d->k_cache[l];
+        e.v_cache = d->v_cache[l];
+        e.n_kv_heads = d->n_kv_heads;
+        e.head_dim = d->head_dim;
+        e.window = d->window;
+        e.q_rows = (int32_t)QD;
+        e.pos_dev = d->pos;
+        e.page_table = b->page_table;
+        e.n_pages = b->n_pages;
+        if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->wqkv[l].data), QD + 2 * KVD, D, d->x, m, D, d->qkv,
+                                 QD + 2 * KVD, &e, ws_g, s)))
+            return st;
+        if ((st = launch_gqa_decode_attn_seqs(d->qkv, d->k_cache[l], d->v_cache[l], d->attn, d->n_q_heads,
+                                              d->n_kv_heads, d->head_dim, d->window, 0, d->pos, scale, ws_a, s,
+                                              (int)m, b->page_table, b->n_pages, QD + 2 * KVD)))
+            return st;
+        vox_epilogue r = {};
+        r.op = VOX_EP_RESIDUAL;
+        r.residual = d->x;
+        r.ldr = D;
+        if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->wo[l].data), D, QD, d->attn, m, QD, d->h, D, &r, ws_g,
+                                 s)))
+            return st;
+        vox_epilogue f = {};
+        f.op = VOX_EP_SILU_MUL;
+        f.rmsnorm = 1;
+        f.eps = d->eps;
+        if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->w13[l].data), 2 * F, D, d->h, m, D, d->act, F, &f,
+                                 ws_g, s)))
+            return st;
+        vox_epilogue r2 = {};
+        r2.op = VOX_EP_RESIDUAL;
+        r2.residual = d->h;
+        r2.ldr = D;
+        if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->w2[l].data), D, F, d->act, m, F, d->x, D, &r2, ws_g,
+                                 s)))
+            return st;
+    }
+    vox_epilogue am = {};
+    am.op = VOX_EP_ARGMAX;
+    am.rmsnorm = 1;
+    am.eps = d->eps;
+    am.argmax = d->token;
+    if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->lm_head.data), d->vocab, D, d->x, m, D, d->logits,
+                             d->vocab, &am, ws_g, s)))
+        return st;
+    return launch_advance_pos(d->pos, s, (int)m);
 }
 
 vox_status vox_encoder_chunk(const vox_encoder* e, void* stream)

@@ -90,6 +90,8 @@ struct GemvArgs {
     int32_t stages;
     int32_t pre;                             // ring stages issued before griddepcontrol.wait
     int32_t evict_first;                     // 1: weight copies marked evict-first in L2
+    const int32_t* pages;                    // KV_APPEND_PAGED: page table [m][window / 64]
+    int64_t n_pages;
 };
 
 // Shared-memory carve-up, computed identically on host and device.
@@ -197,6 +199,24 @@ __device__ __noinline__ GemvBest gemv_epilogue(const GemvArgs& a, int64_t tile, 
                     const int64_t head = rw / a.hd, col = rw - head * a.hd;
                     const int64_t slot_id = (pos + mt) % a.window;
                     cache[(head * a.window + slot_id) * a.hd + col] = f32_to_bf16_bits(val);
+                }
+                break;
+            }
+            case VOX_EP_KV_APPEND_PAGED: {
+                // token mt is sequence mt: its slot pos[mt] mod window, in the page its table names
+                yr[row] = val;
+                const int64_t kvd = (int64_t)a.n_kv * a.hd;
+                const int64_t rel = row - a.q_rows;
+                if (rel >= 0 && rel < 2 * kvd) {
+                    uint16_t* pool = rel < kvd ? a.kcache : a.vcache;
+                    const int64_t rw = rel < kvd ? rel : rel - kvd;
+                    const int64_t head = rw / a.hd, col = rw - head * a.hd;
+                    const int64_t slot_id = a.pos_dev[mt] % a.window;
+                    const int64_t pg = a.pages[(int64_t)mt * (a.window / 64) + slot_id / 64];
+                    if (pg >= 0 && pg < a.n_pages)
+                        pool[((pg * a.n_kv + head) * 64 + slot_id % 64) * a.hd + col] = f32_to_bf16_bits(val);
+                    else
+                        atomicCAS(&g_vox_device_status, 0, 0x105);
                 }
                 break;
             }
@@ -549,7 +569,9 @@ vox_status launch_q4_gemv(const uint8_t* w, int64_t n, int64_t k, const float* x
     a.g = ep ? ep->norm_weight : nullptr;
     a.res = ep ? ep->residual : nullptr;
     a.ldr = ep ? ep->ldr : 0;
-    if (ep && ep->op == VOX_EP_KV_APPEND) {
+    if (ep && (ep->op == VOX_EP_KV_APPEND || ep->op == VOX_EP_KV_APPEND_PAGED)) {
+        a.pages = ep->page_table;
+        a.n_pages = ep->n_pages;
         a.kcache = static_cast<uint16_t*>(ep->k_cache);
         a.vcache = static_cast<uint16_t*>(ep->v_cache);
         a.n_kv = ep->n_kv_heads;

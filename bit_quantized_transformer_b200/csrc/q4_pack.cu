@@ -89,22 +89,33 @@ __global__ void q4_pack_kernel(const uint8_t* __restrict__ gguf, int64_t n, int6
 
 // One thread per (row, block): decodes 32 weights from the packed layout.
 // If row_dev is given, the first row is read from device memory (embedding
-// lookup of a token produced on the GPU) after the upstream kernel finishes.
+// lookup of a token produced on the GPU) after the upstream kernel finishes;
+// with `gather`, output row i is packed row row_dev[i] (one token per
+// sequence of a batch).
 __global__ void q4_dequant_kernel(const uint8_t* __restrict__ packed, int64_t n, int64_t k, int64_t kc,
                                   int64_t row0, const int32_t* __restrict__ row_dev, int64_t nrows,
-                                  void* __restrict__ out, int dtype, int64_t ldo)
+                                  void* __restrict__ out, int dtype, int64_t ldo, int gather)
 {
     pdl_wait();
     int64_t nb = k / 32;
     int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= nrows * nb) return;
     int64_t rr = gid / nb, b = gid % nb;
-    int64_t r0 = row_dev ? (int64_t)(*row_dev) : row0;
-    if (r0 < 0 || r0 + nrows > n) {                      // device-side lookup out of range
-        if (gid == 0) atomicCAS(&g_vox_device_status, 0, 0x0D0);
-        return;
+    int64_t r;
+    if (gather) {
+        r = (int64_t)row_dev[rr];
+        if (r < 0 || r >= n) {                           // device-side lookup out of range
+            if (b == 0) atomicCAS(&g_vox_device_status, 0, 0x0D0);
+            return;
+        }
+    } else {
+        const int64_t r0 = row_dev ? (int64_t)(*row_dev) : row0;
+        if (r0 < 0 || r0 + nrows > n) {                  // device-side lookup out of range
+            if (gid == 0) atomicCAS(&g_vox_device_status, 0, 0x0D0);
+            return;
+        }
+        r = r0 + rr;
     }
-    int64_t r = r0 + rr;
     int64_t tile = r >> 4;
     int i = (int)(r & 15), g = i & 7, rowsel = i >> 3;
     int64_t chunk = b >> 1;
@@ -146,14 +157,14 @@ vox_status launch_q4_pack(const uint8_t* gguf, int64_t n, int64_t k, int gate_up
 
 vox_status launch_q4_dequant(const uint8_t* packed, int64_t n, int64_t k, int64_t row0,
                              const int32_t* row_dev, int64_t nrows, void* out, int dtype, int64_t ldo,
-                             cudaStream_t s)
+                             cudaStream_t s, int gather)
 {
     int64_t kc = ceil_div(k, 64);
     int64_t total = nrows * (k / 32);
     int threads = 128;
     int64_t blocks = ceil_div(total, threads);
     return launch_pdl(q4_dequant_kernel, dim3((unsigned)blocks), dim3(threads), 0, s,
-                      packed, n, k, kc, row0, row_dev, nrows, out, dtype, ldo);
+                      packed, n, k, kc, row0, row_dev, nrows, out, dtype, ldo, gather && row_dev ? 1 : 0);
 }
 
 }  // namespace vox

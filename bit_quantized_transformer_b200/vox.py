@@ -25,7 +25,7 @@ VOX_OK, VOX_ERR_NULL, VOX_ERR_SHAPE, VOX_ERR_ALIGN, VOX_ERR_DTYPE = 0, 1, 2, 3, 
 VOX_ERR_RANGE, VOX_ERR_WORKSPACE, VOX_ERR_TIMEOUT, VOX_ERR_CUDA = 5, 6, 7, 8
 VOX_F32, VOX_BF16, VOX_F16 = 0, 1, 2
 VOX_PACK_PLAIN, VOX_PACK_GATE_UP = 0, 1
-VOX_EP_NONE, VOX_EP_RESIDUAL, VOX_EP_SILU_MUL, VOX_EP_GELU, VOX_EP_KV_APPEND, VOX_EP_ARGMAX = range(6)
+VOX_EP_NONE, VOX_EP_RESIDUAL, VOX_EP_SILU_MUL, VOX_EP_GELU, VOX_EP_KV_APPEND, VOX_EP_ARGMAX, VOX_EP_KV_APPEND_PAGED = range(7)
 
 _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
@@ -42,7 +42,7 @@ class vox_epilogue(ctypes.Structure):
     _fields_ = [("op", _I32), ("rmsnorm", _I32), ("eps", _F), ("norm_weight", _P),
                 ("residual", _P), ("ldr", _I64), ("k_cache", _P), ("v_cache", _P),
                 ("n_kv_heads", _I32), ("head_dim", _I32), ("window", _I32), ("q_rows", _I32),
-                ("pos", _I64), ("pos_dev", _P), ("argmax", _P)]
+                ("pos", _I64), ("pos_dev", _P), ("argmax", _P), ("page_table", _P), ("n_pages", _I64)]
 
 
 class vox_decoder(ctypes.Structure):
@@ -54,6 +54,10 @@ class vox_decoder(ctypes.Structure):
                 ("k_cache", ctypes.POINTER(_P)), ("v_cache", ctypes.POINTER(_P)),
                 ("token", _P), ("pos", _P), ("x", _P), ("h", _P), ("qkv", _P), ("attn", _P),
                 ("act", _P), ("logits", _P), ("workspace", _P), ("ws_bytes", _SZ)]
+
+
+class vox_decoder_batch(ctypes.Structure):
+    _fields_ = [("d", vox_decoder), ("n_seq", _I32), ("n_pages", _I64), ("page_table", _P)]
 
 
 class vox_encoder(ctypes.Structure):
@@ -85,12 +89,17 @@ _SIGS = {
     "vox_gqa_decode_attn": (_I32, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _F, _P, _SZ, _P]),
     "vox_gqa_decode_attn_workspace": (_SZ, [_I32, _I32, _I32, _I32]),
     "vox_gqa_decode_attn_static": (_I32, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _F, _P]),
+    "vox_gqa_decode_attn_paged": (_I32, [_P, _P, _P, _I64, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ,
+                                         _P]),
+    "vox_gqa_decode_attn_paged_workspace": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
     "vox_window_attn": (_I32, [_P, _I64, _P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _I32, _I64,
                                _I32, _I32, _I32, _F, _P]),
     "vox_rmsnorm": (_I32, [_P, _I64, _I64, _I64, _F, _P, _P, _I32, _I64, _P]),
     "vox_decoder_workspace": (_SZ, [ctypes.POINTER(vox_decoder)]),
     "vox_decoder_step": (_I32, [ctypes.POINTER(vox_decoder), _P]),
     "vox_decoder_step_kernels": (_I32, [ctypes.POINTER(vox_decoder), _P]),
+    "vox_decoder_batch_workspace": (_SZ, [ctypes.POINTER(vox_decoder_batch)]),
+    "vox_decoder_batch_step": (_I32, [ctypes.POINTER(vox_decoder_batch), _P]),
     "vox_encoder_chunk": (_I32, [ctypes.POINTER(vox_encoder), _P]),
     "vox_gguf_open": (_I32, [ctypes.c_char_p, ctypes.POINTER(_P)]),
     "vox_gguf_close": (None, [_P]),
@@ -201,6 +210,18 @@ def vox_gqa_decode_attn(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_di
            "vox_gqa_decode_attn")
 
 
+def vox_gqa_decode_attn_paged_workspace(n_seq, n_q_heads, n_kv_heads, head_dim, window) -> int:
+    return lib.vox_gqa_decode_attn_paged_workspace(n_seq, n_q_heads, n_kv_heads, head_dim, window)
+
+
+def vox_gqa_decode_attn_paged(q, k_pool, v_pool, n_pages, page_table, pos, n_seq, out, n_q_heads, n_kv_heads,
+                              head_dim, window, scale, workspace, ws_bytes, stream=None):
+    _check(lib.vox_gqa_decode_attn_paged(ptr(q), ptr(k_pool), ptr(v_pool), n_pages, ptr(page_table), ptr(pos), n_seq,
+                                         ptr(out), n_q_heads, n_kv_heads, head_dim, window, scale, ptr(workspace),
+                                         ws_bytes, stream_ptr(stream)),
+           "vox_gqa_decode_attn_paged")
+
+
 def vox_gqa_decode_attn_static(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_dim, window, pos, scale,
                                stream=None):
     _check(lib.vox_gqa_decode_attn_static(ptr(q), ptr(k_cache), ptr(v_cache), ptr(out), n_q_heads, n_kv_heads,
@@ -230,6 +251,14 @@ def vox_decoder_step(dec: vox_decoder, stream=None):
 
 def vox_decoder_step_kernels(dec: vox_decoder, stream=None):
     _check(lib.vox_decoder_step_kernels(ctypes.byref(dec), stream_ptr(stream)), "vox_decoder_step_kernels")
+
+
+def vox_decoder_batch_workspace(b: vox_decoder_batch) -> int:
+    return lib.vox_decoder_batch_workspace(ctypes.byref(b))
+
+
+def vox_decoder_batch_step(b: vox_decoder_batch, stream=None):
+    _check(lib.vox_decoder_batch_step(ctypes.byref(b), stream_ptr(stream)), "vox_decoder_batch_step")
 
 
 def vox_encoder_chunk(enc: vox_encoder, stream=None):

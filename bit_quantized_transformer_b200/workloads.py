@@ -41,6 +41,116 @@ def stack_rows(*parts):
     return (np.concatenate([p[0] for p in parts], axis=0), np.concatenate([p[1] for p in parts], axis=0))
 
 
+def decoder_weights(shape: synth.DecoderShape, L: int, seed: int, device):
+    """Packed weights of L decoder layers, the embedding and the LM head:
+    (tensors to keep alive, [wqkv], [wo], [w13], [w2], embedding, lm_head)."""
+    keep, wqkv, wo, w13, w2 = [], [], [], [], []
+    for l in range(L):
+        w = synth.decoder_layer_weights(shape, l, seed)
+        for lst, (qs, d), flags in ((wqkv, stack_rows(w["wq"], w["wk"], w["wv"]), V.VOX_PACK_PLAIN),
+                                    (wo, w["wo"], V.VOX_PACK_PLAIN),
+                                    (w13, stack_rows(w["w1"], w["w3"]), V.VOX_PACK_GATE_UP),
+                                    (w2, w["w2"], V.VOX_PACK_PLAIN)):
+            t, desc = pack_q4(qs, d, device, flags)
+            keep.append(t)
+            lst.append(desc)
+    emb_t, emb = pack_q4(*synth.q4_blocks(shape.vocab, shape.dim, seed, synth.EMB_ID), device)
+    lm_t, lm = pack_q4(*synth.q4_blocks(shape.vocab, shape.dim, seed, synth.LM_HEAD_ID), device)
+    keep += [emb_t, lm_t]
+    return keep, wqkv, wo, w13, w2, emb, lm
+
+
+class BatchDecoderModel:
+    """n_seq independent sequences over the synthetic decoder, each with its
+    own rolling cache in 64-slot pages of per-layer pools (synth.page_pool),
+    assigned by synth.page_table.  positions[s] slots of sequence s are taken
+    as present; the next step writes position positions[s]."""
+
+    def __init__(self, shape: synth.DecoderShape, n_seq: int, positions, tokens, seed: int = 0, device="cuda",
+                 n_layers=None, eps: float = 1e-5, window=None, spare_pages: int = 3, device_fill: bool = False):
+        self.shape, self.seed, self.device = shape, seed, device
+        self.L = shape.n_layers if n_layers is None else n_layers
+        self.W = shape.window if window is None else window
+        self.n_seq = n_seq
+        pps = self.W // synth.PAGE_SLOTS
+        self.n_pages = n_seq * pps + spare_pages
+        D, F, QD, KVD = shape.dim, shape.ffn, shape.q_dim, shape.kv_dim
+        keep, wqkv, wo, w13, w2, emb, lm = decoder_weights(shape, self.L, seed, device)
+        self.k_pool, self.v_pool = [], []
+        for l in range(self.L):
+            if device_fill:
+                # timing only: N(0,1) bf16 drawn on the device (seeded torch generator)
+                gen = torch.Generator(device=device)
+                shp = (self.n_pages, shape.n_kv_heads, synth.PAGE_SLOTS, shape.head_dim)
+                for pools, off in ((self.k_pool, 0), (self.v_pool, 1)):
+                    gen.manual_seed(seed * 1000 + 2 * l + off)
+                    pools.append(torch.randn(shp, generator=gen, device=device).to(torch.bfloat16))
+                continue
+            kb, vb = synth.page_pool(shape, l, self.n_pages, seed)
+            self.k_pool.append(bf16_dev(kb, device))
+            self.v_pool.append(bf16_dev(vb, device))
+        self.table_np = synth.page_table(n_seq, self.W, self.n_pages, seed)
+        self.page_table = to_dev(self.table_np, device)
+        self._keep = keep
+        self.wqkv, self.wo, self.w13, self.w2 = wqkv, wo, w13, w2
+        f32 = dict(dtype=torch.float32, device=device)
+        self.token = torch.tensor(list(tokens), dtype=torch.int32, device=device)
+        self.pos = torch.tensor(list(positions), dtype=torch.int64, device=device)
+        self.x = torch.zeros(n_seq, D, **f32)
+        self.h = torch.zeros(n_seq, D, **f32)
+        self.qkv = torch.zeros(n_seq, QD + 2 * KVD, **f32)
+        self.attn = torch.zeros(n_seq, QD, **f32)
+        self.act = torch.zeros(n_seq, F, **f32)
+        self.logits = torch.zeros(n_seq, shape.vocab, **f32)
+        Arr = V.vox_q4_weight * self.L
+        Ptr = ctypes.c_void_p * self.L
+        self._arrs = [Arr(*wqkv), Arr(*wo), Arr(*w13), Arr(*w2), Ptr(*[t.data_ptr() for t in self.k_pool]),
+                      Ptr(*[t.data_ptr() for t in self.v_pool])]
+        b = V.vox_decoder_batch()
+        d = b.d
+        d.n_layers, d.dim, d.n_q_heads, d.n_kv_heads = self.L, D, shape.n_q_heads, shape.n_kv_heads
+        d.head_dim, d.ffn, d.vocab, d.window, d.eps = shape.head_dim, F, shape.vocab, self.W, eps
+        d.wqkv, d.wo, d.w13, d.w2 = [ctypes.cast(a, ctypes.POINTER(V.vox_q4_weight)) for a in self._arrs[:4]]
+        d.embedding, d.lm_head = emb, lm
+        d.k_cache = ctypes.cast(self._arrs[4], ctypes.POINTER(ctypes.c_void_p))
+        d.v_cache = ctypes.cast(self._arrs[5], ctypes.POINTER(ctypes.c_void_p))
+        for name in ("token", "pos", "x", "h", "qkv", "attn", "act", "logits"):
+            setattr(d, name, getattr(self, name).data_ptr())
+        b.n_seq, b.n_pages, b.page_table = n_seq, self.n_pages, self.page_table.data_ptr()
+        ws = V.vox_decoder_batch_workspace(b)
+        self.workspace = torch.zeros(ws, dtype=torch.uint8, device=device)
+        d.workspace, d.ws_bytes = self.workspace.data_ptr(), ws
+        self.batch = b
+
+    def step(self, stream=None):
+        V.vox_decoder_batch_step(self.batch, stream)
+
+    def capture(self):
+        """CUDA graph of one batched step (one eager run on a side stream first)."""
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.step()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step()
+        return g
+
+    def weight_bytes(self) -> int:
+        tot = sum(w.n * w.k * 18 // 32 for w in self.wqkv + self.wo + self.w13 + self.w2)
+        return tot + self.shape.vocab * self.shape.dim * 18 // 32 + self.n_seq * self.shape.dim * 18 // 32
+
+    def kv_bytes(self, positions) -> int:
+        """bf16 K and V bytes the attention reads when sequence s has written positions[s]."""
+        per = sum(min(p + 1, self.W) for p in positions)
+        return self.L * 2 * self.shape.n_kv_heads * per * self.shape.head_dim * 2
+
+    def launches(self) -> int:
+        return 1 + self.L * 6 + 1 + 1
+
+
 class DecoderModel:
     """26-layer synthetic decoder (or fewer layers) with rolling caches.
 

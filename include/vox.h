@@ -135,8 +135,17 @@ enum {
                              n_kv_heads*head_dim): they are also written to y and,
                              rounded to bf16, into slot (pos + i) mod window of the
                              caches for token i ([ROLL])                               */
-    VOX_EP_ARGMAX = 5     /* y = W x, and argmax[i] = index of the largest y[i][:],
+    VOX_EP_ARGMAX = 5,    /* y = W x, and argmax[i] = index of the largest y[i][:],
                              lowest index on ties, a NaN wins over numbers             */
+    VOX_EP_KV_APPEND_PAGED = 6 /* as KV_APPEND, but input row i is sequence i of a batch
+                             with its own paged rolling cache: its k and v go, rounded
+                             to bf16, to slot p = pos_dev[i] mod window of that
+                             sequence, i.e. row p mod 64 of page
+                             page_table[i * (window / 64) + p / 64] of the pools
+                             k_cache / v_cache, bf16 [n_pages][n_kv_heads][64][head_dim]
+                             ([ROLL] per sequence, [BATCH]).  window a multiple of 64;
+                             pos_dev required.  A page index outside [0, n_pages) is
+                             not written and sets the device status word (0x105)   */
 };
 
 typedef struct {
@@ -152,6 +161,8 @@ typedef struct {
     int64_t pos;               /* KV_APPEND: position of input row 0                   */
     const int64_t *pos_dev;    /* if not NULL, the position is read from device memory  */
     int32_t *argmax;           /* ARGMAX: device int32 [m]                              */
+    const int32_t *page_table; /* KV_APPEND_PAGED: device int32 [m][window / 64]        */
+    int64_t n_pages;           /* KV_APPEND_PAGED: pages in each pool                   */
 } vox_epilogue;
 
 /* ----------------------------------------------------------- Q4_0 GEMV (M<=8)
@@ -265,6 +276,32 @@ vox_status vox_gqa_decode_attn_static(const float *q, const void *k_cache, const
                                       float *out, int32_t n_q_heads, int32_t n_kv_heads,
                                       int32_t head_dim, int32_t window, int64_t pos, float scale,
                                       void *stream);
+
+/* ------------------------------------------ batched decode attention (paged)
+ * vox_gqa_decode_attn_paged -- [ROLL] per sequence, [BATCH].  The attention of
+ * vox_gqa_decode_attn for n_seq independent sequences in one call, each with
+ * its own rolling cache held in pages of 64 slots.  Pools: k_pool, v_pool
+ * device bf16 [n_pages][n_kv_heads][64][head_dim], 16-byte aligned; sequence
+ * s's slot p (0 <= p < window) lives in row p mod 64 of page
+ * page_table[s * (window / 64) + p / 64] (page_table: device int32
+ * [n_seq][window / 64]); pos: device int64 [n_seq], the position each
+ * sequence has just written (valid slots: the first min(pos[s] + 1, window)).
+ * q: device fp32 [n_seq][n_q_heads][head_dim]; out: device fp32, same shape,
+ * 16-byte aligned.  The SMs are shared evenly by the sequences.  workspace:
+ * device, vox_gqa_decode_attn_paged_workspace() bytes, 16-byte aligned, no
+ * initial contents needed; calls sharing it must not overlap.  A page index
+ * outside [0, n_pages) reads zeros and sets the device status word (0x203).
+ * Errors: NULL -> VOX_ERR_NULL; n_seq outside 1..64, pos handling as
+ * vox_gqa_decode_attn, window not a positive multiple of 64, n_pages < 1 ->
+ * VOX_ERR_RANGE; head_dim != 128 or a pool beyond 2^31 rows -> VOX_ERR_SHAPE;
+ * misaligned pools, out or workspace -> VOX_ERR_ALIGN; short workspace ->
+ * VOX_ERR_WORKSPACE. */
+vox_status vox_gqa_decode_attn_paged(const float *q, const void *k_pool, const void *v_pool, int64_t n_pages,
+                                     const int32_t *page_table, const int64_t *pos, int32_t n_seq, float *out,
+                                     int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t window,
+                                     float scale, void *workspace, size_t ws_bytes, void *stream);
+size_t vox_gqa_decode_attn_paged_workspace(int32_t n_seq, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                           int32_t window);
 
 /* vox_window_attn -- [ARCH] encoder: causal sliding-window multi-head
  * attention for a chunk of n_q query rows.  Query row i sits at absolute
@@ -386,6 +423,40 @@ vox_status vox_decoder_step(const vox_decoder *dec, void *stream);
  * a short workspace -> VOX_ERR_WORKSPACE; a workspace, cache or activation
  * buffer that is not 16-byte aligned -> VOX_ERR_ALIGN. */
 vox_status vox_decoder_step_kernels(const vox_decoder *dec, void *stream);
+
+/* ------------------------------------------------ batched decoder step
+ * n_seq independent sequences stepped together ([BATCH]; [ROLL] per
+ * sequence): every projection reads its weights once for all sequences (the
+ * GEMV at m = n_seq rows), and each sequence keeps its own rolling cache in
+ * pages of 64 slots drawn from per-layer pools, so sequences of any
+ * positions share one weight stream.  `d` holds the shapes and weights as
+ * for one sequence, with these meanings:
+ *   d.k_cache[l], d.v_cache[l]: the layer's page pools, device bf16
+ *       [n_pages][n_kv_heads][64][head_dim], 16-byte aligned;
+ *   d.token: device int32 [n_seq], the input tokens, replaced by the greedy
+ *       next tokens; d.pos: device int64 [n_seq], each sequence's position,
+ *       advanced by one;
+ *   d.x, d.h, d.qkv, d.attn, d.act, d.logits: device fp32 [n_seq][...] of the
+ *       one-sequence sizes (rows back to back);
+ *   d.workspace: vox_decoder_batch_workspace() bytes, zero-filled once.
+ * page_table: device int32 [n_seq][window / 64] (see vox_gqa_decode_attn_paged);
+ * the caller assigns pages (a rolling window reuses its own pages in place). */
+typedef struct {
+    vox_decoder d;
+    int32_t n_seq;               /* 1..8 */
+    int64_t n_pages;             /* pages in each pool */
+    const int32_t *page_table;
+} vox_decoder_batch;
+
+size_t vox_decoder_batch_workspace(const vox_decoder_batch *b);
+
+/* One greedy step of every sequence: the launches of vox_decoder_step_kernels
+ * with m = n_seq rows (embedding rows gathered by token, the QKV epilogue
+ * VOX_EP_KV_APPEND_PAGED, vox_gqa_decode_attn_paged, argmax per row, every
+ * position advanced); the sequence can be captured in a CUDA graph.  Errors:
+ * as vox_decoder_step_kernels; n_seq outside 1..8, window not a multiple of
+ * 64 or n_pages < 1 -> VOX_ERR_RANGE; NULL page_table -> VOX_ERR_NULL. */
+vox_status vox_decoder_batch_step(const vox_decoder_batch *b, void *stream);
 
 typedef struct {
     int32_t n_layers, dim, n_heads, head_dim, ffn, window, rows, adapter_out;

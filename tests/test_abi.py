@@ -247,3 +247,47 @@ def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_paged_attention_validation(V):
+    """The batched paged attention rejects bad arguments on the host."""
+    L = V.lib
+    ws = V.vox_gqa_decode_attn_paged_workspace(4, 32, 8, 128, 8192)
+    assert ws >= 4 * V.vox_gqa_decode_attn_workspace(32, 8, 128, 8192) - 256
+    a = lambda nseq=4, nq=32, nkv=8, hd=128, W=8192, npg=600, pt=FAKE, wsp=FAKE, wsb=ws, kp=FAKE, out=FAKE: \
+        L.vox_gqa_decode_attn_paged(FAKE, kp, FAKE, npg, pt, FAKE, nseq, out, nq, nkv, hd, W, 0.088, wsp, wsb, None)
+    assert a(pt=None) == V.VOX_ERR_NULL
+    assert a(kp=None) == V.VOX_ERR_NULL
+    assert a(nseq=0) == V.VOX_ERR_RANGE
+    assert a(nseq=65) == V.VOX_ERR_RANGE
+    assert a(nq=30) == V.VOX_ERR_RANGE
+    assert a(W=100) == V.VOX_ERR_RANGE               # not a multiple of the 64-slot page
+    assert a(npg=0) == V.VOX_ERR_RANGE
+    assert a(hd=64) == V.VOX_ERR_SHAPE
+    assert a(npg=1 << 30) == V.VOX_ERR_SHAPE          # pool rows beyond 2^31
+    assert a(wsp=None) == V.VOX_ERR_WORKSPACE
+    assert a(wsb=ws - 16) == V.VOX_ERR_WORKSPACE
+    assert a(kp=FAKE + 2) == V.VOX_ERR_ALIGN
+    assert a(out=FAKE + 4) == V.VOX_ERR_ALIGN
+
+
+def test_paged_append_epilogue_validation(V):
+    L = V.lib
+    w = V.vox_q4_weight(FAKE, 64, 96)
+    ws = V.vox_q4_gemv_workspace(w, 2, None)
+
+    def g(**kw):
+        base = dict(op=V.VOX_EP_KV_APPEND_PAGED, k_cache=FAKE, v_cache=FAKE, n_kv_heads=1, head_dim=16,
+                    window=64, q_rows=0, pos_dev=FAKE, page_table=FAKE, n_pages=4)
+        base.update(kw)
+        ep = V.vox_epilogue(**base)
+        return L.vox_q4_gemv(ctypes.byref(w), FAKE, 2, 96, FAKE, 64, ctypes.byref(ep), FAKE, ws, None)
+
+    assert g(page_table=None) == V.VOX_ERR_NULL
+    assert g(pos_dev=None) == V.VOX_ERR_NULL
+    assert g(window=96) == V.VOX_ERR_RANGE
+    assert g(n_pages=0) == V.VOX_ERR_RANGE
+    assert g(head_dim=32, q_rows=8) == V.VOX_ERR_SHAPE      # 8 + 2 * 32 rows > 64
+    gm = lambda: L.vox_q4_gemm(ctypes.byref(V.vox_q4_weight(FAKE, 128, 128)), FAKE, V.VOX_BF16, 16, 128, FAKE,
+                               V.VOX_F32, 128, ctypes.byref(V.vox_epilogue(op=V.VOX_EP_KV_APPEND_PAGED)), None)
+    assert gm() == V.VOX_ERR_RANGE
