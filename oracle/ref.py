@@ -352,8 +352,27 @@ def attn_error(o, o_ref, probs, v_cache_valid_f64, group):
 
 
 # ------------------------------------------------------- composed references
-def decoder_layer(x, Wd, k_cache, v_cache, pos, n_q_heads, n_kv_heads, eps=RMS_EPS):
-    """One pre-norm decoder layer at M=1 (readings R4-R7).
+def rope(x, pos, theta, head_dim):
+    """Rotary position embedding of a vector of heads x [n_heads * head_dim]
+    at position ``pos`` (reading R17; the pages do not mention positional
+    encoding, so the decoder runs without it by default, reading R5): within
+    each head the pair (x[2i], x[2i+1]) is rotated by the angle
+    pos * theta^(-2i / head_dim), i = 0 .. head_dim/2 - 1.  theta <= 0: x unchanged."""
+    x = np.asarray(x, np.float64)
+    if theta <= 0:
+        return x.copy()
+    y = x.reshape(-1, head_dim).copy()
+    i = np.arange(head_dim // 2)
+    ang = pos * np.power(float(theta), -2.0 * i / head_dim)
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = y[:, 0::2].copy(), y[:, 1::2].copy()
+    y[:, 0::2] = a * c - b * s
+    y[:, 1::2] = a * s + b * c
+    return y.reshape(x.shape)
+
+
+def decoder_layer(x, Wd, k_cache, v_cache, pos, n_q_heads, n_kv_heads, eps=RMS_EPS, rope_theta=0.0):
+    """One pre-norm decoder layer at M=1 (readings R4-R7; optional RoPE R17).
 
     ``Wd`` maps names to dense float64 weight matrices (wq, wk, wv, wo, w1,
     w3, w2).  The caches are updated in place (bf16 storage of the new k, v,
@@ -362,10 +381,10 @@ def decoder_layer(x, Wd, k_cache, v_cache, pos, n_q_heads, n_kv_heads, eps=RMS_E
     """
     x = np.asarray(x, np.float64)
     n = rmsnorm(x, eps)
-    q = Wd["wq"] @ n
-    k = Wd["wk"] @ n
-    v = Wd["wv"] @ n
     hd = k_cache.shape[2]
+    q = rope(Wd["wq"] @ n, pos, rope_theta, hd)
+    k = rope(Wd["wk"] @ n, pos, rope_theta, hd)
+    v = Wd["wv"] @ n
     kv_append(k_cache, v_cache, k.reshape(n_kv_heads, hd), v.reshape(n_kv_heads, hd), pos)
     o = gqa_attn(q.reshape(n_q_heads, hd), k_cache, v_cache, pos).reshape(-1)
     h = x + Wd["wo"] @ o

@@ -823,3 +823,74 @@ def test_planted_mistakes_in_paging_are_caught():
             pin_paged(bad, ref.paged_append)
     with pytest.raises(AssertionError):
         pin_paged(ref.paged_to_cache, append_wrong_row)
+
+
+# ------------------------------------------------------------------- RoPE
+def pin_rope(rope):
+    """Closed forms of the rotary embedding (reading R17)."""
+    rng = np.random.default_rng(21)
+    # a single pair (head_dim 2) turns by exactly pos radians (i = 0: frequency 1)
+    for pos in (0, 1, 2, 7, 100):
+        y = rope(np.array([1.0, 0.0]), pos, 10000.0, 2)
+        assert np.allclose(y, [math.cos(pos), math.sin(pos)], rtol=0, atol=1e-12)
+        y = rope(np.array([0.0, 1.0]), pos, 10000.0, 2)
+        assert np.allclose(y, [-math.sin(pos), math.cos(pos)], rtol=0, atol=1e-12)
+    # the frequency of pair i is theta^(-2i/hd): with hd 4, pair 1 turns by pos / theta^(1/2)
+    y = rope(np.array([0.0, 0.0, 1.0, 0.0]), 3, 100.0, 4)
+    assert np.allclose(y, [0.0, 0.0, math.cos(0.3), math.sin(0.3)], rtol=0, atol=1e-12)
+    x = rng.standard_normal(3 * 8)
+    assert np.array_equal(rope(x, 0, 1e6, 8), x)                          # position 0: identity
+    assert np.array_equal(rope(x, 55, 0.0, 8), x)                         # off
+    y = rope(x, 123, 1e4, 8)
+    assert np.allclose(np.hypot(y[0::2], y[1::2]), np.hypot(x[0::2], x[1::2]), rtol=1e-12)   # pairs keep length
+    # relative position: <R(m) q, R(n) k> depends on m - n only
+    q, k = rng.standard_normal(16), rng.standard_normal(16)
+    for m, n in ((5, 2), (40, 37), (1003, 1000)):
+        assert abs(rope(q, m, 1e4, 16) @ rope(k, n, 1e4, 16) - rope(q, m - n, 1e4, 16) @ k) < 1e-9
+
+
+def test_rope_closed_forms():
+    pin_rope(ref.rope)
+
+
+def test_decoder_layer_rope_off_is_unchanged_and_rope_at_pos0_is_identity():
+    """rope_theta = 0 is the default layer; at position 0 RoPE changes nothing."""
+    rng = np.random.default_rng(22)
+    D, nq, nkv, hd, F, W = 8, 2, 1, 4, 6, 5
+    Wd = {k: rng.standard_normal(s) for k, s in (("wq", (nq * hd, D)), ("wk", (nkv * hd, D)),
+                                                  ("wv", (nkv * hd, D)), ("wo", (D, nq * hd)),
+                                                  ("w1", (F, D)), ("w3", (F, D)), ("w2", (D, F)))}
+    x = rng.standard_normal(D)
+    kc = np.zeros((nkv, W, hd), np.uint16)
+    for pos in (0, 3):
+        a = ref.decoder_layer(x, Wd, kc.copy(), kc.copy(), pos, nq, nkv)
+        b = ref.decoder_layer(x, Wd, kc.copy(), kc.copy(), pos, nq, nkv, rope_theta=0.0)
+        assert np.array_equal(a["out"], b["out"])
+        c = ref.decoder_layer(x, Wd, kc.copy(), kc.copy(), pos, nq, nkv, rope_theta=1e4)
+        if pos == 0:
+            assert np.array_equal(a["out"], c["out"])
+        else:
+            assert np.allclose(c["q"], ref.rope(Wd["wq"] @ a["n"], pos, 1e4, hd), rtol=0, atol=1e-12)
+            assert not np.allclose(a["q"], c["q"])
+
+
+def test_planted_mistakes_in_rope_are_caught():
+    def half_split(x, pos, theta, hd):               # rotates (x[i], x[i + hd/2]) instead of adjacent pairs
+        x = np.asarray(x, np.float64)
+        y = x.reshape(-1, hd).copy()
+        i = np.arange(hd // 2)
+        ang = pos * np.power(float(theta), -2.0 * i / hd)
+        a, b = y[:, :hd // 2].copy(), y[:, hd // 2:].copy()
+        y[:, :hd // 2] = a * np.cos(ang) - b * np.sin(ang)
+        y[:, hd // 2:] = a * np.sin(ang) + b * np.cos(ang)
+        return y.reshape(x.shape)
+
+    def wrong_sign(x, pos, theta, hd):
+        return ref.rope(x, -pos, theta, hd)
+
+    def wrong_frequency(x, pos, theta, hd):          # theta^(-i/hd)
+        return ref.rope(x, pos, math.sqrt(theta), hd) if theta > 0 else np.asarray(x, np.float64).copy()
+
+    for bad in (half_split, wrong_sign, wrong_frequency):
+        with pytest.raises(AssertionError):
+            pin_rope(bad)
