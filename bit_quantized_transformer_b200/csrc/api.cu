@@ -104,6 +104,11 @@ static vox_status check_epilogue(const vox_epilogue* ep, int64_t n, int64_t k, i
     if (op < VOX_EP_NONE || op > VOX_EP_KV_APPEND_PAGED) return VOX_ERR_RANGE;
     if (ep && ep->rmsnorm && !allow_rms) return VOX_ERR_RANGE;
     if (ep && ep->rmsnorm && !(ep->eps >= 0.f)) return VOX_ERR_RANGE;
+    if (ep && ep->rope_theta != 0.f) {
+        if (op != VOX_EP_KV_APPEND && op != VOX_EP_KV_APPEND_PAGED) return VOX_ERR_RANGE;
+        if (!(ep->rope_theta > 0.f) || ep->rope_theta > 3.0e38f) return VOX_ERR_RANGE;
+        if (ep->head_dim % 16 || ep->head_dim < 16 || ep->q_rows % ep->head_dim) return VOX_ERR_RANGE;
+    }
     int64_t ncols = op == VOX_EP_SILU_MUL ? n / 2 : n;
     if (ldy < ncols) return VOX_ERR_SHAPE;
     (void)k;

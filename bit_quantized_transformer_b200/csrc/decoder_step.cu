@@ -92,6 +92,7 @@ struct PsArgs {
     uint8_t* ws;
     int32_t n_layers, dim, q_dim, kv_dim, ffn, vocab, n_kv, group, window;
     float eps, qscale;
+    float rope;                      // rotary theta of q and k, 0 = off
     uint32_t act_bytes;                      // shared bytes of the activation / merge region
     int32_t test_withhold;                   // test hook: warp 0 of CTA 0 first waits on a barrier nothing completes
 };
@@ -458,12 +459,27 @@ struct PsBest {
     int32_t i;
 };
 
+// Rotary embedding of a q or k tile's rows g and g + 8 (base: the region's
+// first row); rows 2i and 2i + 1 of a head sit in lanes g and g ^ 1.  Whole
+// warp; not inlined, so that only steps with RoPE on pay for it.
+__device__ __noinline__ float2 ps_rope(float2 v, int64_t tile, int g, int64_t base, int64_t pos, float theta)
+{
+    const float p0 = __shfl_xor_sync(0xffffffffu, v.x, 4), p1 = __shfl_xor_sync(0xffffffffu, v.y, 4);
+    return make_float2(rope_rotate(v.x, p0, (tile * 16 + g - base) % kPsHd, kPsHd, pos, theta),
+                       rope_rotate(v.y, p1, (tile * 16 + g + 8 - base) % kPsHd, kPsHd, pos, theta));
+}
+
 // res0 / res1: the residual of rows g and g + 8 (WO, W2), loaded ahead.
 __device__ __forceinline__ void ps_epilogue(const PsArgs& P, const PsPhase& f, int64_t tile, float v0, float v1,
                                             float rr, int64_t pos, PsBest& best, float res0, float res1)
 {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const float val[2] = {v0 * rr, v1 * rr};
+    float val[2] = {v0 * rr, v1 * rr};
+    if (f.kind == PS_QKV && P.rope > 0.f && tile * 16 < P.q_dim + P.kv_dim) {
+        const float2 r = ps_rope(make_float2(val[0], val[1]), tile, g, tile * 16 < P.q_dim ? 0 : P.q_dim, pos, P.rope);
+        val[0] = r.x;
+        val[1] = r.y;
+    }
     if (f.kind == PS_LM) {
         float bv = -INFINITY;
         int32_t bi = 0x7fffffff;
@@ -1125,6 +1141,7 @@ vox_status launch_decoder_step(const vox_decoder* d, uint8_t* ws, cudaStream_t s
     a.window = d->window;
     a.eps = d->eps;
     a.qscale = (1.0f / sqrtf((float)kPsHd)) * 1.4426950408889634f;
+    a.rope = d->rope_theta;
     a.act_bytes = ps_act_bytes(d);
     const char* hook = getenv("VOX_TEST_WITHHOLD_STAGE");      // test of the bounded waits only
     a.test_withhold = hook && hook[0] == '1';

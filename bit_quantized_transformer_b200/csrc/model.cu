@@ -92,6 +92,7 @@ vox_status check_decoder(const vox_decoder* d, bool check_ws = true)
         d->n_q_heads / d->n_kv_heads > 8 || d->dim % 32 || d->ffn % 32 || d->ffn % 8)
         return VOX_ERR_SHAPE;
     if (d->window < 1) return VOX_ERR_RANGE;
+    if (!(d->rope_theta >= 0.f) || d->rope_theta > 3.0e38f) return VOX_ERR_RANGE;
     if (check_ws && d->ws_bytes < vox_decoder_workspace(d)) return VOX_ERR_WORKSPACE;
     if (!al16(d->workspace)) return VOX_ERR_ALIGN;
     const int64_t D = d->dim, QD = (int64_t)d->n_q_heads * d->head_dim, KVD = (int64_t)d->n_kv_heads * d->head_dim;
@@ -169,6 +170,7 @@ vox_status vox_decoder_step_kernels(const vox_decoder* d, void* stream)
         e.window = d->window;
         e.q_rows = (int32_t)QD;
         e.pos_dev = d->pos;
+        e.rope_theta = d->rope_theta;
         if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->wqkv[l].data), QD + 2 * KVD, D, d->x, 1, D, d->qkv,
                                  QD + 2 * KVD, &e, ws_g, s)))
             return st;
@@ -255,6 +257,7 @@ vox_status vox_decoder_batch_step(const vox_decoder_batch* b, void* stream)
         e.window = d->window;
         e.q_rows = (int32_t)QD;
         e.pos_dev = d->pos;
+        e.rope_theta = d->rope_theta;
         e.page_table = b->page_table;
         e.n_pages = b->n_pages;
         if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->wqkv[l].data), QD + 2 * KVD, D, d->x, m, D, d->qkv,

@@ -92,6 +92,7 @@ struct GemvArgs {
     int32_t evict_first;                     // 1: weight copies marked evict-first in L2
     const int32_t* pages;                    // KV_APPEND_PAGED: page table [m][window / 64]
     int64_t n_pages;
+    float rope;                              // KV_APPEND(_PAGED): rotary theta, 0 = off
 };
 
 // Shared-memory carve-up, computed identically on host and device.
@@ -167,6 +168,23 @@ __device__ __noinline__ GemvBest gemv_epilogue(const GemvArgs& a, int64_t tile, 
     for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int e = 0; e < 2; ++e) v[2 * h + e] = acc[2 * h + e] * rr[e];
+    if (a.rope > 0.f && tile * 16 < (int64_t)a.q_rows + (int64_t)a.n_kv * a.hd) {
+        // q or k rows (a 16-row tile lies in one region): rows 2i and 2i + 1
+        // of a head sit in lanes g and g ^ 1, four lanes apart
+        const int64_t base = tile * 16 < a.q_rows ? 0 : a.q_rows;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float partner = __shfl_xor_sync(0xffffffffu, v[2 * h + e], 4);
+                const int mt = 2 * t + e;
+                if (mt < a.m) {
+                    const int64_t col = (tile * 16 + g + 8 * h - base) % a.hd;
+                    const int64_t p = a.op == VOX_EP_KV_APPEND_PAGED ? a.pos_dev[mt] : pos + mt;
+                    v[2 * h + e] = rope_rotate(v[2 * h + e], partner, col, a.hd, p, a.rope);
+                }
+            }
+    }
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const int mt = 2 * t + e;
@@ -570,6 +588,7 @@ vox_status launch_q4_gemv(const uint8_t* w, int64_t n, int64_t k, const float* x
     a.res = ep ? ep->residual : nullptr;
     a.ldr = ep ? ep->ldr : 0;
     if (ep && (ep->op == VOX_EP_KV_APPEND || ep->op == VOX_EP_KV_APPEND_PAGED)) {
+        a.rope = ep->rope_theta;
         a.pages = ep->page_table;
         a.n_pages = ep->n_pages;
         a.kcache = static_cast<uint16_t*>(ep->k_cache);

@@ -115,4 +115,27 @@ __device__ __forceinline__ void gemv_record(uint4 q, uint2 dd, uint32_t bs, uint
     }
 }
 
+// Rotary embedding: (cos, sin) of the angle pos * theta^(-2i/hd) of pair
+// i = col / 2.  The angle is reduced to turns in double precision, so long
+// positions keep it accurate; the sine and cosine of the reduced angle are
+// taken in single precision.  Not inlined: only the q and k tiles of a
+// projection with RoPE on reach it.
+static __device__ __noinline__ float2 rope_cs(int64_t col, int hd, int64_t pos, float theta)
+{
+    const double inv = exp2(-(2.0 * (double)(col >> 1) / hd) * log2((double)theta));
+    double turns = (double)pos * inv * 0.15915494309189535;     // 1 / (2 pi)
+    turns -= floor(turns);
+    float s, c;
+    sincospif(2.0f * (float)turns, &s, &c);
+    return make_float2(c, s);
+}
+
+// One element of an adjacent pair after the rotation (col even: the pair's
+// first element, col odd: its second); v is this element, partner the other.
+__device__ __forceinline__ float rope_rotate(float v, float partner, int64_t col, int hd, int64_t pos, float theta)
+{
+    const float2 cs = rope_cs(col, hd, pos, theta);
+    return (col & 1) ? fmaf(partner, cs.y, v * cs.x) : fmaf(-partner, cs.y, v * cs.x);
+}
+
 }  // namespace vox

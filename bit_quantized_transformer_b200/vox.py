@@ -42,7 +42,8 @@ class vox_epilogue(ctypes.Structure):
     _fields_ = [("op", _I32), ("rmsnorm", _I32), ("eps", _F), ("norm_weight", _P),
                 ("residual", _P), ("ldr", _I64), ("k_cache", _P), ("v_cache", _P),
                 ("n_kv_heads", _I32), ("head_dim", _I32), ("window", _I32), ("q_rows", _I32),
-                ("pos", _I64), ("pos_dev", _P), ("argmax", _P), ("page_table", _P), ("n_pages", _I64)]
+                ("pos", _I64), ("pos_dev", _P), ("argmax", _P), ("page_table", _P), ("n_pages", _I64),
+                ("rope_theta", _F)]
 
 
 class vox_decoder(ctypes.Structure):
@@ -53,7 +54,7 @@ class vox_decoder(ctypes.Structure):
                 ("embedding", vox_q4_weight), ("lm_head", vox_q4_weight),
                 ("k_cache", ctypes.POINTER(_P)), ("v_cache", ctypes.POINTER(_P)),
                 ("token", _P), ("pos", _P), ("x", _P), ("h", _P), ("qkv", _P), ("attn", _P),
-                ("act", _P), ("logits", _P), ("workspace", _P), ("ws_bytes", _SZ)]
+                ("act", _P), ("logits", _P), ("workspace", _P), ("ws_bytes", _SZ), ("rope_theta", _F)]
 
 
 class vox_decoder_batch(ctypes.Structure):

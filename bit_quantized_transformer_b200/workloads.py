@@ -67,7 +67,8 @@ class BatchDecoderModel:
     as present; the next step writes position positions[s]."""
 
     def __init__(self, shape: synth.DecoderShape, n_seq: int, positions, tokens, seed: int = 0, device="cuda",
-                 n_layers=None, eps: float = 1e-5, window=None, spare_pages: int = 3, device_fill: bool = False):
+                 n_layers=None, eps: float = 1e-5, window=None, spare_pages: int = 3, device_fill: bool = False,
+                 rope_theta: float = 0.0):
         self.shape, self.seed, self.device = shape, seed, device
         self.L = shape.n_layers if n_layers is None else n_layers
         self.W = shape.window if window is None else window
@@ -116,6 +117,7 @@ class BatchDecoderModel:
         d.v_cache = ctypes.cast(self._arrs[5], ctypes.POINTER(ctypes.c_void_p))
         for name in ("token", "pos", "x", "h", "qkv", "attn", "act", "logits"):
             setattr(d, name, getattr(self, name).data_ptr())
+        d.rope_theta = rope_theta
         b.n_seq, b.n_pages, b.page_table = n_seq, self.n_pages, self.page_table.data_ptr()
         ws = V.vox_decoder_batch_workspace(b)
         self.workspace = torch.zeros(ws, dtype=torch.uint8, device=device)
@@ -160,7 +162,7 @@ class DecoderModel:
     """
 
     def __init__(self, shape: synth.DecoderShape, seed: int = 0, device="cuda", n_layers=None,
-                 filled: int = 0, token: int = 0, eps: float = 1e-5, window=None):
+                 filled: int = 0, token: int = 0, eps: float = 1e-5, window=None, rope_theta: float = 0.0):
         self.shape = shape
         self.seed = seed
         self.device = device
@@ -208,6 +210,7 @@ class DecoderModel:
         dec = V.vox_decoder()
         dec.n_layers, dec.dim, dec.n_q_heads, dec.n_kv_heads = self.L, D, shape.n_q_heads, shape.n_kv_heads
         dec.head_dim, dec.ffn, dec.vocab, dec.window, dec.eps = shape.head_dim, F, shape.vocab, self.W, eps
+        dec.rope_theta = rope_theta
         dec.wqkv, dec.wo, dec.w13, dec.w2 = [ctypes.cast(a, ctypes.POINTER(V.vox_q4_weight)) for a in self._arrs[:4]]
         dec.embedding, dec.lm_head = emb, lm
         dec.k_cache = ctypes.cast(self._arrs[4], ctypes.POINTER(ctypes.c_void_p))

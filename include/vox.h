@@ -163,6 +163,12 @@ typedef struct {
     int32_t *argmax;           /* ARGMAX: device int32 [m]                              */
     const int32_t *page_table; /* KV_APPEND_PAGED: device int32 [m][window / 64]        */
     int64_t n_pages;           /* KV_APPEND_PAGED: pages in each pool                   */
+    float rope_theta;          /* KV_APPEND(_PAGED): 0 = off (the pages name no positional
+                                  encoding); > 0: rotary embedding of the q and k rows
+                                  before they are stored: in each head, the pair
+                                  (y[2i], y[2i+1]) turns by pos * theta^(-2i/head_dim),
+                                  pos the token's position.  Needs head_dim % 16 == 0
+                                  and q_rows % head_dim == 0                            */
 } vox_epilogue;
 
 /* ----------------------------------------------------------- Q4_0 GEMV (M<=8)
@@ -383,6 +389,8 @@ typedef struct {
                                     q+2kv, q_dim, ffn, vocab floats                     */
     void *workspace;             /* device, vox_decoder_workspace() bytes, zero-filled once  */
     size_t ws_bytes;
+    float rope_theta;            /* 0: no positional encoding (default); > 0: rotary
+                                    embedding of q and k, see vox_epilogue.rope_theta   */
 } vox_decoder;
 
 /* Bytes of decoder workspace (device, 16-byte aligned) that both forms of

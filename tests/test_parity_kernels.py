@@ -526,3 +526,41 @@ def test_rmsnorm(env):
     V.vox_rmsnorm(WL.to_dev(x, "cuda"), 5, 1280, 1280, 1e-5, None, out, V.VOX_F32, 1280)
     check_status(V)
     np.testing.assert_allclose(np_of(out), ref.rmsnorm(x), rtol=1e-5, atol=1e-6)
+
+
+# ------------------------------------------------------------------- RoPE
+@pytest.mark.parametrize("pos,theta", [(0, 1e6), (7, 1e4), (8191, 1e6), (100000, 1e6), (123457, 500.0)])
+def test_gemv_kv_append_rope(env, pos, theta):
+    """The QKV epilogue with the rotary embedding: the GPU's q and k rows,
+    turned back by the oracle's inverse rotation, match the plain product;
+    the cache holds bf16 of the rotated k rows (two tokens, positions pos
+    and pos + 1)."""
+    torch, V, WL = env
+    n_q, n_kv, hd, W, k, m = 4, 2, 128, 256, 384, 2
+    QD, KVD = n_q * hd, n_kv * hd
+    n = QD + 2 * KVD
+    qs, d = synth.q4_blocks(n, k, 0, 8200)
+    packed, w = WL.pack_q4(qs, d, "cuda")
+    x = synth.activations(m, k, 0, 8201)
+    kc = torch.zeros(n_kv, W, hd, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    y = torch.full((m, n), float("nan"), device="cuda")
+    e = V.vox_epilogue(op=V.VOX_EP_KV_APPEND, k_cache=kc.data_ptr(), v_cache=vc.data_ptr(), n_kv_heads=n_kv,
+                       head_dim=hd, window=W, q_rows=QD, pos=pos, rope_theta=theta)
+    wsb = V.vox_q4_gemv_workspace(w, m, e)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    V.vox_q4_gemv(w, WL.to_dev(x, "cuda"), m, k, y, n, e, ws, wsb)
+    check_status(V)
+    yv = np_of(y).astype(np.float64)
+    Wm = ref.q4_weights(qs, d)
+    y_ref = x.astype(np.float64) @ Wm.T
+    back = yv.copy()
+    for i in range(m):
+        back[i, :QD] = ref.rope(yv[i, :QD], -(pos + i), theta, hd)
+        back[i, QD:QD + KVD] = ref.rope(yv[i, QD:QD + KVD], -(pos + i), theta, hd)
+    assert ref.gemv_error(back, y_ref, x, Wm) <= TOL
+    if pos > 0:                                        # the rotation did happen
+        assert ref.gemv_error(yv, y_ref, x, Wm) > 10 * TOL
+    kb = bf16_bits(kc)
+    for i in range(m):
+        assert np.array_equal(kb[:, (pos + i) % W], ref.f32_to_bf16(np_of(y)[i, QD:QD + KVD]).reshape(n_kv, hd))

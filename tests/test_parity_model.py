@@ -374,3 +374,31 @@ def test_encoder_chunk_last_layer(env):
     x_out = check_encoder_layer(shape, em, shape.n_layers - 1, 0)
     assert np.all(np.isfinite(x_out))
     check_adapter(shape, em, x_out, 0)
+
+
+@pytest.mark.parametrize("form", FORMS)
+def test_decoder_layer_rope(env, form):
+    """One layer with the rotary embedding on (theta 1e6) at position 1024,
+    both forms: q and k turned back by the oracle's inverse rotation match
+    the plain QKV product, the cache holds the rotated k, and the rest of the
+    layer is checked on the GPU's own inputs."""
+    torch, V, WL = env
+    shape = synth.DecoderShape()
+    tok, theta, filled = 4242, 1e6, 1024
+    dm = WL.DecoderModel(shape, seed=0, n_layers=1, filled=filled, token=tok, rope_theta=theta)
+    run_step(dm, form)
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    D, QD, KVD, hd = shape.dim, shape.q_dim, shape.kv_dim, shape.head_dim
+    eq, ed = synth.q4_blocks(shape.vocab, D, 0, synth.EMB_ID)
+    x0 = ref.c_dequant_f32(eq, ed, row0=tok, nrows=1)[0]
+    w = synth.decoder_layer_weights(shape, 0, 0)
+    qs = np.concatenate([w["wq"][0], w["wk"][0], w["wv"][0]])
+    ds = np.concatenate([w["wq"][1], w["wk"][1], w["wv"][1]])
+    qkv = np_of(dm.qkv).astype(np.float64)
+    back = qkv.copy()
+    back[:QD] = ref.rope(qkv[:QD], -filled, theta, hd)
+    back[QD:QD + KVD] = ref.rope(qkv[QD:QD + KVD], -filled, theta, hd)
+    err = gemv_err(back[None], ref.rmsnorm(x0)[None], qs, ds)
+    assert err <= TOL, err
+    check_layer_tail(shape, 0, dm, 0, filled)
