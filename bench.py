@@ -64,9 +64,11 @@ def parse_args(argv=None):
                         "case (--kernel, --shape, --launches), sized for an ncu capture; batch: --seqs "
                         "sequences stepped together over paged caches (26 layers, KV 8192 wrapped)")
     p.add_argument("--seqs", type=int, default=8, help="batch workload: sequences (1..8)")
-    p.add_argument("--kernel", choices=["gemv", "attn", "gemm", "step"], default="gemv",
+    p.add_argument("--kernel", choices=["gemv", "attn", "gemm", "step", "stepk", "encoder"], default="gemv",
                    help="kernel workload: gemv N K (M = 1), attn POS (decoder-shaped layer), gemm N K M, "
-                        "step L (the persistent decoder step with L full-size layers, KV 8192 wrapped)")
+                        "step L (the persistent decoder step with L full-size layers, KV 8192 wrapped), "
+                        "stepk L (the same step as the kernel sequence, eager), encoder L (the encoder chunk "
+                        "with L layers and the adapter, eager)")
     p.add_argument("--shape", type=int, nargs="*", default=None)
     p.add_argument("--launches", type=int, default=4)
     return p.parse_args(argv)
@@ -951,8 +953,24 @@ def run_kernel_case(args):
     from bit_quantized_transformer_b200 import vox as V
     from bit_quantized_transformer_b200 import workloads as WL
 
-    shp = args.shape or {"gemv": [4096, 3072], "attn": [8492], "gemm": [131072, 3072, 256], "step": [2]}[args.kernel]
-    if args.kernel == "step":
+    shp = args.shape or {"gemv": [4096, 3072], "attn": [8492], "gemm": [131072, 3072, 256], "step": [2],
+                         "stepk": [26], "encoder": [32]}[args.kernel]
+    if args.kernel == "stepk":
+        shape = synth.DecoderShape(n_layers=shp[0])
+        dm = WL.DecoderModel(shape, seed=0, filled=FILLED, token=17)
+        for _ in range(args.launches):
+            dm.step_kernels()
+        what = {"kernel": "decoder step kernel sequence", "layers": shp[0],
+                "launches_per_step": dm.step_kernels_launches(),
+                "bytes_per_step": dm.weight_bytes() + dm.kv_bytes(FILLED)}
+    elif args.kernel == "encoder":
+        shape = synth.EncoderShape(n_layers=shp[0])
+        em = WL.EncoderModel(shape, seed=0)
+        for _ in range(args.launches):
+            em.reset()
+            em.run()
+        what = {"kernel": "encoder chunk", "layers": shp[0], "gemm_flop_per_chunk": em.gemm_flops()}
+    elif args.kernel == "step":
         shape = synth.DecoderShape(n_layers=shp[0])
         dm = WL.DecoderModel(shape, seed=0, filled=FILLED, token=17)
         for _ in range(args.launches):
