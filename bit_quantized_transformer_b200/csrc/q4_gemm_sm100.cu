@@ -49,6 +49,7 @@ struct GemmArgs {
     int32_t op;
     const float* res;
     int64_t ldr;
+    int32_t splits;                  // K splits = CTAs of a cluster along z (1: no split)
 };
 
 template <int BN>
@@ -111,11 +112,47 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b)
 
 __device__ __forceinline__ float gelu_erf_g(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
 
-template <int BN>
+// The epilogue of one output element: residual add or GELU, fp32 or bf16 store.
+__device__ __forceinline__ void gemm_store(const GemmArgs& a, int64_t mi, int64_t row, float o)
+{
+    if (a.op == VOX_EP_RESIDUAL) o += a.res[mi * a.ldr + row];
+    else if (a.op == VOX_EP_GELU) o = gelu_erf_g(o);
+    if (a.y_bf16)
+        static_cast<uint16_t*>(a.y)[mi * a.ldy + row] = f32_to_bf16_bits(o);
+    else
+        static_cast<float*>(a.y)[mi * a.ldy + row] = o;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// Distributed-shared-memory load; issued without a memory clobber so that
+// several can be in flight before their values are summed.
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+// SPLIT: K split over the CTAs of a cluster along z (a.splits > 1); the
+// instance without it carries none of the reduction code.
+template <int BN, bool SPLIT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap, const GemmArgs a)
 {
     using C = GemmCfg<BN>;
+    static_assert(BN * kGemmRows * 4 <= C::bars, "the split-K partial tile must fit the ring");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::bars);
@@ -128,7 +165,10 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t group = blockIdx.x;              // 8 row tiles = 128 weight rows
     const int64_t m0 = (int64_t)blockIdx.y * BN;
-    const int kc = a.kc;
+    // this CTA's K chunks [kb0, kb0 + nk): split blockIdx.z of a.splits
+    const int S = SPLIT ? a.splits : 1;
+    const int kb0 = SPLIT ? (int)((int64_t)blockIdx.z * a.kc / S) : 0;
+    const int nk = SPLIT ? (int)((int64_t)(blockIdx.z + 1) * a.kc / S) - kb0 : a.kc;
 
     if (tid == 0) {
         for (int s = 0; s < C::stages; ++s) {
@@ -158,9 +198,10 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
             prefetch_tmap(&xmap);
             prefetch_tmap(&wmap);
             const uint32_t bytes = (uint32_t)kGemmRawBytes + C::xbytes;   // rows past the matrix read as zeros
-            for (int kb = 0; kb < kc; ++kb) {
-                const int s = kb % C::stages;
-                const uint32_t ph = (uint32_t)((kb / C::stages) & 1);
+            for (int i = 0; i < nk; ++i) {
+                const int kb = kb0 + i;
+                const int s = i % C::stages;
+                const uint32_t ph = (uint32_t)((i / C::stages) & 1);
                 if (!s_fail[0] && !mbar_wait_bounded(&empty[s], ph ^ 1u, 0x301)) s_fail[0] = 1;
                 if (s_fail[0]) break;
                 uint8_t* st = smem + s * C::stage;
@@ -174,9 +215,9 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         if (lane == 0) {
             const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                    ((uint32_t)(kGemmRows >> 4) << 24);
-            for (int kb = 0; kb < kc; ++kb) {
-                const int s = kb % C::stages;
-                const uint32_t ph = (uint32_t)((kb / C::stages) & 1);
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % C::stages;
+                const uint32_t ph = (uint32_t)((i / C::stages) & 1);
                 if (!s_fail[0] && !mbar_wait_bounded(&aready[s], ph, 0x302)) s_fail[0] = 1;
                 if (s_fail[0]) break;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -185,7 +226,7 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16(tmem, umma_desc_sw128(as + kk * 32), umma_desc_sw128(xs + kk * 32), idesc,
-                              (kb > 0 || kk > 0) ? 1u : 0u);
+                              (i > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&empty[s]);
             }
             umma_commit(&accb[0]);
@@ -198,9 +239,9 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         const int g = lane >> 2, t = lane & 3;
         const uint32_t M_L = 0x000F000Fu, C_B = 0x43004300u, B136 = 0x43084308u;   // 128.0, 136.0 (bf16x2)
         const uint32_t row_g = (uint32_t)(dw * 16 + g), row_g8 = row_g + 8u;
-        for (int kb = 0; kb < kc; ++kb) {
-            const int s = kb % C::stages;
-            const uint32_t ph = (uint32_t)((kb / C::stages) & 1);
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % C::stages;
+            const uint32_t ph = (uint32_t)((i / C::stages) & 1);
             if (!s_fail[0] && !mbar_wait_bounded(&full[s], ph, 0x303)) s_fail[0] = 1;
             uint8_t* st = smem + s * C::stage;
             uint8_t* A = st + C::xbytes;
@@ -243,27 +284,66 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const int64_t row = group * kGemmRows + r;
         const int c0 = (dw >> 2) * (BN / 2);
+        // split K: the partial tile goes to the idle ring as [token][row] fp32
+        float* part = reinterpret_cast<float*>(smem);
         for (int cc = 0; cc < BN / 2; cc += 8) {
             float v[8];
             tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c0 + cc), v);
-            if (row < a.n) {
+            if constexpr (SPLIT) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) part[(c0 + cc + j) * kGemmRows + r] = v[j];
+            } else if (row < a.n) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int64_t mi = m0 + c0 + cc + j;
                     if (mi >= a.m) break;
-                    float o = v[j];
-                    if (a.op == VOX_EP_RESIDUAL) o += a.res[mi * a.ldr + row];
-                    else if (a.op == VOX_EP_GELU) o = gelu_erf_g(o);
-                    if (a.y_bf16)
-                        static_cast<uint16_t*>(a.y)[mi * a.ldy + row] = f32_to_bf16_bits(o);
-                    else
-                        static_cast<float*>(a.y)[mi * a.ldy + row] = o;
+                    gemm_store(a, mi, row, v[j]);
                 }
             }
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
+    if constexpr (SPLIT) {
+        // Every CTA of the cluster holds its partial tile; CTA `rank` sums
+        // tokens [rank BN / S, (rank + 1) BN / S) over the ranks in order
+        // 0 .. S-1 (deterministic) through distributed shared memory and
+        // runs the epilogue on them.  Every thread of every CTA reaches both
+        // cluster barriers, also after a wait that gave up.
+        cluster_sync_all();
+        uint32_t rank;
+        asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+        const uint32_t pl = smem_addr(smem);
+        uint32_t rb[8];
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2) rb[s2] = cluster_map(pl, (uint32_t)(s2 < S ? s2 : 0));
+        const int cb = (int)(rank * BN / S), ce = (int)((rank + 1) * BN / S);
+        const int nel = (ce - cb) * kGemmRows;
+        // four elements per thread per round, all their loads in flight before the sums
+        for (int e0 = tid; e0 < nel; e0 += 4 * kGemmThreads) {
+            float v[4][8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * kGemmThreads;
+                const uint32_t off = e < nel ? (uint32_t)((cb + e / kGemmRows) * kGemmRows + e % kGemmRows) * 4u : 0u;
+#pragma unroll
+                for (int s2 = 0; s2 < 8; ++s2) v[u][s2] = (s2 < S && e < nel) ? ld_cluster_f32(rb[s2] + off) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * kGemmThreads;
+                if (e >= nel) break;
+                float o = v[u][0];
+#pragma unroll
+                for (int s2 = 1; s2 < 8; ++s2)
+                    if (s2 < S) o += v[u][s2];
+                const int c = cb + e / kGemmRows, rr = e % kGemmRows;
+                const int64_t row = group * kGemmRows + rr, mi = m0 + c;
+                if (row < a.n && mi < a.m) gemm_store(a, mi, row, o);
+            }
+        }
+        cluster_sync_all();
+    }
     if (warp == 1) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::tmem_cols)
@@ -284,35 +364,107 @@ static vox_status launch_gemm_bn(const GemmArgs& a, const void* x, int64_t ldx, 
     st = make_tmap_2d(&wmap, a.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)a.kc * (kChunkBytes / 4),
                       (uint64_t)a.tiles, (uint64_t)a.kc * kChunkBytes, kChunkBytes / 4, 8, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != VOX_OK) return st;
-    static std::atomic<unsigned long long> attr_done{0};
-    st = smem_attr_per_device(reinterpret_cast<const void*>(q4_gemm_kernel<BN>), C::smem, attr_done);
+    static std::atomic<unsigned long long> attr_done{0}, attr_done_split{0};
+    dim3 grid((unsigned)ceil_div(a.tiles, 8), (unsigned)ceil_div(a.m, BN), (unsigned)a.splits);
+    if (a.splits > 1) {
+        st = smem_attr_per_device(reinterpret_cast<const void*>(q4_gemm_kernel<BN, true>), C::smem, attr_done_split);
+        if (st != VOX_OK) return st;
+        return launch_pdl_cluster(q4_gemm_kernel<BN, true>, grid, dim3(kGemmThreads), (size_t)C::smem, s,
+                                  (unsigned)a.splits, xmap, wmap, a);
+    }
+    st = smem_attr_per_device(reinterpret_cast<const void*>(q4_gemm_kernel<BN, false>), C::smem, attr_done);
     if (st != VOX_OK) return st;
-    dim3 grid((unsigned)ceil_div(a.tiles, 8), (unsigned)ceil_div(a.m, BN));
-    return launch_pdl(q4_gemm_kernel<BN>, grid, dim3(kGemmThreads), (size_t)C::smem, s, xmap, wmap, a);
+    return launch_pdl(q4_gemm_kernel<BN, false>, grid, dim3(kGemmThreads), (size_t)C::smem, s, xmap, wmap, a);
 }
 
-static int pick_bn(int64_t tiles, int64_t m)
+// Clusters of `splits` CTAs of q4_gemm_kernel<BN> that the device runs at
+// once (the occupancy query accounts for how the SMs fall into GPCs), cached
+// per device; 0 if the query fails.
+template <int BN>
+static int gemm_max_clusters(int splits)
 {
-    const char* e = getenv("VOX_GEMM_BN");
-    if (e) {
-        int v = atoi(e);
-        if (v == 32 || v == 64 || v == 128 || v == 256) return v;
+    static std::atomic<int> cache[64][9];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || splits < 1 || splits > 8) return 0;
+    int v = cache[dev][splits].load(std::memory_order_relaxed);
+    if (v) return v - 1;
+    using C = GemmCfg<BN>;
+    static std::atomic<unsigned long long> attr_done{0};
+    if (smem_attr_per_device(reinterpret_cast<const void*>(q4_gemm_kernel<BN, true>), C::smem, attr_done) != VOX_OK)
+        return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, (unsigned)splits);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = C::smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = (unsigned)splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, q4_gemm_kernel<BN, true>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
     }
+    cache[dev][splits].store(n + 1, std::memory_order_relaxed);
+    return n;
+}
+
+static int max_clusters(int bn, int splits)
+{
+    switch (bn) {
+    case 32: return gemm_max_clusters<32>(splits);
+    case 64: return gemm_max_clusters<64>(splits);
+    case 128: return gemm_max_clusters<128>(splits);
+    default: return gemm_max_clusters<256>(splits);
+    }
+}
+
+// Tile width BN and K splits by a cost model in microseconds fitted to B200
+// measurements of this kernel: a K chunk takes about 0.54, 0.6, 0.6 and
+// 0.9 us per CTA for BN 32, 64, 128 and 256; a CTA has about 6 us of fixed
+// cost (12 at BN 256, whose epilogue is four times larger), and a split adds
+// about 2 us of cluster reduction.  Cost = waves x (chunks per split x chunk
+// time + fixed + reduction).  Splits (at most 8, one portable cluster, and
+// at least 2 chunks each) are only taken when all clusters run at once.
+// VOX_GEMM_BN and VOX_GEMM_SPLITS override the choice.
+static void pick_tile(int64_t tiles, int64_t m, int kc, int& bn_out, int& splits_out)
+{
     const int64_t groups = ceil_div(tiles, 8);
     const int64_t sms = device_sm_count();
-    int best = 256;
-    int64_t best_cost = INT64_MAX;
+    const char* ebn = getenv("VOX_GEMM_BN");
+    const char* esp = getenv("VOX_GEMM_SPLITS");
+    const int fbn = ebn ? atoi(ebn) : 0, fsp = esp ? atoi(esp) : 0;
+    double best_cost = 1e300;
+    int best_bn = 256, best_s = 1;
     for (int bn = 256; bn >= 32; bn >>= 1) {
-        if (bn > 32 && (bn >> 1) >= m) continue;            // a smaller tile already covers every row
-        const int64_t ctas = groups * ceil_div(m, bn);
-        const int64_t waves = ceil_div(ctas, sms);
-        const int64_t cost = waves * (bn > 64 ? bn : 64);    // per-stage time ~ max(MMA, dequant)
-        if (cost < best_cost) {
-            best_cost = cost;
-            best = bn;
+        if (fbn && bn != fbn) continue;
+        if (!fbn && bn > 32 && (bn >> 1) >= m) continue;    // a smaller tile already covers every row
+        const double t_chunk = bn == 256 ? 0.9 : bn >= 64 ? 0.6 : 0.54;
+        const double fixed = bn == 256 ? 12.0 : 6.0;
+        for (int sp = 1; sp <= 8; ++sp) {
+            if (fsp && sp != fsp) continue;
+            if (sp > 1 && kc / sp < 2) break;
+            const int64_t clusters = groups * ceil_div(m, bn);
+            int64_t waves = ceil_div(clusters * sp, sms);
+            if (sp > 1) {
+                const int mc = max_clusters(bn, sp);
+                if (mc < 1) continue;
+                waves = ceil_div(clusters, mc);
+                if (!fsp && waves > 1) continue;
+            }
+            const double cost = (double)waves * ((double)ceil_div(kc, sp) * t_chunk + fixed + (sp > 1 ? 2.0 : 0.0));
+            if (cost < best_cost) {
+                best_cost = cost;
+                best_bn = bn;
+                best_s = sp;
+            }
         }
     }
-    return best;
+    bn_out = best_bn;
+    splits_out = best_s;
 }
 
 vox_status launch_q4_gemm(const uint8_t* w, int64_t n, int64_t k, const void* x, int64_t m, int64_t ldx, void* y,
@@ -331,7 +483,10 @@ vox_status launch_q4_gemm(const uint8_t* w, int64_t n, int64_t k, const void* x,
     a.op = ep ? ep->op : VOX_EP_NONE;
     a.res = ep ? ep->residual : nullptr;
     a.ldr = ep ? ep->ldr : 0;
-    switch (pick_bn(a.tiles, m)) {
+    int bn = 256, splits = 1;
+    pick_tile(a.tiles, m, a.kc, bn, splits);
+    a.splits = splits;
+    switch (bn) {
     case 32: return launch_gemm_bn<32>(a, x, ldx, s);
     case 64: return launch_gemm_bn<64>(a, x, ldx, s);
     case 128: return launch_gemm_bn<128>(a, x, ldx, s);

@@ -79,6 +79,35 @@ inline vox_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
     return VOX_OK;
 }
 
+// The same launch as one grid of thread-block clusters of cluster_z CTAs
+// along z (the CTAs of a cluster are co-scheduled and share distributed
+// shared memory).
+template <typename... KArgs, typename... Args>
+inline vox_status launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                     cudaStream_t stream, unsigned cluster_z, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = cluster_z;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    if (e != cudaSuccess) {
+        set_cuda_error(e);
+        return VOX_ERR_CUDA;
+    }
+    return VOX_OK;
+}
+
 // ------------------------------------------------------------- device side
 // Device status word: a bounded wait that gives up records where it stopped.
 // Read (and cleared) by the host through vox_device_status in api.cu.

@@ -564,3 +564,36 @@ def test_gemv_kv_append_rope(env, pos, theta):
     kb = bf16_bits(kc)
     for i in range(m):
         assert np.array_equal(kb[:, (pos + i) % W], ref.f32_to_bf16(np_of(y)[i, QD:QD + KVD]).reshape(n_kv, hd))
+
+
+@pytest.mark.parametrize("splits,bn", [(1, 64), (2, 128), (3, 256), (7, 128), (8, 32)])
+def test_gemm_split_k(env, monkeypatch, splits, bn):
+    """The GEMM with K split over a cluster of CTAs (partial tiles summed in
+    rank order through distributed shared memory): within tolerance of the
+    oracle for the residual and GELU epilogues, ragged rows and tokens, and
+    identical bits on a second call."""
+    torch, V, WL = env
+    monkeypatch.setenv("VOX_GEMM_SPLITS", str(splits))
+    monkeypatch.setenv("VOX_GEMM_BN", str(bn))
+    n, k, m = 1296, 1280, 200
+    qs, d = synth.q4_blocks(n, k, 0, 13101)
+    xb = synth.bf16_normal((m, k), 0, 13102)
+    res = synth.activations(m, n, 0, 13103)
+    packed, w = WL.pack_q4(qs, d, "cuda")
+    x = ref.bf16_to_f64(xb)
+    Wd = ref.q4_weights(qs, d)
+    yref = x @ Wd.T
+    xd = WL.bf16_dev(xb, "cuda")
+    outs = []
+    for _ in range(2):
+        y = WL.to_dev(res, "cuda")
+        ep = V.vox_epilogue(op=V.VOX_EP_RESIDUAL, residual=y.data_ptr(), ldr=n)
+        V.vox_q4_gemm(w, xd, V.VOX_BF16, m, k, y, V.VOX_F32, n, ep)
+        check_status(V)
+        outs.append(np_of(y))
+    assert np.array_equal(outs[0].view(np.uint32), outs[1].view(np.uint32))
+    assert ref.gemv_error(outs[0] - res, yref, x, Wd) <= TOL
+    yb = torch.zeros((m, n), dtype=torch.bfloat16, device="cuda")
+    V.vox_q4_gemm(w, xd, V.VOX_BF16, m, k, yb, V.VOX_BF16, n, V.vox_epilogue(op=V.VOX_EP_GELU))
+    check_status(V)
+    assert ref.gemv_error(ref.bf16_to_f64(bf16_bits(yb)), ref.gelu(yref), x, Wd) <= TOL
