@@ -5,27 +5,37 @@
 // n_hist + i and sees key position p iff pos_i - window < p <= pos_i; keys
 // before n_hist come from the history rows, the rest from the chunk itself.
 //
-// One CTA per (32 query rows, head): two warps of 16 query rows each, so
-// the 256-row chunk x 32 heads gives 256 CTAs.  The keys a CTA needs (its
-// 32 rows' windows, 781 positions at window 750) stream through a 3-stage
-// ring of 64-key K and V tiles filled with 16-byte cp.async copies, so the
-// loads of tile i + 2 overlap the math of tile i.  Per tile (80-byte rows,
-// which ldmatrix reads without bank conflicts):
+// One CTA of eight warps per (32 query rows, head), so the 256-row chunk x
+// 32 heads gives 256 CTAs, two per SM.  The keys a CTA needs (its 32 rows'
+// windows, 781 positions at window 750) are cut into 64-key tiles, dealt to
+// four key splits in rounds (round r holds tiles 4r .. 4r+3): warp w takes
+// query rows 16 (w & 1) .. +15 and the tiles of split w >> 1.  A round's
+// four K and V tiles are loaded by the whole CTA with 16-byte cp.async
+// copies into one of two buffers, so the next round's loads overlap this
+// round's math.  Per tile (80-byte rows, which ldmatrix reads without bank
+// conflicts):
 //   S = Q K^T        mma m16n8k16 bf16, head_dim padded to 48 with zeros
 //   online softmax in the exp2 domain, masked by position
 //   O += P V         P split into bf16 hi + lo parts (two MMAs)
+// At the end each warp leaves its rows' (m, l, O) in shared memory and the
+// CTA merges the four splits of every row max-first in split order.
 #include "tma.cuh"
 
 namespace vox {
 
 constexpr int kWinQ = 32;       // query rows per CTA
-constexpr int kWinWarps = kWinQ / 16;
+constexpr int kWinSplits = 4;   // key splits per CTA
+constexpr int kWinWarps = (kWinQ / 16) * kWinSplits;
 constexpr int kWinThreads = 32 * kWinWarps;
 constexpr int kWinK = 64;       // keys per tile
-constexpr int kWinStages = 3;
 constexpr int kWinHd = 40;
 constexpr int kWinRow = kWinHd * 2;   // 80 bytes
 constexpr int kWinTile = kWinK * kWinRow;   // one K or V tile
+constexpr int kWinRound = 2 * kWinSplits * kWinTile;   // K and V tiles of one round (40 KB)
+constexpr int kWinSmem = 2 * kWinRound;                 // two round buffers (80 KB)
+// merge area (reuses the round buffers): per warp O[16][40] then (m, l)[16]
+constexpr int kWinMergeFloats = 16 * kWinHd + 32;
+static_assert(kWinWarps * kWinMergeFloats * 4 <= kWinSmem, "merge area must fit the round buffers");
 
 struct WinArgs {
     const uint16_t* q;
@@ -60,39 +70,43 @@ __device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], uint32_t addr)
                  : "r"(addr) : "memory");
 }
 
-// Copies of key tile [j0, j0 + 64) of head h (K and V) into one ring stage;
-// rows at or past j_end are zero-filled.
-__device__ __forceinline__ void win_load_tile(const WinArgs& a, int h, int64_t j0, int64_t j_end, uint8_t* sK,
-                                              uint8_t* sV, int tid)
+// Copies of round r's tiles (tile 4r + sp for split sp, keys from j_begin)
+// into one round buffer: K tiles first, then V tiles; rows at or past j_end
+// (and tiles past the last) are zero-filled.
+__device__ __forceinline__ void win_load_round(const WinArgs& a, int h, int64_t j_begin, int64_t r, int64_t j_end,
+                                               uint8_t* buf, int tid)
 {
-    for (int i = tid; i < kWinK * 5 * 2; i += kWinThreads) {
-        const int mat = i / (kWinK * 5), rem = i - mat * (kWinK * 5), kr = rem / 5, u = rem - kr * 5;
-        const int64_t j = j0 + kr;
+    for (int i = tid; i < 2 * kWinSplits * kWinK * 5; i += kWinThreads) {
+        const int mat = i / (kWinSplits * kWinK * 5), rem = i - mat * (kWinSplits * kWinK * 5);
+        const int sp = rem / (kWinK * 5), rem2 = rem - sp * (kWinK * 5), kr = rem2 / 5, u = rem2 - kr * 5;
+        const int64_t j = j_begin + (r * kWinSplits + sp) * kWinK + kr;
         const bool in = j < j_end;
         const int64_t jj = in ? j : j_end - 1;                 // a valid address; nothing is read when !in
         const uint16_t* src = jj < a.n_hist ? (mat ? a.vh : a.kh) + jj * a.ld_hist
                                             : (mat ? a.vn : a.kn) + (jj - a.n_hist) * a.ld_new;
-        cp_async16((mat ? sV : sK) + kr * kWinRow + u * 16, src + h * kWinHd + u * 8, in ? 16u : 0u);
+        cp_async16(buf + (mat * kWinSplits + sp) * kWinTile + kr * kWinRow + u * 16, src + h * kWinHd + u * 8,
+                   in ? 16u : 0u);
     }
 }
 
-__global__ void __launch_bounds__(kWinThreads) window_attn_kernel(const WinArgs a)
+__global__ void __launch_bounds__(kWinThreads, 2) window_attn_kernel(const WinArgs a)
 {
-    __shared__ __align__(128) uint8_t sKs[kWinStages][kWinTile];
-    __shared__ __align__(128) uint8_t sVs[kWinStages][kWinTile];
+    extern __shared__ __align__(128) uint8_t win_smem[];
     pdl_wait();
     pdl_launch_dependents();
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
+    const int rg = warp & 1, sp = warp >> 1;                 // row group, key split
     const int h = blockIdx.y;
     const int64_t q0 = (int64_t)blockIdx.x * kWinQ;
-    const int64_t qw = q0 + warp * 16;                       // first query row of this warp
+    const int64_t qw = q0 + rg * 16;                          // first query row of this warp
     const int64_t W = a.window;
     const int64_t n_keys = a.n_hist + a.n_q;
 
     // Q fragments: rows qw+g, qw+g+8; dims 16kk + {2t, 2t+1, 2t+8, 2t+9}
-    uint32_t qa[3][4];
+    // (register order a0a1: row g k lo, a2a3: row g+8 k lo, a4a5: row g k hi, a6a7: row g+8 k hi)
+    uint32_t A[3][4];
 #pragma unroll
     for (int kk = 0; kk < 3; ++kk) {
 #pragma unroll
@@ -101,18 +115,9 @@ __global__ void __launch_bounds__(kWinThreads) window_attn_kernel(const WinArgs 
             const bool ok = row < a.n_q;
             const uint16_t* qr = a.q + (ok ? row : 0) * a.ldq + h * kWinHd;
             const int d0 = 16 * kk + 2 * t, d1 = d0 + 8;
-            qa[kk][hf] = (ok && d0 < kWinHd) ? ld_pair(qr + d0) : 0u;
-            qa[kk][2 + hf] = (ok && d1 < kWinHd) ? ld_pair(qr + d1) : 0u;
+            A[kk][hf] = (ok && d0 < kWinHd) ? ld_pair(qr + d0) : 0u;
+            A[kk][2 + hf] = (ok && d1 < kWinHd) ? ld_pair(qr + d1) : 0u;
         }
-    }
-    // fragment register order: a0a1 (row g, k lo), a2a3 (row g+8, k lo), a4a5 (row g, k hi), a6a7 (row g+8, k hi)
-    uint32_t A[3][4];
-#pragma unroll
-    for (int kk = 0; kk < 3; ++kk) {
-        A[kk][0] = qa[kk][0];
-        A[kk][1] = qa[kk][1];
-        A[kk][2] = qa[kk][2];
-        A[kk][3] = qa[kk][3];
     }
 
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
@@ -126,25 +131,20 @@ __global__ void __launch_bounds__(kWinThreads) window_attn_kernel(const WinArgs 
     const int64_t j_begin = p_lo - W + 1 > 0 ? p_lo - W + 1 : 0;
     const int64_t j_end = p_hi + 1 < n_keys ? p_hi + 1 : n_keys;
     const int64_t ntiles = j_end > j_begin ? (j_end - j_begin + kWinK - 1) / kWinK : 0;
+    const int64_t nrounds = (ntiles + kWinSplits - 1) / kWinSplits;
 
-    // prologue: the first two tiles in flight
-#pragma unroll
-    for (int st = 0; st < kWinStages - 1; ++st) {
-        if (st < ntiles) win_load_tile(a, h, j_begin + (int64_t)st * kWinK, j_end, sKs[st], sVs[st], tid);
+    if (nrounds > 0) win_load_round(a, h, j_begin, 0, j_end, win_smem, tid);
+    cp_async_commit();
+    for (int64_t r = 0; r < nrounds; ++r) {
+        cp_async_wait<0>();                                  // round r has landed (this thread's copies)
+        __syncthreads();                                     // ... everyone's; and round r-1's buffer is free
+        if (r + 1 < nrounds) win_load_round(a, h, j_begin, r + 1, j_end, win_smem + ((r + 1) & 1) * kWinRound, tid);
         cp_async_commit();
-    }
-    for (int64_t it = 0; it < ntiles; ++it) {
-        const int64_t j0 = j_begin + it * kWinK;
-        cp_async_wait<kWinStages - 2>();                     // tile `it` has landed (this thread's copies)
-        __syncthreads();                                     // ... everyone's; and stage it-1 is free
-        {
-            const int64_t nx = it + kWinStages - 1;
-            const int sn = (int)(nx % kWinStages);
-            if (nx < ntiles) win_load_tile(a, h, j_begin + nx * kWinK, j_end, sKs[sn], sVs[sn], tid);
-            cp_async_commit();
-        }
-        const int sc = (int)(it % kWinStages);
-        const uint32_t sKa = smem_addr(sKs[sc]), sVa = smem_addr(sVs[sc]);
+        const int64_t tile = r * kWinSplits + sp;
+        if (tile >= ntiles) continue;                        // warp-uniform: this split has no tile this round
+        const int64_t j0 = j_begin + tile * kWinK;
+        uint8_t* buf = win_smem + (r & 1) * kWinRound;
+        const uint32_t sKa = smem_addr(buf + sp * kWinTile), sVa = smem_addr(buf + (kWinSplits + sp) * kWinTile);
 
         // ---- S = Q K^T : 8 n-tiles of 8 keys
         float s[8][4];
@@ -251,25 +251,50 @@ __global__ void __launch_bounds__(kWinThreads) window_attn_kernel(const WinArgs 
         }
     }
 
-    // ---- normalise and store rows g, g+8
+    // ---- this warp's (m, l, O) of its 16 rows -> shared memory, then the
+    // four splits of every (row, dim) merged max-first in split order
+    __syncthreads();                                         // every warp is done with the round buffers
+    float* mw = reinterpret_cast<float*>(win_smem) + warp * kWinMergeFloats;
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-        const int64_t qi = qw + g + 8 * hf;
-        if (qi >= a.n_q) continue;
-        const float inv = 1.0f / l_run[hf];
+        const int row = g + 8 * hf;
 #pragma unroll
         for (int n = 0; n < 5; ++n) {
             const int d = 8 * n + 2 * t;
-            const float v0 = o[n][2 * hf] * inv, v1 = o[n][2 * hf + 1] * inv;
-            const int64_t idx = qi * a.ldo + h * kWinHd + d;
-            if (a.out_bf16) {
-                static_cast<uint16_t*>(a.out)[idx] = f32_to_bf16_bits(v0);
-                static_cast<uint16_t*>(a.out)[idx + 1] = f32_to_bf16_bits(v1);
-            } else {
-                static_cast<float*>(a.out)[idx] = v0;
-                static_cast<float*>(a.out)[idx + 1] = v1;
-            }
+            mw[row * kWinHd + d] = o[n][2 * hf];
+            mw[row * kWinHd + d + 1] = o[n][2 * hf + 1];
         }
+        if (t == 0) {
+            mw[16 * kWinHd + 2 * row] = m_run[hf];
+            mw[16 * kWinHd + 2 * row + 1] = l_run[hf];
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < kWinQ * kWinHd; e += kWinThreads) {
+        const int row = e / kWinHd, d = e - row * kWinHd;
+        const int64_t qi = q0 + row;
+        if (qi >= a.n_q) continue;
+        const int rgi = row >> 4, rl = row & 15;
+        float M = -INFINITY;
+#pragma unroll
+        for (int s2 = 0; s2 < kWinSplits; ++s2)
+            M = fmaxf(M, reinterpret_cast<const float*>(win_smem)[(2 * s2 + rgi) * kWinMergeFloats + 16 * kWinHd + 2 * rl]);
+        float O = 0.f, L = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < kWinSplits; ++s2) {
+            const float* ms = reinterpret_cast<const float*>(win_smem) + (2 * s2 + rgi) * kWinMergeFloats;
+            const float mv = ms[16 * kWinHd + 2 * rl];
+            if (mv == -INFINITY) continue;
+            const float f = exp2f(mv - M);
+            O = fmaf(f, ms[rl * kWinHd + d], O);
+            L = fmaf(f, ms[16 * kWinHd + 2 * rl + 1], L);
+        }
+        const float v = O / L;
+        const int64_t idx = qi * a.ldo + h * kWinHd + d;
+        if (a.out_bf16)
+            static_cast<uint16_t*>(a.out)[idx] = f32_to_bf16_bits(v);
+        else
+            static_cast<float*>(a.out)[idx] = v;
     }
 }
 
@@ -299,8 +324,11 @@ vox_status launch_window_attn(const void* q, int64_t ldq, const void* k_hist, co
     a.n_heads = n_heads;
     a.window = window;
     a.sl2 = scale * 1.4426950408889634f;
+    static std::atomic<unsigned long long> attr_done{0};
+    vox_status st = smem_attr_per_device(reinterpret_cast<const void*>(window_attn_kernel), kWinSmem, attr_done);
+    if (st != VOX_OK) return st;
     dim3 grid((unsigned)ceil_div(n_q, kWinQ), (unsigned)n_heads);
-    return launch_pdl(window_attn_kernel, grid, dim3(kWinThreads), 0, s, a);
+    return launch_pdl(window_attn_kernel, grid, dim3(kWinThreads), kWinSmem, s, a);
 }
 
 }  // namespace vox
