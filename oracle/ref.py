@@ -414,6 +414,15 @@ def window_attn(Q, K, V, q_pos0, window, n_heads, head_dim, scale=None):
     return out
 
 
+def roll_history(hist, new, window):
+    """Streaming chunks (voxtral.c page, "주요 기능": the encoder takes the audio
+    in overlapping chunks; reading R18): the next chunk's history of a layer
+    is the last `window` rows of this chunk's history followed by its own new
+    k (or v) rows, oldest first."""
+    both = np.concatenate([np.asarray(hist), np.asarray(new)], axis=0)
+    return both[both.shape[0] - window:].copy()
+
+
 def encoder_layer(X, Wd, k_hist, v_hist, window, n_heads, head_dim, eps=RMS_EPS):
     """One pre-norm encoder layer over a chunk of rows (R8, R9).
 

@@ -894,3 +894,38 @@ def test_planted_mistakes_in_rope_are_caught():
     for bad in (half_split, wrong_sign, wrong_frequency):
         with pytest.raises(AssertionError):
             pin_rope(bad)
+
+
+# ------------------------------------------------------- streaming history
+def pin_roll(roll):
+    """After any sequence of chunks the history is exactly the last `window`
+    positions seen, oldest first (a list model), for chunks shorter than,
+    equal to and longer than the window."""
+    for W, sizes in ((5, [2, 3, 1, 4]), (4, [4, 4]), (3, [7, 1, 2]), (750, [256, 256, 256, 256])):
+        hist = -np.arange(W, 0, -1).reshape(W, 1)                 # positions -W .. -1
+        seen = list(range(-W, 0))
+        nxt = 0
+        for n in sizes:
+            new = np.arange(nxt, nxt + n).reshape(n, 1)
+            nxt += n
+            seen += list(range(nxt - n, nxt))
+            hist = roll(hist, new, W)
+            assert hist.shape == (W, 1) and hist[:, 0].tolist() == seen[-W:]
+
+
+def test_roll_history_list_model():
+    pin_roll(ref.roll_history)
+
+
+def test_planted_mistakes_in_roll_are_caught():
+    def first_rows(hist, new, window):
+        both = np.concatenate([hist, new])
+        return both[:window].copy()
+
+    def new_first(hist, new, window):
+        both = np.concatenate([new, hist])
+        return both[both.shape[0] - window:].copy()
+
+    for bad in (first_rows, new_first):
+        with pytest.raises(AssertionError):
+            pin_roll(bad)
