@@ -183,9 +183,13 @@ __device__ __forceinline__ int32_t ld_relaxed_s32(const int32_t* p)
     return v;
 }
 
+// Record `where` in the status word, then raise the abort flag.  The fence
+// orders the two: a CTA that sees the flag and records its own code finds
+// this code already there, so the word names the wait that gave up first.
 __device__ __forceinline__ void ps_raise(const PsArgs& P, const PsWs& W, int32_t where)
 {
     atomicCAS(&g_vox_device_status, 0, where);
+    __threadfence();
     atomicExch(reinterpret_cast<int32_t*>(P.ws + W.abort), 1);
 }
 

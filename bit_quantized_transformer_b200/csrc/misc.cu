@@ -137,6 +137,41 @@ vox_status launch_cast_rows(const float* x, int64_t m, int64_t n, int64_t ldx, v
                       static_cast<const float*>(nullptr), out, (int)(out_dtype == VOX_BF16), ldo, 0);
 }
 
+// ------------------------------------------------------------ history roll
+// Streaming encoder chunks ("주요 기능": the encoder takes the audio in
+// overlapping chunks): the next chunk's history of one layer is the last
+// `window` rows of this chunk's history followed by its own R new rows.
+// Row i of the result is history row i + R while i + R < window, else new
+// row i - (window - R) (when R >= window only new rows remain).  bf16 rows
+// of `dim` elements, copied 16 bytes at a time; the output never aliases the
+// inputs.
+__global__ void hist_roll_kernel(const uint16_t* __restrict__ hist, int64_t ld_hist, const uint16_t* __restrict__ nw,
+                                 int64_t ld_new, int64_t R, int64_t window, int64_t dim, uint16_t* __restrict__ out,
+                                 int64_t ld_out)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t per_row = dim / 8;
+    const int64_t total = window * per_row;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / per_row, c = (i - r * per_row) * 8;
+        const int64_t src_h = r + R;
+        const uint16_t* src = src_h < window ? hist + src_h * ld_hist + c : nw + (src_h - window) * ld_new + c;
+        *reinterpret_cast<uint4*>(out + r * ld_out + c) = *reinterpret_cast<const uint4*>(src);
+    }
+}
+
+vox_status launch_hist_roll(const void* hist, int64_t ld_hist, const void* nw, int64_t ld_new, int64_t R,
+                            int64_t window, int64_t dim, void* out, int64_t ld_out, cudaStream_t s)
+{
+    const int64_t total = window * (dim / 8);
+    int64_t blocks = ceil_div(total, 256);
+    if (blocks > 4 * 148) blocks = 4 * 148;
+    return launch_pdl(hist_roll_kernel, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const uint16_t*>(hist),
+                      ld_hist, static_cast<const uint16_t*>(nw), ld_new, R, window, dim, static_cast<uint16_t*>(out),
+                      ld_out);
+}
+
 // --------------------------------------------------------- position advance
 __global__ void advance_pos_kernel(int64_t* pos, int n)
 {

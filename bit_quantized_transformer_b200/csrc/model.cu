@@ -35,6 +35,8 @@ vox_status launch_gqa_decode_attn_seqs(const float*, const void*, const void*, f
                                        const int64_t*, float, void*, cudaStream_t, int, const int32_t*, int64_t,
                                        int64_t);
 vox_status launch_advance_pos(int64_t*, cudaStream_t, int n = 1);
+vox_status launch_hist_roll(const void*, int64_t, const void*, int64_t, int64_t, int64_t, int64_t, void*, int64_t,
+                            cudaStream_t);
 vox_status launch_rmsnorm(const float*, int64_t, int64_t, int64_t, float, const float*, void*, int, int64_t,
                           cudaStream_t);
 vox_status launch_cast_rows(const float*, int64_t, int64_t, int64_t, void*, int, int64_t, cudaStream_t);
@@ -321,6 +323,14 @@ vox_status vox_encoder_chunk(const vox_encoder* e, void* stream)
         if ((st = check_w(e->wup[l], F, D))) return st;
         if ((st = check_w(e->wdown[l], D, F))) return st;
         if (!e->k_hist[l] || !e->v_hist[l]) return VOX_ERR_NULL;
+        if (e->k_hist_next || e->v_hist_next) {
+            if (!e->k_hist_next || !e->v_hist_next || !e->k_hist_next[l] || !e->v_hist_next[l]) return VOX_ERR_NULL;
+            const void* outs[2] = {e->k_hist_next[l], e->v_hist_next[l]};
+            for (const void* o : outs) {
+                if (!al16(o)) return VOX_ERR_ALIGN;
+                if (o == e->k_hist[l] || o == e->v_hist[l]) return VOX_ERR_ALIGN;
+            }
+        }
     }
     if ((st = check_w(e->adapter, e->adapter_out, 4 * D))) return st;
     if ((st = check_w(e->adapter2, e->adapter_out, e->adapter_out))) return st;
@@ -337,6 +347,12 @@ vox_status vox_encoder_chunk(const vox_encoder* e, void* stream)
         if ((st = launch_window_attn(qkv, 3 * D, e->k_hist[l], e->v_hist[l], D, e->window, qkv + D, qkv + 2 * D,
                                      3 * D, R, e->att, VOX_BF16, D, e->n_heads, e->head_dim, e->window, scale, s)))
             return st;
+        if (e->k_hist_next) {
+            if ((st = launch_hist_roll(e->k_hist[l], D, qkv + D, 3 * D, R, e->window, D, e->k_hist_next[l], D, s)))
+                return st;
+            if ((st = launch_hist_roll(e->v_hist[l], D, qkv + 2 * D, 3 * D, R, e->window, D, e->v_hist_next[l], D, s)))
+                return st;
+        }
         vox_epilogue r = {};
         r.op = VOX_EP_RESIDUAL;
         r.residual = e->x;

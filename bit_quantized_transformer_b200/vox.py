@@ -69,7 +69,8 @@ class vox_encoder(ctypes.Structure):
                 ("adapter", vox_q4_weight), ("adapter2", vox_q4_weight),
                 ("k_hist", ctypes.POINTER(_P)), ("v_hist", ctypes.POINTER(_P)),
                 ("x", _P), ("xn", _P), ("qkv", _P), ("att", _P), ("up", _P), ("adapter_mid", _P),
-                ("adapter_out_buf", _P), ("tap", _P)]
+                ("adapter_out_buf", _P), ("tap", _P), ("k_hist_next", ctypes.POINTER(_P)),
+                ("v_hist_next", ctypes.POINTER(_P))]
 
 
 _W = ctypes.POINTER(vox_q4_weight)

@@ -307,7 +307,7 @@ class EncoderModel:
     """Synthetic encoder chunk: rows x dim input, per-layer history caches, adapter."""
 
     def __init__(self, shape: synth.EncoderShape, seed: int = 0, device="cuda", n_layers=None, eps: float = 1e-5,
-                 tap: bool = False):
+                 tap: bool = False, stream: bool = False):
         self.shape = shape
         self.L = shape.n_layers if n_layers is None else n_layers
         D, F, R = shape.dim, shape.ffn, shape.rows
@@ -358,6 +358,31 @@ class EncoderModel:
         e.tap = self.tap.data_ptr() if tap else None
         self.enc = e
         self.adapter, self.adapter2 = ad, ad2
+        # streaming: a second set of history buffers that receives the next chunk's history
+        self.k_next = self.v_next = None
+        if stream:
+            self.k_next = [torch.zeros_like(t) for t in self.k_hist]
+            self.v_next = [torch.zeros_like(t) for t in self.v_hist]
+            self._point_history()
+
+    def _point_history(self):
+        Ptr = ctypes.c_void_p * self.L
+        self._hist_arrs = [Ptr(*[t.data_ptr() for t in lst]) for lst in (self.k_hist, self.v_hist, self.k_next,
+                                                                          self.v_next)]
+        e = self.enc
+        e.k_hist, e.v_hist, e.k_hist_next, e.v_hist_next = [ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))
+                                                            for a in self._hist_arrs]
+
+    def swap_history(self):
+        """After a streamed chunk: the written next histories become the histories."""
+        self.k_hist, self.k_next = self.k_next, self.k_hist
+        self.v_hist, self.v_next = self.v_next, self.v_hist
+        self._point_history()
+
+    def set_input(self, x: np.ndarray):
+        """A new chunk input (fp32 [rows][dim]); reset() restores it."""
+        self.x0 = to_dev(x, self.x.device)
+        self.x.copy_(self.x0)
 
     def reset(self):
         self.x.copy_(self.x0)

@@ -488,13 +488,24 @@ typedef struct {
                                     layer's input x (tap[0]) and its residual stream h
                                     after attention (tap[1]), so that layer can be checked
                                     on its own inputs                                   */
+    void *const *k_hist_next;    /* host array [n_layers] of device bf16 [window][dim], or
+                                    NULL: streaming (P4 주요 기능, overlapping chunks):
+                                    receives the next chunk's history of each layer, the
+                                    last `window` rows of this chunk's history followed by
+                                    its own k (v) rows; must not alias k_hist (v_hist).  The
+                                    caller swaps the two sets between chunks             */
+    void *const *v_hist_next;
 } vox_encoder;
 
 /* One encoder chunk: 32 x {RMSNorm, QKV GEMM, window attention, O GEMM +
  * residual, RMSNorm, up GEMM + GELU, down GEMM + residual}, then the 4x
  * downsample (rows 4r..4r+3 concatenated) and the adapter ([ARCH]: Linear
  * 4dim -> adapter_out, exact-erf GELU, Linear adapter_out -> adapter_out;
- * the GELU output is rounded to bf16 in adapter_mid). */
+ * the GELU output is rounded to bf16 in adapter_mid).  With k_hist_next and
+ * v_hist_next set, every layer also writes the next chunk's history after its
+ * attention, so consecutive chunks see each other through the 750-row window.
+ * Errors: NULL fields -> VOX_ERR_NULL; shapes -> VOX_ERR_SHAPE; misaligned
+ * buffers or a next history that is one of the inputs -> VOX_ERR_ALIGN. */
 vox_status vox_encoder_chunk(const vox_encoder *enc, void *stream);
 
 #ifdef __cplusplus

@@ -402,3 +402,44 @@ def test_decoder_layer_rope(env, form):
     err = gemv_err(back[None], ref.rmsnorm(x0)[None], qs, ds)
     assert err <= TOL, err
     check_layer_tail(shape, 0, dm, 0, filled)
+
+
+def test_encoder_streaming_two_chunks(env):
+    """Two chunks streamed through a 1-layer encoder: after the first, the
+    next history is bit for bit the oracle's roll of the old history and the
+    chunk's own k, v rows; the second chunk's window attention, on the GPU's
+    q, k, v and that history, matches the oracle."""
+    torch, V, WL = env
+    shape = synth.EncoderShape(n_layers=1)
+    D, R, W, nh, hd = shape.dim, shape.rows, shape.window, shape.n_heads, shape.head_dim
+    em = WL.EncoderModel(shape, seed=0, n_layers=1, stream=True)
+    kh0, vh0 = bits(em.k_hist[0]), bits(em.v_hist[0])
+    em.reset()
+    em.run()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    qkv1 = bits(em.qkv)
+    assert np.array_equal(bits(em.k_next[0]), ref.roll_history(kh0, qkv1[:, D:2 * D], W))
+    assert np.array_equal(bits(em.v_next[0]), ref.roll_history(vh0, qkv1[:, 2 * D:], W))
+    em.swap_history()
+    em.set_input(synth.activations(R, D, 0, synth.ENC_X_ID + 7))
+    em.run()
+    torch.cuda.synchronize()
+    assert V.vox_device_status(True) == 0
+    kh, vh = bits(em.k_hist[0]), bits(em.v_hist[0])
+    qkv = bits(em.qkv)
+    Q = ref.bf16_to_f64(qkv[:, :D])
+    K = np.concatenate([ref.bf16_to_f64(kh), ref.bf16_to_f64(qkv[:, D:2 * D])])
+    Vv = np.concatenate([ref.bf16_to_f64(vh), ref.bf16_to_f64(qkv[:, 2 * D:])])
+    att = ref.bf16_to_f64(bits(em.att))
+    for i in list(range(0, R, 17)) + [R - 1]:
+        o_ref = ref.window_attn(Q[i:i + 1], K, Vv, W + i, W, nh, hd)[0]
+        p = W + i
+        half_ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(o_ref), 1e-30))) - 8)
+        for hh in range(nh):
+            sl = slice(hh * hd, (hh + 1) * hd)
+            sc = (K[p - W + 1:p + 1, sl] @ Q[i, sl]) / math.sqrt(hd)
+            pr = np.exp(sc - sc.max()); pr /= pr.sum()
+            den = np.linalg.norm(pr) * np.linalg.norm(Vv[p - W + 1:p + 1, sl], axis=0)
+            excess = np.maximum(np.abs(att[i, sl] - o_ref[sl]) - half_ulp[sl], 0.0)
+            assert np.max(excess / den) <= TOL, ("attention", i, hh)
