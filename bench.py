@@ -357,23 +357,26 @@ def run_ours(args):
     assert step_bytes == sum(decoder_bytes(shape))
     peak, peak_src = measured_peaks()
 
-    # The two forms of the product's token step: one persistent launch
-    # (vox_decoder_step) and the per-kernel launch sequence
-    # (vox_decoder_step_kernels), each replayed from a CUDA graph (the
-    # persistent launch is launched directly if the runtime will not capture
-    # it).  Both are timed briefly; the faster one is the headline.
+    # The three forms of the product's token step: one persistent launch
+    # (vox_decoder_step), the per-kernel launch sequence
+    # (vox_decoder_step_kernels) and persistent projection segments between
+    # attention launches (vox_decoder_step_fused), each replayed from a CUDA
+    # graph (launched directly if the runtime will not capture it).  All are
+    # timed briefly; the fastest one is the headline.
     g_p = try_graph(dm.step)
     step_p = g_p.replay if g_p is not None else dm.step
+    g_f = try_graph(dm.step_fused)
+    step_f = g_f.replay if g_f is not None else dm.step_fused
     g_k = dm.capture(dm.step_kernels)
     forms = {}
-    for name, fn in (("persistent", step_p), ("kernels", g_k.replay)):
+    for name, fn in (("persistent", step_p), ("kernels", g_k.replay), ("fused", step_f)):
         for _ in range(max(3, args.warmup)):
             fn()
         torch.cuda.synchronize()
         assert V.vox_device_status(True) == 0, f"device status after the {name} warm-up"
         forms[name] = time_fn(fn, 10, world) / 10
     form = min(forms, key=forms.get)
-    step = step_p if form == "persistent" else g_k.replay
+    step = {"persistent": step_p, "kernels": g_k.replay, "fused": step_f}[form]
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
@@ -425,6 +428,8 @@ def run_ours(args):
         dm.token.copy_(tok_h, non_blocking=True)
         if form == "persistent":
             V.vox_decoder_step(dm.dec, s)
+        elif form == "fused":
+            step_f()
         else:
             g_k.replay()
         out_h.copy_(dm.token, non_blocking=True)
@@ -447,8 +452,11 @@ def run_ours(args):
             "vs_baseline": None, "dtype": "q4_0 weights, fp16/bf16 tensor-core inputs, f32 accumulate",
             "data": "synthetic",
             "config": decoder_config(shape, world),
-            "launch": ("one persistent cooperative launch per step" if form == "persistent" else
-                       f"the {dm.step_kernels_launches()}-launch kernel sequence per step") + ", replayed from a CUDA graph",
+            "launch": {"persistent": "one persistent cooperative launch per step",
+                       "fused": f"{dm.step_fused_launches()} launches per step (attention + persistent projection "
+                                "segments)",
+                       "kernels": f"the {dm.step_kernels_launches()}-launch kernel sequence per step"}[form] +
+                      ", replayed from a CUDA graph",
             "roofline": roof,
             "step_form": form,
             "forms_ms_per_step": forms,
@@ -459,12 +467,14 @@ def run_ours(args):
                         "frac": k1_gbs / peak},
             "k4_attention": {"kernel": "gqa_decode_attn_kernel+attn_combine_kernel", "gbs":
                              attn_bytes / (ms_a / 1e3) / 1e9, "us_per_layer": ms_a / dm.L * 1e3},
-            "gpu_launches": (dm.step_launches() if form == "persistent" else dm.step_kernels_launches()) * args.steps,
+            "gpu_launches": {"persistent": dm.step_launches(), "fused": dm.step_fused_launches(),
+                             "kernels": dm.step_kernels_launches()}[form] * args.steps,
             "clocks": clk,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4,
                     "ms_per_step": e2e_local / e2e_steps,
-                    "api": ("vox_decoder_step through the C ABI" if form == "persistent" else
-                            "vox_decoder_step_kernels captured once in a CUDA graph, replayed") +
+                    "api": {"persistent": "vox_decoder_step through the C ABI",
+                            "fused": "vox_decoder_step_fused captured once in a CUDA graph, replayed",
+                            "kernels": "vox_decoder_step_kernels captured once in a CUDA graph, replayed"}[form] +
                            " each step, token H2D before and D2H after, host synchronised every step"},
             "cpu_baseline": cpu,
         }

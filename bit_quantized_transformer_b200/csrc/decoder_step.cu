@@ -93,6 +93,7 @@ struct PsArgs {
     int32_t n_layers, dim, q_dim, kv_dim, ffn, vocab, n_kv, group, window;
     float eps, qscale;
     float rope;                      // rotary theta of q and k, 0 = off
+    int32_t ph_begin, ph_end;        // the phases this launch runs (all: 0 .. 5 n_layers + 1)
     uint32_t act_bytes;                      // shared bytes of the activation / merge region
     int32_t test_withhold;                   // test hook: warp 0 of CTA 0 first waits on a barrier nothing completes
 };
@@ -973,7 +974,10 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
         if (tid == 0 && b == 0) atomicCAS(&g_vox_device_status, 0, 0x5D0);
         tok = 0;
     }
-    const int nph = 5 * P.n_layers + 1;
+    // this launch's phases [ph_begin, nph): the whole step, or one segment of
+    // GEMV phases between two attention launches
+    const int nph_all = 5 * P.n_layers + 1;
+    const int nph = P.ph_end;
 
     PsRing ring;
     ring.base = smem + SL.ring + (uint32_t)warp * kPsStages * kPsStageBytes;
@@ -986,10 +990,10 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
     }
     __syncwarp();
     ring.issued = ring.consumed = 0;
-    ring.cur.ph = 0;
+    ring.cur.ph = P.ph_begin;
     ring.cur.idx = 0;
-    ring.cur.f = ps_phase(P, 0, b, G, warp, nch);
-    ps_ring_fill(P, ring, nph, b, G, warp, lane, nch, 0);
+    ring.cur.f = ps_phase(P, P.ph_begin, b, G, warp, nch);
+    ps_ring_fill(P, ring, nph, b, G, warp, lane, nch, P.ph_begin);
 
     bool ok = true;
     if (P.test_withhold && b == 0 && warp == 0) {
@@ -1005,9 +1009,9 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
         }
     }
     PsBest best = {-INFINITY, 0x7fffffff};
-    int ph = 0;
+    int ph = P.ph_begin;
     for (; ph < nph; ++ph) {
-        if (ph > 0 && !ps_grid_barrier(P, W, s_flag, 0x510)) break;
+        if (ph > P.ph_begin && !ps_grid_barrier(P, W, s_flag, 0x510)) break;
         const PsPhase f = ps_phase(P, ph, b, G, warp, nch);
         if (f.kind == PS_ATTN) {
             if (kPsPrefetch < kPsStages) ps_ring_fill(P, ring, nph, b, G, warp, lane, nch, ph);
@@ -1036,7 +1040,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) decoder_step_kernel(const __gri
 
     // ---- greedy argmax: warps -> CTA -> one 64-bit atomic max; the last CTA
     // to arrive writes the token, clears the key and advances the position
-    if (ph == nph) {
+    if (ph == nph && nph == nph_all) {
         if (lane == 0) {
             s_best_v[warp] = best.v;
             s_best_i[warp] = best.i;
@@ -1102,7 +1106,7 @@ bool decoder_step_fits(const vox_decoder* d)
     return ps_smem_layout(ps_act_bytes(d)).total <= 227 * 1024;
 }
 
-vox_status launch_decoder_step(const vox_decoder* d, uint8_t* ws, cudaStream_t s)
+vox_status launch_decoder_step(const vox_decoder* d, uint8_t* ws, cudaStream_t s, int ph_begin, int ph_end)
 {
     PsArgs a;
     memset(&a, 0, sizeof(a));
@@ -1146,6 +1150,8 @@ vox_status launch_decoder_step(const vox_decoder* d, uint8_t* ws, cudaStream_t s
     a.eps = d->eps;
     a.qscale = (1.0f / sqrtf((float)kPsHd)) * 1.4426950408889634f;
     a.rope = d->rope_theta;
+    a.ph_begin = ph_begin;
+    a.ph_end = ph_end < 0 ? 5 * L + 1 : ph_end;
     a.act_bytes = ps_act_bytes(d);
     const char* hook = getenv("VOX_TEST_WITHHOLD_STAGE");      // test of the bounded waits only
     a.test_withhold = hook && hook[0] == '1';

@@ -48,7 +48,7 @@ vox_status launch_window_attn(const void*, int64_t, const void*, const void*, in
 size_t decoder_step_ws_bytes(int n_layers, int n_kv, int group);
 const char* decoder_step_unsupported(const vox_decoder* d);
 bool decoder_step_fits(const vox_decoder* d);
-vox_status launch_decoder_step(const vox_decoder* d, uint8_t* ws, cudaStream_t s);
+vox_status launch_decoder_step(const vox_decoder* d, uint8_t* ws, cudaStream_t s, int ph_begin = 0, int ph_end = -1);
 void set_error_text(const char* text);
 }  // namespace vox
 
@@ -142,6 +142,37 @@ vox_status vox_decoder_step(const vox_decoder* d, void* stream)
     }
     return launch_decoder_step(d, static_cast<uint8_t*>(d->workspace) + dec_ps_offset(d),
                                static_cast<cudaStream_t>(stream));
+}
+
+vox_status vox_decoder_step_fused(const vox_decoder* d, void* stream)
+{
+    vox_status st = check_decoder(d);
+    if (st) return st;
+    if (const char* why = decoder_step_unsupported(d)) {
+        set_error_text(why);
+        return VOX_ERR_SHAPE;
+    }
+    if (!decoder_step_fits(d)) {
+        set_error_text("the activations of the widest projection do not fit shared memory");
+        return VOX_ERR_SHAPE;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws_g = static_cast<uint8_t*>(d->workspace);
+    uint8_t* ws_a = ws_g + ((dec_gemv_ws(d) + 255) & ~(size_t)255);
+    uint8_t* ws_p = ws_g + dec_ps_offset(d);
+    const float scale = 1.0f / sqrtf((float)d->head_dim);
+    const int L = d->n_layers;
+    // layer 0's QKV (from the embedding row), then per layer the attention and
+    // one persistent launch for Wo, W1||W3, W2 and the next QKV (the LM head
+    // and the position advance after the last layer)
+    if ((st = launch_decoder_step(d, ws_p, s, 0, 1))) return st;
+    for (int l = 0; l < L; ++l) {
+        if ((st = launch_gqa_decode_attn(d->qkv, d->k_cache[l], d->v_cache[l], d->attn, d->n_q_heads, d->n_kv_heads,
+                                         d->head_dim, d->window, 0, d->pos, scale, ws_a, s)))
+            return st;
+        if ((st = launch_decoder_step(d, ws_p, s, 5 * l + 2, l == L - 1 ? 5 * L + 1 : 5 * l + 6))) return st;
+    }
+    return VOX_OK;
 }
 
 vox_status vox_decoder_step_kernels(const vox_decoder* d, void* stream)

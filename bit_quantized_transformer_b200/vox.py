@@ -100,6 +100,7 @@ _SIGS = {
     "vox_decoder_workspace": (_SZ, [ctypes.POINTER(vox_decoder)]),
     "vox_decoder_step": (_I32, [ctypes.POINTER(vox_decoder), _P]),
     "vox_decoder_step_kernels": (_I32, [ctypes.POINTER(vox_decoder), _P]),
+    "vox_decoder_step_fused": (_I32, [ctypes.POINTER(vox_decoder), _P]),
     "vox_decoder_batch_workspace": (_SZ, [ctypes.POINTER(vox_decoder_batch)]),
     "vox_decoder_batch_step": (_I32, [ctypes.POINTER(vox_decoder_batch), _P]),
     "vox_encoder_chunk": (_I32, [ctypes.POINTER(vox_encoder), _P]),
@@ -253,6 +254,10 @@ def vox_decoder_step(dec: vox_decoder, stream=None):
 
 def vox_decoder_step_kernels(dec: vox_decoder, stream=None):
     _check(lib.vox_decoder_step_kernels(ctypes.byref(dec), stream_ptr(stream)), "vox_decoder_step_kernels")
+
+
+def vox_decoder_step_fused(dec: vox_decoder, stream=None):
+    _check(lib.vox_decoder_step_fused(ctypes.byref(dec), stream_ptr(stream)), "vox_decoder_step_fused")
 
 
 def vox_decoder_batch_workspace(b: vox_decoder_batch) -> int:

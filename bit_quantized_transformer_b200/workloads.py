@@ -231,6 +231,11 @@ class DecoderModel:
         """The same step as the library's per-kernel launch sequence."""
         V.vox_decoder_step_kernels(self.dec, stream)
 
+    def step_fused(self, stream=None):
+        """The same step with the projections between attentions fused into
+        persistent launches."""
+        V.vox_decoder_step_fused(self.dec, stream)
+
     # ----------------------------------------------------------- graphs
     def capture(self, fn=None):
         """Capture `fn` (default: one decoder step) into a CUDA graph.  One
@@ -287,6 +292,10 @@ class DecoderModel:
     def step_launches(self) -> int:
         """Kernels one vox_decoder_step launches."""
         return 1
+
+    def step_fused_launches(self) -> int:
+        """Launches of one vox_decoder_step_fused: its own kernels."""
+        return 1 + 3 * self.L
 
     def step_kernels_launches(self) -> int:
         """Kernels one vox_decoder_step_kernels launches."""

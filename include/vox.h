@@ -421,6 +421,17 @@ size_t vox_decoder_workspace(const vox_decoder *dec);
  * these limits).  Other errors as vox_decoder_step_kernels. */
 vox_status vox_decoder_step(const vox_decoder *dec, void *stream);
 
+/* vox_decoder_step_fused -- the same step as 1 + 3 n_layers launches: layer
+ * 0's QKV projection, then per layer the split-KV attention (two launches,
+ * as vox_gqa_decode_attn) and one persistent cooperative launch that runs the
+ * layer's Wo, W1||W3 and W2 projections and the next layer's QKV (after the
+ * last layer: the LM head, argmax and position advance) with grid-wide
+ * barriers between them, streaming each projection's weights into shared
+ * memory while the grid waits at the barrier before it.  Same arithmetic and
+ * limits as vox_decoder_step; can be captured in a CUDA graph.  Errors as
+ * vox_decoder_step. */
+vox_status vox_decoder_step_fused(const vox_decoder *dec, void *stream);
+
 /* vox_decoder_step_kernels -- the same step as a sequence of launches of the
  * library's kernels on one stream (embedding row, per layer the QKV GEMV with
  * rolling append, attention + combine, Wo, W1||W3 and W2 GEMVs, then the LM

@@ -97,14 +97,17 @@ def check_layer_tail(shape, layer, dm, seed, pos_written):
     return w, o
 
 
-FORMS = ["persistent", "kernels"]
+FORMS = ["persistent", "kernels", "fused"]
 
 
 def run_step(dm, form, stream=None):
     """One decoder step in the given form: one persistent launch
-    (vox_decoder_step) or the per-kernel launch sequence."""
+    (vox_decoder_step), the per-kernel launch sequence, or persistent
+    projection segments between attention launches (vox_decoder_step_fused)."""
     if form == "persistent":
         dm.step(stream)
+    elif form == "fused":
+        dm.step_fused(stream)
     else:
         dm.step_kernels(stream)
 
@@ -252,8 +255,9 @@ def test_persistent_step_small_shapes(env, window, filled):
         assert err <= TOL, (form, err)
         assert int(dm.token.item()) == int(np.argmax(logits))
         out[form] = np_of(dm.x)
-    # the two forms reach the same residual stream within the tolerance's scale
-    assert np.max(np.abs(out["persistent"] - out["kernels"])) <= 1e-2 * np.max(np.abs(out["kernels"]))
+    # the forms reach the same residual stream within the tolerance's scale
+    for form in ("persistent", "fused"):
+        assert np.max(np.abs(out[form] - out["kernels"])) <= 1e-2 * np.max(np.abs(out["kernels"]))
 
 
 def test_persistent_step_first_layer_from_embedding(env):
