@@ -16,6 +16,8 @@ roofline   = the dominant kernel (the Q4_0 GEMV, ~69% of the step's bytes),
              timed inside this run over the step's own 105 GEMV launches
 e2e        = the same metric through the Python API with the token copied
              host->device before and device->host after every step
+             (e2e_eager: the same with the C ABI's step called every step,
+             no graph)
 cpu_baseline / --impl reference = the CPU oracle (oracle/) on the host cores
 
 Multi-GPU: one process per GPU (torchrun), independent replicas (the path
@@ -441,6 +443,21 @@ def run_ours(args):
     _, e2e_value = aggregate(e2e_local, e2e_steps, step_bytes, world)
     assert V.vox_device_status(True) == 0, "device status after the end-to-end steps"
 
+    # the same without a graph: every step calls the C ABI's kernel-sequence
+    # step eagerly (its host-side checks and launches included)
+    def e2e_eager_step():
+        dm.token.copy_(tok_h, non_blocking=True)
+        V.vox_decoder_step_kernels(dm.dec, s)
+        out_h.copy_(dm.token, non_blocking=True)
+        s.synchronize()
+        tok_h[0] = out_h[0]
+
+    e2e_eager_step()
+    eager_steps = max(5, min(e2e_steps, 100))
+    e2e_eager_local = time_fn(e2e_eager_step, eager_steps, world)
+    _, e2e_eager_value = aggregate(e2e_eager_local, eager_steps, step_bytes, world)
+    assert V.vox_device_status(True) == 0, "device status after the eager end-to-end steps"
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_seconds)
@@ -476,6 +493,10 @@ def run_ours(args):
                             "fused": "vox_decoder_step_fused captured once in a CUDA graph, replayed",
                             "kernels": "vox_decoder_step_kernels captured once in a CUDA graph, replayed"}[form] +
                            " each step, token H2D before and D2H after, host synchronised every step"},
+            "e2e_eager": {"value": e2e_eager_value, "unit": UNIT, "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4,
+                          "ms_per_step": e2e_eager_local / eager_steps,
+                          "api": "vox_decoder_step_kernels called through the C ABI every step (no graph), token "
+                                 "H2D before and D2H after, host synchronised every step"},
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
