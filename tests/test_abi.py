@@ -291,3 +291,94 @@ def test_paged_append_epilogue_validation(V):
     gm = lambda: L.vox_q4_gemm(ctypes.byref(V.vox_q4_weight(FAKE, 128, 128)), FAKE, V.VOX_BF16, 16, 128, FAKE,
                                V.VOX_F32, 128, ctypes.byref(V.vox_epilogue(op=V.VOX_EP_KV_APPEND_PAGED)), None)
     assert gm() == V.VOX_ERR_RANGE
+
+
+def _fake_decoder(V, L=2, D=256, nq=4, nkv=2, hd=128, F=512, vocab=1024, W=128):
+    """A decoder descriptor whose every pointer is FAKE (never dereferenced:
+    the host checks below fail first) and whose weights have the right shapes."""
+    keep = []
+    Arr = V.vox_q4_weight * L
+    QD, KVD = nq * hd, nkv * hd
+    arrs = [Arr(*[V.vox_q4_weight(FAKE, n, k) for _ in range(L)])
+            for n, k in ((QD + 2 * KVD, D), (D, QD), (2 * F, D), (D, F))]
+    Ptr = ctypes.c_void_p * L
+    caches = [Ptr(*[FAKE] * L), Ptr(*[FAKE] * L)]
+    keep += arrs + caches
+    d = V.vox_decoder()
+    d.n_layers, d.dim, d.n_q_heads, d.n_kv_heads, d.head_dim, d.ffn, d.vocab, d.window = L, D, nq, nkv, hd, F, vocab, W
+    d.eps = 1e-5
+    d.wqkv, d.wo, d.w13, d.w2 = [ctypes.cast(a, ctypes.POINTER(V.vox_q4_weight)) for a in arrs]
+    d.embedding = V.vox_q4_weight(FAKE, vocab, D)
+    d.lm_head = V.vox_q4_weight(FAKE, vocab, D)
+    d.k_cache, d.v_cache = [ctypes.cast(c, ctypes.POINTER(ctypes.c_void_p)) for c in caches]
+    for name in ("token", "pos", "x", "h", "qkv", "attn", "act", "logits", "workspace"):
+        setattr(d, name, FAKE)
+    d.ws_bytes = 1 << 40
+    return d, keep
+
+
+def test_batch_fused_and_rope_validation(V):
+    """Host checks of the batched step, the fused step and the RoPE setting:
+    each bad field is refused before anything reaches the device."""
+    L = V.lib
+    d, keep = _fake_decoder(V)
+    d.rope_theta = -1.0
+    assert L.vox_decoder_step_kernels(ctypes.byref(d), None) == V.VOX_ERR_RANGE
+    assert L.vox_decoder_step_fused(ctypes.byref(d), None) == V.VOX_ERR_RANGE
+    d.rope_theta = float("nan")
+    assert L.vox_decoder_step_fused(ctypes.byref(d), None) == V.VOX_ERR_RANGE
+    d.rope_theta = 0.0
+    d.attn = None
+    assert L.vox_decoder_step_fused(ctypes.byref(d), None) == V.VOX_ERR_NULL
+    d.attn = FAKE
+    b = V.vox_decoder_batch()
+    b.d = d
+    b.n_seq, b.n_pages, b.page_table = 0, 10, FAKE
+    assert L.vox_decoder_batch_step(ctypes.byref(b), None) == V.VOX_ERR_RANGE
+    b.n_seq = 9
+    assert L.vox_decoder_batch_step(ctypes.byref(b), None) == V.VOX_ERR_RANGE
+    b.n_seq = 4
+    b.page_table = None
+    assert L.vox_decoder_batch_step(ctypes.byref(b), None) == V.VOX_ERR_NULL
+    b.page_table = FAKE
+    b.n_pages = 0
+    assert L.vox_decoder_batch_step(ctypes.byref(b), None) == V.VOX_ERR_RANGE
+    b.n_pages = 10
+    b.d.window = 100                                  # not a multiple of the 64-slot page
+    assert L.vox_decoder_batch_step(ctypes.byref(b), None) == V.VOX_ERR_RANGE
+    b.d.window = 128
+    b.d.rope_theta = -2.0
+    assert L.vox_decoder_batch_step(ctypes.byref(b), None) == V.VOX_ERR_RANGE
+    assert L.vox_decoder_batch_workspace(None) == 0
+    ep = V.vox_epilogue(op=V.VOX_EP_RESIDUAL, residual=FAKE, ldr=64, rope_theta=1e4)   # RoPE only with an append
+    w = V.vox_q4_weight(FAKE, 64, 96)
+    assert L.vox_q4_gemv(ctypes.byref(w), FAKE, 1, 96, FAKE, 64, ctypes.byref(ep), FAKE, 256, None) == V.VOX_ERR_RANGE
+    ep = V.vox_epilogue(op=V.VOX_EP_KV_APPEND, k_cache=FAKE, v_cache=FAKE, n_kv_heads=1, head_dim=24, window=4,
+                        q_rows=0, pos=0, rope_theta=1e4)                             # head_dim not a multiple of 16
+    assert L.vox_q4_gemv(ctypes.byref(w), FAKE, 1, 96, FAKE, 64, ctypes.byref(ep), FAKE, 256, None) == V.VOX_ERR_RANGE
+
+
+def test_encoder_streaming_validation(V):
+    """A streamed chunk refuses a next history that is one of its inputs."""
+    L = V.lib
+    Ln = 1
+    Arr = V.vox_q4_weight * Ln
+    D, F, R = 1280, 5120, 256
+    arrs = [Arr(V.vox_q4_weight(FAKE, n, k)) for n, k in ((3 * D, D), (D, D), (F, D), (D, F))]
+    Ptr = ctypes.c_void_p * Ln
+    kh, vh = Ptr(FAKE), Ptr(FAKE + 4096)
+    e = V.vox_encoder()
+    e.n_layers, e.dim, e.n_heads, e.head_dim, e.ffn, e.window, e.rows, e.adapter_out = Ln, D, 32, 40, F, 750, R, 3072
+    e.eps = 1e-5
+    e.wqkv, e.wo, e.wup, e.wdown = [ctypes.cast(a, ctypes.POINTER(V.vox_q4_weight)) for a in arrs]
+    e.adapter = V.vox_q4_weight(FAKE, 3072, 4 * D)
+    e.adapter2 = V.vox_q4_weight(FAKE, 3072, 3072)
+    e.k_hist, e.v_hist = ctypes.cast(kh, ctypes.POINTER(ctypes.c_void_p)), ctypes.cast(vh, ctypes.POINTER(ctypes.c_void_p))
+    for name in ("x", "xn", "qkv", "att", "up", "adapter_mid", "adapter_out_buf"):
+        setattr(e, name, FAKE)
+    kn_alias, vn = Ptr(FAKE), Ptr(FAKE + 8192)
+    e.k_hist_next = ctypes.cast(kn_alias, ctypes.POINTER(ctypes.c_void_p))
+    e.v_hist_next = ctypes.cast(vn, ctypes.POINTER(ctypes.c_void_p))
+    assert L.vox_encoder_chunk(ctypes.byref(e), None) == V.VOX_ERR_ALIGN
+    e.v_hist_next = None
+    assert L.vox_encoder_chunk(ctypes.byref(e), None) == V.VOX_ERR_NULL
