@@ -33,7 +33,11 @@
 //    a warp covers alone is finished from its registers; a tile cut between
 //    warps is summed in warp order from shared memory.  Residuals are loaded
 //    before the main loop.  All sums have a fixed order: the result does not
-//    depend on timing.
+//    depend on timing.  The phase's input vector is scaled by one power of
+//    two per 128 columns (the columns one warp converts) into [2^13, 2^14)
+//    before the fp16 conversion; a record's block MMAs start from the
+//    block's offset constant (`gemv_record_m1`), and a full stage with no
+//    tile end runs its records in groups of four with constant offsets.
 //  * ATTN phases: 16-slot units (kv head, slots) are split evenly over CTAs;
 //    inside a CTA the warps take units round robin, each unit two stages
 //    (its K rows, then its V rows) of two 2-D TMA boxes each (64 columns x
@@ -432,7 +436,9 @@ __device__ __forceinline__ float ps_convert(const PsArgs& P, const float* x, boo
             float am = fmaxf(fmaxf(fabsf(xg.x), fabsf(xg.y)), fmaxf(fabsf(xg.z), fabsf(xg.w)));
             am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
             am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));     // max over the 32-column block
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 8));
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 16));    // max over the warp's 128 columns
             int E = (int)((__float_as_uint(am) >> 23) & 0xFFu);
             E = E < 14 ? 14 : E;
             const float sc = __uint_as_float((uint32_t)(267 - E) << 23);
@@ -449,7 +455,10 @@ __device__ __forceinline__ float ps_convert(const PsArgs& P, const float* x, boo
                 const int word = blk * 16 + 2 * (q & 1) * 4 + (q >> 2) * 2 + ((q & 3) >> 1);
                 s_bs32[word] = *reinterpret_cast<const uint32_t*>(&h01);
                 s_bs32[word + 4] = *reinterpret_cast<const uint32_t*>(&h23);
-                if (q == 0) s_cb[blk] = make_float2(-(1032.0f * s + 72.0f * shi), inv);
+                if (q == 0) {
+                    const float c = -(1032.0f * s + 72.0f * shi);
+                    reinterpret_cast<float4*>(s_cb)[blk] = make_float4(c, inv, c, inv);
+                }
             }
         }
     }
@@ -546,7 +555,7 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
     (void)W;
     (void)ph;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    const int kc = f.kc, nblk = 2 * kc;
+    const int kc = f.kc;
     float* s_piece = reinterpret_cast<float*>(smem + SL.piece);
     const uint32_t tk = smem_token();
     const uint32_t bs_a = smem_addr(smem + SL.act) + tk;
@@ -592,6 +601,29 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
             }
             const uint32_t base = smem_addr(ring.base) + (ring.consumed % kPsStages) * kPsStageBytes + smem_token();
             const int nrec = (int)min64(kPsRecs, we - r);
+            if (nrec == kPsRecs && cin + kPsRecs < kc && r + kPsRecs < we) {
+                // a full stage with no tile end and no range end: chunks cin .. cin + 6,
+                // all records' MMAs in flight together, added straight into the tile's sums
+                const uint32_t bsb = bs_a + 128u * (uint32_t)cin + 16u * (uint32_t)t;
+                const uint32_t cbc = cb_a + 32u * (uint32_t)cin;
+#pragma unroll 1
+                for (int u0 = 0; u0 < kPsRecs; u0 += 4) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (u0 + u >= kPsRecs) break;
+                        const uint32_t o = (uint32_t)(u0 + u);
+                        const uint4 qv = lds128(base + o * kChunkBytes + 16 * lane);
+                        const uint2 e = lds64(base + o * kChunkBytes + kChunkQsBytes + 8 * g);
+                        gemv_record_m1(qv, e, bsb + 128u * o, cbc + 32u * o, acc0, acc2);
+                    }
+                }
+                cin += kPsRecs;
+                r += kPsRecs;
+                __syncwarp();
+                ++ring.consumed;
+                ps_ring_fill(P, ring, nph, b, G, warp, lane, nch, ph);
+                continue;
+            }
             for (int q0 = 0; q0 < nrec; q0 += 2) {
                 // two records' MMAs back to back (a missing second record repeats
                 // the first; its result is not used), then their bookkeeping
@@ -603,7 +635,8 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
                     const uint4 qv = lds128(base + ri * kChunkBytes + 16 * lane);
                     const uint2 e = lds64(base + ri * kChunkBytes + kChunkQsBytes + 8 * g);
                     p[u][0] = p[u][1] = p[u][2] = p[u][3] = 0.f;
-                    gemv_record<1>(qv, e, bs_a, cb_a, nblk, ch, 1, 0, t, p[u]);
+                    gemv_record_m1(qv, e, bs_a + 128u * (uint32_t)ch + 16u * (uint32_t)t, cb_a + 32u * (uint32_t)ch,
+                                   p[u][0], p[u][2]);
                 }
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
@@ -1095,7 +1128,7 @@ static uint32_t ps_act_bytes(const vox_decoder* d)
     const int64_t kmax = d->dim > d->ffn ? (d->dim > (int64_t)d->n_q_heads * kPsHd ? d->dim : (int64_t)d->n_q_heads * kPsHd)
                                          : (d->ffn > (int64_t)d->n_q_heads * kPsHd ? d->ffn : (int64_t)d->n_q_heads * kPsHd);
     const int64_t kc = (kmax + 63) / 64;
-    const int64_t gemv = kc * 128 + 2 * kc * 8;
+    const int64_t gemv = kc * 128 + kc * 32;                   // B fragments, two constant quads per chunk
     const int group = d->n_q_heads / d->n_kv_heads;
     const int64_t mrg = (int64_t)kPsWarps * (group * kPsHd + 2 * group) * 4;
     return (uint32_t)(gemv > mrg ? gemv : mrg);

@@ -115,6 +115,47 @@ __device__ __forceinline__ void gemv_record(uint4 q, uint2 dd, uint32_t bs, uint
     }
 }
 
+// One record's math for one warp at M = 1 in the persistent step: each
+// block's two chained MMAs start from the block's offset constant instead of
+// zero, so they return the block's dot product in scaled units; the two
+// blocks' d weight them, and the chunk's inverse activation scale (one value
+// for both blocks, the activations being scaled per 128 columns) multiplies
+// their sum.  At M = 1 each block keeps (constant, 1/scale, constant,
+// 1/scale) in shared memory: one 16-byte load is the MMA's accumulator input
+// as it stands (elements 0 and 2, rows g and g + 8 of token 0, start from the
+// constant; 1 and 3 belong to the unused token columns).  bsb: this lane's
+// B-fragment words of the chunk's first block (the second block's are 64
+// bytes on); cbc: the chunk's two constant quads.  p0 += row g, p2 += row g + 8.
+__device__ __forceinline__ void gemv_record_m1(uint4 q, uint2 dd, uint32_t bsb, uint32_t cbc, float& p0, float& p2)
+{
+    const uint32_t M_P = 0x000F000Fu, M_Q = 0x00F000F0u, C_P = 0x64006400u, C_Q = 0x54005400u;
+    const float2 d0 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+    const float2 d1 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+    float c[2][4];
+    float inv = 0.f;
+#pragma unroll
+    for (int bb = 0; bb < 2; ++bb) {
+        const float4 k4 = lds128f(cbc + 16u * bb);
+        const uint4 B = lds128(bsb + 64u * bb);
+        const uint32_t w0 = bb ? q.z : q.x;
+        const uint32_t w1 = bb ? q.w : q.y;
+        const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
+        const uint32_t alo[4] = {lop3_and_or(w0, M_P, C_P), lop3_and_or(w0s, M_P, C_P),
+                                 lop3_and_or(w1, M_P, C_P), lop3_and_or(w1s, M_P, C_P)};
+        const uint32_t ahi[4] = {lop3_and_or(w0, M_Q, C_Q), lop3_and_or(w0s, M_Q, C_Q),
+                                 lop3_and_or(w1, M_Q, C_Q), lop3_and_or(w1s, M_Q, C_Q)};
+        const float kin[4] = {k4.x, k4.y, k4.z, k4.w};
+        float cc[4];
+        mma_f16_16816(cc, alo, B.x, B.y, kin);
+        mma_f16_16816(cc, ahi, B.z, B.w, cc);
+        c[bb][0] = cc[0];
+        c[bb][2] = cc[2];
+        inv = k4.y;
+    }
+    p0 = fmaf(inv, fmaf(d1.x, c[1][0], d0.x * c[0][0]), p0);
+    p2 = fmaf(inv, fmaf(d1.y, c[1][2], d0.y * c[0][2]), p2);
+}
+
 // Rotary embedding: (cos, sin) of the angle pos * theta^(-2i/hd) of pair
 // i = col / 2.  The angle is reduced to turns in double precision, so long
 // positions keep it accurate; the sine and cosine of the reduced angle are
