@@ -36,8 +36,8 @@
 //    depend on timing.  The phase's input vector is scaled by one power of
 //    two per 128 columns (the columns one warp converts) into [2^13, 2^14)
 //    before the fp16 conversion; a record's block MMAs start from the
-//    block's offset constant (`gemv_record_m1`), and a full stage with no
-//    tile end runs its records in groups of four with constant offsets.
+//    block's offset constant (`gemv_record_m1`), and the records of a stage
+//    run in groups of four up to each tile end.
 //  * ATTN phases: 16-slot units (kv head, slots) are split evenly over CTAs;
 //    inside a CTA the warps take units round robin, each unit two stages
 //    (its K rows, then its V rows) of two 2-D TMA boxes each (64 columns x
@@ -586,7 +586,10 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
         return row < f.n ? __ldcg(res_src + row) : 0.f;
     };
 
-    // ---- main loop: this warp's records, two at a time
+    // ---- main loop: this warp's records.  A stage is cut at tile ends; each
+    // run of records inside one tile goes in groups of four (their MMAs in
+    // flight together, chunk addresses as constant offsets) straight into the
+    // tile's sums, and the tile is closed once, at its end or the range end.
     if (we > wb && ok) {
         int64_t tile = wb / kc;
         int cin = (int)(wb - tile * kc);
@@ -601,63 +604,38 @@ __device__ __forceinline__ void ps_gemv_phase(const PsArgs& P, const PsWs& W, co
             }
             const uint32_t base = smem_addr(ring.base) + (ring.consumed % kPsStages) * kPsStageBytes + smem_token();
             const int nrec = (int)min64(kPsRecs, we - r);
-            if (nrec == kPsRecs && cin + kPsRecs < kc && r + kPsRecs < we) {
-                // a full stage with no tile end and no range end: chunks cin .. cin + 6,
-                // all records' MMAs in flight together, added straight into the tile's sums
+            for (int u = 0; u < nrec;) {
+                const int run = nrec - u < kc - cin ? nrec - u : kc - cin;     // records up to the tile end
+                const uint32_t rec_a = base + (uint32_t)u * kChunkBytes;
                 const uint32_t bsb = bs_a + 128u * (uint32_t)cin + 16u * (uint32_t)t;
                 const uint32_t cbc = cb_a + 32u * (uint32_t)cin;
 #pragma unroll 1
-                for (int u0 = 0; u0 < kPsRecs; u0 += 4) {
+                for (int v0 = 0; v0 < run; v0 += 4) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        if (u0 + u >= kPsRecs) break;
-                        const uint32_t o = (uint32_t)(u0 + u);
-                        const uint4 qv = lds128(base + o * kChunkBytes + 16 * lane);
-                        const uint2 e = lds64(base + o * kChunkBytes + kChunkQsBytes + 8 * g);
+                    for (int v = 0; v < 4; ++v) {
+                        if (v0 + v >= run) break;
+                        const uint32_t o = (uint32_t)(v0 + v);
+                        const uint4 qv = lds128(rec_a + o * kChunkBytes + 16 * lane);
+                        const uint2 e = lds64(rec_a + o * kChunkBytes + kChunkQsBytes + 8 * g);
                         gemv_record_m1(qv, e, bsb + 128u * o, cbc + 32u * o, acc0, acc2);
                     }
                 }
-                cin += kPsRecs;
-                r += kPsRecs;
-                __syncwarp();
-                ++ring.consumed;
-                ps_ring_fill(P, ring, nph, b, G, warp, lane, nch, ph);
-                continue;
-            }
-            for (int q0 = 0; q0 < nrec; q0 += 2) {
-                // two records' MMAs back to back (a missing second record repeats
-                // the first; its result is not used), then their bookkeeping
-                float p[2][4];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int ri = q0 + u < nrec ? q0 + u : q0;
-                    const int ch = cin + u < kc ? cin + u : cin + u - kc;
-                    const uint4 qv = lds128(base + ri * kChunkBytes + 16 * lane);
-                    const uint2 e = lds64(base + ri * kChunkBytes + kChunkQsBytes + 8 * g);
-                    p[u][0] = p[u][1] = p[u][2] = p[u][3] = 0.f;
-                    gemv_record_m1(qv, e, bs_a + 128u * (uint32_t)ch + 16u * (uint32_t)t, cb_a + 32u * (uint32_t)ch,
-                                   p[u][0], p[u][2]);
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    if (q0 + u >= nrec) break;
-                    acc0 += p[u][0];
-                    acc2 += p[u][2];
-                    ++r;
-                    if (++cin == kc || r == we) {
-                        if (whole && cin == kc) {
-                            ps_epilogue(P, f, tile, acc0, acc2, rr, pos, best, res_of(tile, 0), res_of(tile, 1));
-                        } else if (t == 0) {
-                            // a piece of a tile shared with other warps: slot 0 is the warp's first tile
-                            const int slot = (tile == wb / kc) ? 0 : 1;
-                            s_piece[(warp * 2 + slot) * 16 + g] = acc0;
-                            s_piece[(warp * 2 + slot) * 16 + g + 8] = acc2;
-                        }
-                        acc0 = acc2 = 0.f;
-                        cin = 0;
-                        ++tile;
-                        whole = true;
+                u += run;
+                r += run;
+                cin += run;
+                if (cin == kc || r == we) {
+                    if (whole && cin == kc) {
+                        ps_epilogue(P, f, tile, acc0, acc2, rr, pos, best, res_of(tile, 0), res_of(tile, 1));
+                    } else if (t == 0) {
+                        // a piece of a tile shared with other warps: slot 0 is the warp's first tile
+                        const int slot = (tile == wb / kc) ? 0 : 1;
+                        s_piece[(warp * 2 + slot) * 16 + g] = acc0;
+                        s_piece[(warp * 2 + slot) * 16 + g + 8] = acc2;
                     }
+                    acc0 = acc2 = 0.f;
+                    cin = 0;
+                    ++tile;
+                    whole = true;
                 }
             }
             __syncwarp();
