@@ -112,10 +112,12 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b)
 
 __device__ __forceinline__ float gelu_erf_g(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
 
-// The epilogue of one output element: residual add or GELU, fp32 or bf16 store.
-__device__ __forceinline__ void gemm_store(const GemmArgs& a, int64_t mi, int64_t row, float o)
+// The epilogue of one output element: residual add (the residual value `res`
+// loaded by the caller, ahead of the sums; 0 unless op is VOX_EP_RESIDUAL) or
+// GELU, then an fp32 or bf16 store.
+__device__ __forceinline__ void gemm_store_pre(const GemmArgs& a, int64_t mi, int64_t row, float o, float res)
 {
-    if (a.op == VOX_EP_RESIDUAL) o += a.res[mi * a.ldr + row];
+    if (a.op == VOX_EP_RESIDUAL) o += res;
     else if (a.op == VOX_EP_GELU) o = gelu_erf_g(o);
     if (a.y_bf16)
         static_cast<uint16_t*>(a.y)[mi * a.ldy + row] = f32_to_bf16_bits(o);
@@ -138,10 +140,12 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank)
 
 // Distributed-shared-memory load; issued without a memory clobber so that
 // several can be in flight before their values are summed.
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr)
+// 16 bytes of another CTA's shared memory in the cluster (address from mapa).
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr)
 {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr));
     return v;
 }
 
@@ -293,11 +297,17 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
 #pragma unroll
                 for (int j = 0; j < 8; ++j) part[(c0 + cc + j) * kGemmRows + r] = v[j];
             } else if (row < a.n) {
+                float rv[8];                         // residuals of the 8 tokens, loaded together
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int64_t mi = m0 + c0 + cc + j;
+                    rv[j] = (a.op == VOX_EP_RESIDUAL && mi < a.m) ? a.res[mi * a.ldr + row] : 0.f;
+                }
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int64_t mi = m0 + c0 + cc + j;
                     if (mi >= a.m) break;
-                    gemm_store(a, mi, row, v[j]);
+                    gemm_store_pre(a, mi, row, v[j], rv[j]);
                 }
             }
         }
@@ -318,28 +328,50 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
 #pragma unroll
         for (int s2 = 0; s2 < 8; ++s2) rb[s2] = cluster_map(pl, (uint32_t)(s2 < S ? s2 : 0));
         const int cb = (int)(rank * BN / S), ce = (int)((rank + 1) * BN / S);
-        const int nel = (ce - cb) * kGemmRows;
-        // four elements per thread per round, all their loads in flight before the sums
-        for (int e0 = tid; e0 < nel; e0 += 4 * kGemmThreads) {
-            float v[4][8];
+        // groups of 4 consecutive rows of one token (16 bytes of every rank's
+        // partial tile), two groups per thread per round: all their loads (the
+        // ranks' partials and the residuals) in flight before the sums
+        const int nq = (ce - cb) * (kGemmRows / 4);
+        for (int q0 = tid; q0 < nq; q0 += 2 * kGemmThreads) {
+            float4 v[2][8];
+            float rv[2][4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * kGemmThreads;
-                const uint32_t off = e < nel ? (uint32_t)((cb + e / kGemmRows) * kGemmRows + e % kGemmRows) * 4u : 0u;
+            for (int u = 0; u < 2; ++u) {
+                const int qd = q0 + u * kGemmThreads;
+                const int c = cb + qd / (kGemmRows / 4), r4 = 4 * (qd % (kGemmRows / 4));
+                const uint32_t off = qd < nq ? (uint32_t)(c * kGemmRows + r4) * 4u : 0u;
 #pragma unroll
-                for (int s2 = 0; s2 < 8; ++s2) v[u][s2] = (s2 < S && e < nel) ? ld_cluster_f32(rb[s2] + off) : 0.f;
+                for (int s2 = 0; s2 < 8; ++s2)
+                    v[u][s2] = (s2 < S && qd < nq) ? ld_cluster_f32x4(rb[s2] + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const int64_t mi = m0 + c;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int64_t row = group * kGemmRows + r4 + e;
+                    rv[u][e] = (a.op == VOX_EP_RESIDUAL && qd < nq && row < a.n && mi < a.m) ? a.res[mi * a.ldr + row]
+                                                                                             : 0.f;
+                }
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * kGemmThreads;
-                if (e >= nel) break;
-                float o = v[u][0];
+            for (int u = 0; u < 2; ++u) {
+                const int qd = q0 + u * kGemmThreads;
+                if (qd >= nq) break;
+                float4 o = v[u][0];
 #pragma unroll
                 for (int s2 = 1; s2 < 8; ++s2)
-                    if (s2 < S) o += v[u][s2];
-                const int c = cb + e / kGemmRows, rr = e % kGemmRows;
-                const int64_t row = group * kGemmRows + rr, mi = m0 + c;
-                if (row < a.n && mi < a.m) gemm_store(a, mi, row, o);
+                    if (s2 < S) {
+                        o.x += v[u][s2].x;
+                        o.y += v[u][s2].y;
+                        o.z += v[u][s2].z;
+                        o.w += v[u][s2].w;
+                    }
+                const int c = cb + qd / (kGemmRows / 4), r4 = 4 * (qd % (kGemmRows / 4));
+                const int64_t mi = m0 + c;
+                const float ov[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int64_t row = group * kGemmRows + r4 + e;
+                    if (row < a.n && mi < a.m) gemm_store_pre(a, mi, row, ov[e], rv[u][e]);
+                }
             }
         }
         cluster_sync_all();
