@@ -413,11 +413,10 @@ static vox_status launch_gemm_bn(const GemmArgs& a, const void* x, int64_t ldx, 
 // once (the occupancy query accounts for how the SMs fall into GPCs), cached
 // per device; 0 if the query fails.
 template <int BN>
-static int gemm_max_clusters(int splits)
+static int gemm_max_clusters(int dev, int splits)
 {
     static std::atomic<int> cache[64][9];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || splits < 1 || splits > 8) return 0;
+    if (dev < 0 || dev >= 64 || splits < 1 || splits > 8) return 0;
     int v = cache[dev][splits].load(std::memory_order_relaxed);
     if (v) return v - 1;
     using C = GemmCfg<BN>;
@@ -444,13 +443,13 @@ static int gemm_max_clusters(int splits)
     return n;
 }
 
-static int max_clusters(int bn, int splits)
+static int max_clusters(int dev, int bn, int splits)
 {
     switch (bn) {
-    case 32: return gemm_max_clusters<32>(splits);
-    case 64: return gemm_max_clusters<64>(splits);
-    case 128: return gemm_max_clusters<128>(splits);
-    default: return gemm_max_clusters<256>(splits);
+    case 32: return gemm_max_clusters<32>(dev, splits);
+    case 64: return gemm_max_clusters<64>(dev, splits);
+    case 128: return gemm_max_clusters<128>(dev, splits);
+    default: return gemm_max_clusters<256>(dev, splits);
     }
 }
 
@@ -466,6 +465,8 @@ static void pick_tile(int64_t tiles, int64_t m, int kc, int& bn_out, int& splits
 {
     const int64_t groups = ceil_div(tiles, 8);
     const int64_t sms = device_sm_count();
+    int dev = -1;                                             // looked up once: the capacity cache is per device
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
     const char* ebn = getenv("VOX_GEMM_BN");
     const char* esp = getenv("VOX_GEMM_SPLITS");
     const int fbn = ebn ? atoi(ebn) : 0, fsp = esp ? atoi(esp) : 0;
@@ -474,20 +475,25 @@ static void pick_tile(int64_t tiles, int64_t m, int kc, int& bn_out, int& splits
     for (int bn = 256; bn >= 32; bn >>= 1) {
         if (fbn && bn != fbn) continue;
         if (!fbn && bn > 32 && (bn >> 1) >= m) continue;    // a smaller tile already covers every row
-        const double t_chunk = bn == 256 ? 0.9 : bn >= 64 ? 0.6 : 0.54;
-        const double fixed = bn == 256 ? 12.0 : 6.0;
+        // measured on B200 (one wave): a K chunk costs about 0.53 us whatever the
+        // tile width (its 128 x 64 weights are dequantised once per CTA), and a
+        // CTA's fixed cost grows with the tile (accumulator read-out, epilogue)
+        const double t_chunk = 0.53;
+        const double fixed = bn == 256 ? 8.5 : bn == 128 ? 6.0 : bn == 64 ? 4.3 : 3.5;
         for (int sp = 1; sp <= 8; ++sp) {
             if (fsp && sp != fsp) continue;
             if (sp > 1 && kc / sp < 2) break;
             const int64_t clusters = groups * ceil_div(m, bn);
             int64_t waves = ceil_div(clusters * sp, sms);
             if (sp > 1) {
-                const int mc = max_clusters(bn, sp);
+                const int mc = max_clusters(dev, bn, sp);
                 if (mc < 1) continue;
                 waves = ceil_div(clusters, mc);
                 if (!fsp && waves > 1) continue;
             }
-            const double cost = (double)waves * ((double)ceil_div(kc, sp) * t_chunk + fixed + (sp > 1 ? 2.0 : 0.0));
+            // the cluster reduction: each rank sums bn / sp tokens x 128 rows over the ranks
+            const double reduce = sp > 1 ? 0.5 + 0.23e-3 * (double)(bn * kGemmRows / sp) : 0.0;
+            const double cost = (double)waves * ((double)ceil_div(kc, sp) * t_chunk + fixed + reduce);
             if (cost < best_cost) {
                 best_cost = cost;
                 best_bn = bn;
