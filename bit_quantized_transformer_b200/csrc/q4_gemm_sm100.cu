@@ -16,9 +16,14 @@
 //               issues tcgen05.mma kind::f16 (M=128, N=BN, K=16, bf16 in, fp32
 //               accumulate) on shared-memory descriptors, committing each
 //               stage back to the producer;
-//   warps 2-9   dequantise: warp w takes the record of row tile w, lane
+//   warps 2-9   dequantise: warp w takes the record of row tile w - 2, lane
 //               (g, t) its 16 bytes of codes (rows g and g+8, both 32-column
-//               blocks); each 32-bit word gives four bf16 pairs 128 + q by
+//               blocks); VOX_GEMM_DQ_WARPS=16 builds two warps per record, one
+//               block each (measured slower: per chunk about 600 cycles of
+//               conversion and stores, 400 of waiting for the stage and 90 for
+//               the proxy fence, and more warps do not shorten it; the chunk's
+//               shared-memory traffic, A written then read by the MMA next to
+//               the X tile, is the likely bound).  Each 32-bit word gives four bf16 pairs 128 + q by
 //               OR-ing the nibble into the fraction of 128.0 (exact), then
 //               an exact subtraction of 136 gives q - 8, which is widened to
 //               fp32 and multiplied by d in fp32 (exact: 4 x 11 significant
@@ -33,7 +38,14 @@
 
 namespace vox {
 
-constexpr int kGemmThreads = 320;
+#ifndef VOX_GEMM_DQ_WARPS
+#define VOX_GEMM_DQ_WARPS 8
+#endif
+constexpr int kGemmDqWarps = VOX_GEMM_DQ_WARPS;     // dequantising (and epilogue) warps: 8 or 16
+static_assert(kGemmDqWarps == 8 || kGemmDqWarps == 16, "8 or 16 dequantising warps");
+constexpr int kGemmThreads = 32 * (2 + kGemmDqWarps);
+constexpr int kGemmRecWarps = kGemmDqWarps / 8;     // warps per 16-row record (each takes 2 / this blocks)
+constexpr int kGemmEpiParts = kGemmDqWarps / 4;     // accumulator column parts per tensor-memory lane quarter
 constexpr int kGemmRows = 128;                      // MMA M (weight rows per CTA)
 constexpr int kGemmRawBytes = 8 * kChunkBytes;      // 4608
 constexpr int kGemmABytes = kGemmRows * 128;        // 16 KB bf16 tile, 64 columns
@@ -177,7 +189,7 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     if (tid == 0) {
         for (int s = 0; s < C::stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&aready[s], 8);
+            mbar_init(&aready[s], kGemmDqWarps);
             mbar_init(&empty[s], 1);
         }
         mbar_init(&accb[0], 1);
@@ -237,28 +249,30 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         }
     } else {
         // ------------------------------------------------- dequant + epilogue
-        const int dw = warp - 2;                    // 0..7: the row tile this warp dequantises
+        const int dw = warp - 2;                    // 0 .. kGemmDqWarps-1
+        const int rt = dw / kGemmRecWarps;          // the row tile (record) this warp dequantises
         const int q = warp & 3;                     // tensor-memory lane quarter of this warp
         const int r = 32 * q + lane;                // weight row of the epilogue
         const int g = lane >> 2, t = lane & 3;
         const uint32_t M_L = 0x000F000Fu, C_B = 0x43004300u, B136 = 0x43084308u;   // 128.0, 136.0 (bf16x2)
-        const uint32_t row_g = (uint32_t)(dw * 16 + g), row_g8 = row_g + 8u;
+        const uint32_t row_g = (uint32_t)(rt * 16 + g), row_g8 = row_g + 8u;
         for (int i = 0; i < nk; ++i) {
             const int s = i % C::stages;
             const uint32_t ph = (uint32_t)((i / C::stages) & 1);
             if (!s_fail[0] && !mbar_wait_bounded(&full[s], ph, 0x303)) s_fail[0] = 1;
             uint8_t* st = smem + s * C::stage;
             uint8_t* A = st + C::xbytes;
-            if (dw * 16 < (int)(a.n - group * kGemmRows)) {
-                const uint8_t* rec = st + C::xbytes + kGemmABytes + dw * kChunkBytes;
+            if (rt * 16 < (int)(a.n - group * kGemmRows)) {
+                const uint8_t* rec = st + C::xbytes + kGemmABytes + rt * kChunkBytes;
                 const uint4 qv = *reinterpret_cast<const uint4*>(rec + 16 * lane);
                 const uint2 dd = *reinterpret_cast<const uint2*>(rec + kChunkQsBytes + 8 * g);
                 // scales in fp32 (exact): d(row g, block 0), d(row g+8, block 0), d(g, 1), d(g+8, 1)
                 const float2 d0 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
                 const float2 d1 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
-                const float D[4] = {d0.x, d0.y, d1.x, d1.y};
+
 #pragma unroll
                 for (int bb = 0; bb < 2; ++bb) {
+                    if (kGemmRecWarps == 2 && bb != (dw & 1)) continue;    // two warps share a record: one block each
 #pragma unroll
                     for (int wi = 0; wi < 2; ++wi) {
                         const uint32_t w = wi ? (bb ? qv.w : qv.y) : (bb ? qv.z : qv.x);
@@ -268,7 +282,7 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
                         for (int h = 0; h < 4; ++h) {
                             const uint32_t raw = lop3_and_or(src[h], M_L, C_B);            // 128 + q, exact
                             const uint32_t qm = bf16x2_sub(raw, B136);          // q - 8, exact
-                            const float dd_ = D[bb * 2 + (h & 1)];
+                            const float dd_ = (h & 1) ? (bb ? d1.y : d0.y) : (bb ? d1.x : d0.x);
                             const uint32_t v = pack_bf16x2(__uint_as_float(qm << 16) * dd_,
                                                            __uint_as_float(qm & 0xFFFF0000u) * dd_);
                             const uint32_t row = (h & 1) ? row_g8 : row_g;
@@ -287,10 +301,10 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         if (!s_fail[0] && !mbar_wait_bounded(&accb[0], 0, 0x304)) s_fail[0] = 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const int64_t row = group * kGemmRows + r;
-        const int c0 = (dw >> 2) * (BN / 2);
+        const int c0 = (dw >> 2) * (BN / kGemmEpiParts);   // this warp's accumulator columns
         // split K: the partial tile goes to the idle ring as [token][row] fp32
         float* part = reinterpret_cast<float*>(smem);
-        for (int cc = 0; cc < BN / 2; cc += 8) {
+        for (int cc = 0; cc < BN / kGemmEpiParts; cc += 8) {
             float v[8];
             tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c0 + cc), v);
             if constexpr (SPLIT) {
@@ -329,14 +343,15 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         for (int s2 = 0; s2 < 8; ++s2) rb[s2] = cluster_map(pl, (uint32_t)(s2 < S ? s2 : 0));
         const int cb = (int)(rank * BN / S), ce = (int)((rank + 1) * BN / S);
         // groups of 4 consecutive rows of one token (16 bytes of every rank's
-        // partial tile), two groups per thread per round: all their loads (the
+        // partial tile), QPT groups per thread per round: all their loads (the
         // ranks' partials and the residuals) in flight before the sums
         const int nq = (ce - cb) * (kGemmRows / 4);
-        for (int q0 = tid; q0 < nq; q0 += 2 * kGemmThreads) {
-            float4 v[2][8];
-            float rv[2][4];
+        constexpr int QPT = kGemmThreads >= 512 ? 1 : 2;          // groups per thread per round
+        for (int q0 = tid; q0 < nq; q0 += QPT * kGemmThreads) {
+            float4 v[QPT][8];
+            float rv[QPT][4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < QPT; ++u) {
                 const int qd = q0 + u * kGemmThreads;
                 const int c = cb + qd / (kGemmRows / 4), r4 = 4 * (qd % (kGemmRows / 4));
                 const uint32_t off = qd < nq ? (uint32_t)(c * kGemmRows + r4) * 4u : 0u;
@@ -352,7 +367,7 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < QPT; ++u) {
                 const int qd = q0 + u * kGemmThreads;
                 if (qd >= nq) break;
                 float4 o = v[u][0];
