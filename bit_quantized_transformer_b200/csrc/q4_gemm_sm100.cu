@@ -16,7 +16,14 @@
 //               issues tcgen05.mma kind::f16 (M=128, N=BN, K=16, bf16 in, fp32
 //               accumulate) on shared-memory descriptors, committing each
 //               stage back to the producer;
-//   warps 2-9   dequantise: warp w takes the record of row tile w - 2, lane
+//   warps 2-9   dequantise into tensor memory (VOX_GEMM_A_TMEM, the
+//               default): warp w converts block (w - 2) >> 2 of the rows of its
+//               lane quarter (w & 3), one row per lane, gathering the row's
+//               codes from the 4 lanes' slots of its record, and writes the
+//               bf16 pairs with tcgen05.st into the stage's 32 columns after
+//               the accumulator; the MMA then reads A from tensor memory.
+//               With VOX_GEMM_A_TMEM=0 the tile goes to shared memory instead:
+//               warp w takes the record of row tile w - 2, lane
 //               (g, t) its 16 bytes of codes (rows g and g+8, both 32-column
 //               blocks); VOX_GEMM_DQ_WARPS=16 builds two warps per record, one
 //               block each (measured slower: per chunk about 600 cycles of
@@ -44,11 +51,17 @@ namespace vox {
 constexpr int kGemmDqWarps = VOX_GEMM_DQ_WARPS;     // dequantising (and epilogue) warps: 8 or 16
 static_assert(kGemmDqWarps == 8 || kGemmDqWarps == 16, "8 or 16 dequantising warps");
 constexpr int kGemmThreads = 32 * (2 + kGemmDqWarps);
-constexpr int kGemmRecWarps = kGemmDqWarps / 8;     // warps per 16-row record (each takes 2 / this blocks)
+[[maybe_unused]] constexpr int kGemmRecWarps = kGemmDqWarps / 8;   // warps per 16-row record (shared-memory tile)
 constexpr int kGemmEpiParts = kGemmDqWarps / 4;     // accumulator column parts per tensor-memory lane quarter
+#ifndef VOX_GEMM_A_TMEM
+#define VOX_GEMM_A_TMEM 1
+#endif
+constexpr bool kATmem = VOX_GEMM_A_TMEM != 0;       // dequantised tile in tensor memory (else shared memory)
+static_assert(!kATmem || kGemmDqWarps == 8, "the tensor-memory tile is written by 8 warps (2 per lane quarter)");
 constexpr int kGemmRows = 128;                      // MMA M (weight rows per CTA)
 constexpr int kGemmRawBytes = 8 * kChunkBytes;      // 4608
-constexpr int kGemmABytes = kGemmRows * 128;        // 16 KB bf16 tile, 64 columns
+constexpr int kGemmABytes = kATmem ? 0 : kGemmRows * 128;   // the 16 KB bf16 tile of 64 columns, if in shared memory
+constexpr int kGemmACols = 32;                      // tensor-memory columns of one stage's tile (64 bf16 per row)
 
 struct GemmArgs {
     const uint8_t* w;
@@ -71,7 +84,11 @@ struct GemmCfg {
     static constexpr int stages = (200 * 1024 / stage) > 6 ? 6 : (200 * 1024 / stage);
     static constexpr int bars = stages * stage;
     static constexpr int smem = bars + (3 * stages + 2) * 8 + 16 + 1024;
-    static constexpr int tmem_cols = BN < 32 ? 32 : BN;
+    // accumulator columns [0, BN), then (A in tensor memory) 32 columns per stage; a power of two
+    static constexpr int tmem_need = (BN < 32 ? 32 : BN) + (kATmem ? stages * kGemmACols : 0);
+    static constexpr int tmem_cols = tmem_need <= 32 ? 32 : tmem_need <= 64 ? 64 : tmem_need <= 128 ? 128
+                                   : tmem_need <= 256 ? 256 : 512;
+    static_assert(tmem_need <= 512, "tensor memory holds 512 columns");
 };
 
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr)
@@ -95,6 +112,28 @@ __device__ __forceinline__ void umma_bf16(uint32_t dtmem, uint64_t adesc, uint64
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(dtmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// The same MMA with A (M x 16, rows on lanes, K pairs along columns) read from tensor memory.
+__device__ __forceinline__ void umma_bf16_ta(uint32_t dtmem, uint32_t atmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(dtmem), "r"(atmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// 16 consecutive 32-bit tensor-memory columns of this warp's 32 lanes (one
+// value per lane and column), then wait for the stores.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+                   "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+                 : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar)
@@ -238,11 +277,18 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
                 if (s_fail[0]) break;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 const uint32_t xs = smem_addr(smem + s * C::stage);
-                const uint32_t as = xs + C::xbytes;
+                if constexpr (kATmem) {
+                    const uint32_t at = tmem + (uint32_t)(BN < 32 ? 32 : BN) + (uint32_t)(s * kGemmACols);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16(tmem, umma_desc_sw128(as + kk * 32), umma_desc_sw128(xs + kk * 32), idesc,
-                              (i > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16_ta(tmem, at + 8u * kk, umma_desc_sw128(xs + kk * 32), idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                } else {
+                    const uint32_t as = xs + C::xbytes;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem, umma_desc_sw128(as + kk * 32), umma_desc_sw128(xs + kk * 32), idesc,
+                                  (i > 0 || kk > 0) ? 1u : 0u);
+                }
                 umma_commit(&empty[s]);
             }
             umma_commit(&accb[0]);
@@ -250,52 +296,93 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     } else {
         // ------------------------------------------------- dequant + epilogue
         const int dw = warp - 2;                    // 0 .. kGemmDqWarps-1
-        const int rt = dw / kGemmRecWarps;          // the row tile (record) this warp dequantises
         const int q = warp & 3;                     // tensor-memory lane quarter of this warp
         const int r = 32 * q + lane;                // weight row of the epilogue
-        const int g = lane >> 2, t = lane & 3;
         const uint32_t M_L = 0x000F000Fu, C_B = 0x43004300u, B136 = 0x43084308u;   // 128.0, 136.0 (bf16x2)
-        const uint32_t row_g = (uint32_t)(rt * 16 + g), row_g8 = row_g + 8u;
-        for (int i = 0; i < nk; ++i) {
-            const int s = i % C::stages;
-            const uint32_t ph = (uint32_t)((i / C::stages) & 1);
-            if (!s_fail[0] && !mbar_wait_bounded(&full[s], ph, 0x303)) s_fail[0] = 1;
-            uint8_t* st = smem + s * C::stage;
-            uint8_t* A = st + C::xbytes;
-            if (rt * 16 < (int)(a.n - group * kGemmRows)) {
-                const uint8_t* rec = st + C::xbytes + kGemmABytes + rt * kChunkBytes;
-                const uint4 qv = *reinterpret_cast<const uint4*>(rec + 16 * lane);
-                const uint2 dd = *reinterpret_cast<const uint2*>(rec + kChunkQsBytes + 8 * g);
-                // scales in fp32 (exact): d(row g, block 0), d(row g+8, block 0), d(g, 1), d(g+8, 1)
-                const float2 d0 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
-                const float2 d1 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+        if constexpr (kATmem) {
+            // lane = weight row 32 q + lane (this warp's tensor-memory lanes); block
+            // dw >> 2 (32 columns = 16 tensor-memory columns) of every chunk.  The
+            // row's codes sit in the 4 lanes' slots (g, t = 0..3) of its record.
+            const int bbk = dw >> 2;
+            const int rrow = 32 * q + lane;
+            const int rtile = rrow >> 4, rg = rrow & 7, rhalf = (rrow >> 3) & 1;
+            const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(BN < 32 ? 32 : BN) + 16u * (uint32_t)bbk;
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % C::stages;
+                const uint32_t ph = (uint32_t)((i / C::stages) & 1);
+                if (!s_fail[0] && !mbar_wait_bounded(&full[s], ph, 0x303)) s_fail[0] = 1;
+                const uint8_t* rec = smem + s * C::stage + C::xbytes + rtile * kChunkBytes;
+                uint2 wv[4];
+#pragma unroll
+                for (int t4 = 0; t4 < 4; ++t4) wv[t4] = *reinterpret_cast<const uint2*>(rec + 16 * (4 * rg + t4) + 8 * bbk);
+                const uint32_t db = *reinterpret_cast<const uint32_t*>(rec + kChunkQsBytes + 8 * rg + 4 * bbk);
+                const float dsc = __half2float(__ushort_as_half((unsigned short)(rhalf ? db >> 16 : db & 0xFFFFu)));
+                uint32_t vals[16];
+#pragma unroll
+                for (int t4 = 0; t4 < 4; ++t4)
+#pragma unroll
+                    for (int wi = 0; wi < 2; ++wi)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t w = wi ? wv[t4].y : wv[t4].x;
+                            // this row's nibble pair of the word: row g (w, w >> 4), row g + 8 (w >> 8, w >> 12)
+                            const uint32_t src = rhalf ? (hh ? w >> 12 : w >> 8) : (hh ? w >> 4 : w);
+                            const uint32_t raw = lop3_and_or(src, M_L, C_B);          // 128 + q, exact
+                            const uint32_t qm = bf16x2_sub(raw, B136);                 // q - 8, exact
+                            // K pair 16 hh + 8 wi + 2 t4 of the block: column 8 hh + 4 wi + t4
+                            vals[8 * hh + 4 * wi + t4] =
+                                pack_bf16x2(__uint_as_float(qm << 16) * dsc, __uint_as_float(qm & 0xFFFF0000u) * dsc);
+                        }
+                tmem_st16(ta + (uint32_t)(s * kGemmACols), vals);
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&aready[s]);
+            }
+        } else {
+            const int rt = dw / kGemmRecWarps;      // the row tile (record) this warp dequantises
+            const int g = lane >> 2, t = lane & 3;
+            const uint32_t row_g = (uint32_t)(rt * 16 + g), row_g8 = row_g + 8u;
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % C::stages;
+                const uint32_t ph = (uint32_t)((i / C::stages) & 1);
+                if (!s_fail[0] && !mbar_wait_bounded(&full[s], ph, 0x303)) s_fail[0] = 1;
+                uint8_t* st = smem + s * C::stage;
+                uint8_t* A = st + C::xbytes;
+                if (rt * 16 < (int)(a.n - group * kGemmRows)) {
+                    const uint8_t* rec = st + C::xbytes + kGemmABytes + rt * kChunkBytes;
+                    const uint4 qv = *reinterpret_cast<const uint4*>(rec + 16 * lane);
+                    const uint2 dd = *reinterpret_cast<const uint2*>(rec + kChunkQsBytes + 8 * g);
+                    // scales in fp32 (exact): d(row g, block 0), d(row g+8, block 0), d(g, 1), d(g+8, 1)
+                    const float2 d0 = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+                    const float2 d1 = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
 
-#pragma unroll
-                for (int bb = 0; bb < 2; ++bb) {
-                    if (kGemmRecWarps == 2 && bb != (dw & 1)) continue;    // two warps share a record: one block each
-#pragma unroll
-                    for (int wi = 0; wi < 2; ++wi) {
-                        const uint32_t w = wi ? (bb ? qv.w : qv.y) : (bb ? qv.z : qv.x);
-                        // nibble pairs: (w, w>>8) low halves, (w>>4, w>>12) high halves; rows g, g+8
-                        const uint32_t src[4] = {w, w >> 8, w >> 4, w >> 12};
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const uint32_t raw = lop3_and_or(src[h], M_L, C_B);            // 128 + q, exact
-                            const uint32_t qm = bf16x2_sub(raw, B136);          // q - 8, exact
-                            const float dd_ = (h & 1) ? (bb ? d1.y : d0.y) : (bb ? d1.x : d0.x);
-                            const uint32_t v = pack_bf16x2(__uint_as_float(qm << 16) * dd_,
-                                                           __uint_as_float(qm & 0xFFFF0000u) * dd_);
-                            const uint32_t row = (h & 1) ? row_g8 : row_g;
-                            // columns 32 bb + 16 (h >> 1) + 8 wi + 2t, +1: unit 4 bb + 2 (h >> 1) + wi
-                            const uint32_t unit = (uint32_t)(bb * 4 + (h >> 1) * 2 + wi);
-                            *reinterpret_cast<uint32_t*>(A + sw128_offset(row, unit) + 4 * t) = v;
+    #pragma unroll
+                    for (int bb = 0; bb < 2; ++bb) {
+                        if (kGemmRecWarps == 2 && bb != (dw & 1)) continue;    // two warps share a record: one block each
+    #pragma unroll
+                        for (int wi = 0; wi < 2; ++wi) {
+                            const uint32_t w = wi ? (bb ? qv.w : qv.y) : (bb ? qv.z : qv.x);
+                            // nibble pairs: (w, w>>8) low halves, (w>>4, w>>12) high halves; rows g, g+8
+                            const uint32_t src[4] = {w, w >> 8, w >> 4, w >> 12};
+    #pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                const uint32_t raw = lop3_and_or(src[h], M_L, C_B);            // 128 + q, exact
+                                const uint32_t qm = bf16x2_sub(raw, B136);          // q - 8, exact
+                                const float dd_ = (h & 1) ? (bb ? d1.y : d0.y) : (bb ? d1.x : d0.x);
+                                const uint32_t v = pack_bf16x2(__uint_as_float(qm << 16) * dd_,
+                                                               __uint_as_float(qm & 0xFFFF0000u) * dd_);
+                                const uint32_t row = (h & 1) ? row_g8 : row_g;
+                                // columns 32 bb + 16 (h >> 1) + 8 wi + 2t, +1: unit 4 bb + 2 (h >> 1) + wi
+                                const uint32_t unit = (uint32_t)(bb * 4 + (h >> 1) * 2 + wi);
+                                *reinterpret_cast<uint32_t*>(A + sw128_offset(row, unit) + 4 * t) = v;
+                            }
                         }
                     }
                 }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&aready[s]);
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&aready[s]);
         }
         // ---- epilogue
         if (!s_fail[0] && !mbar_wait_bounded(&accb[0], 0, 0x304)) s_fail[0] = 1;
