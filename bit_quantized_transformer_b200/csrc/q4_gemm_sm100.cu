@@ -57,7 +57,9 @@ constexpr int kGemmEpiParts = kGemmDqWarps / 4;     // accumulator column parts 
 #define VOX_GEMM_A_TMEM 1
 #endif
 constexpr bool kATmem = VOX_GEMM_A_TMEM != 0;       // dequantised tile in tensor memory (else shared memory)
-static_assert(!kATmem || kGemmDqWarps == 8, "the tensor-memory tile is written by 8 warps (2 per lane quarter)");
+// with the tensor-memory tile, the dequantising warps form groups of 8 (2 per
+// lane quarter) that take alternate chunks
+constexpr int kGemmDqGroups = kATmem ? kGemmDqWarps / 8 : 1;
 constexpr int kGemmRows = 128;                      // MMA M (weight rows per CTA)
 constexpr int kGemmRawBytes = 8 * kChunkBytes;      // 4608
 constexpr int kGemmABytes = kATmem ? 0 : kGemmRows * 128;   // the 16 KB bf16 tile of 64 columns, if in shared memory
@@ -228,7 +230,7 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     if (tid == 0) {
         for (int s = 0; s < C::stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&aready[s], kGemmDqWarps);
+            mbar_init(&aready[s], kGemmDqWarps / kGemmDqGroups);
             mbar_init(&empty[s], 1);
         }
         mbar_init(&accb[0], 1);
@@ -303,11 +305,12 @@ q4_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
             // lane = weight row 32 q + lane (this warp's tensor-memory lanes); block
             // dw >> 2 (32 columns = 16 tensor-memory columns) of every chunk.  The
             // row's codes sit in the 4 lanes' slots (g, t = 0..3) of its record.
-            const int bbk = dw >> 2;
+            const int grp = dw >> 3;                // chunks grp, grp + groups, ...
+            const int bbk = (dw >> 2) & 1;
             const int rrow = 32 * q + lane;
             const int rtile = rrow >> 4, rg = rrow & 7, rhalf = (rrow >> 3) & 1;
             const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(BN < 32 ? 32 : BN) + 16u * (uint32_t)bbk;
-            for (int i = 0; i < nk; ++i) {
+            for (int i = grp; i < nk; i += kGemmDqGroups) {
                 const int s = i % C::stages;
                 const uint32_t ph = (uint32_t)((i / C::stages) & 1);
                 if (!s_fail[0] && !mbar_wait_bounded(&full[s], ph, 0x303)) s_fail[0] = 1;
