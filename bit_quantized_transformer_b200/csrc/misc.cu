@@ -123,18 +123,101 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, int64_t n, int64_t l
     }
 }
 
+// The same with 16-byte accesses: each thread keeps its VPT float4 of the
+// row in registers between the sum of squares and the scaling (one pass over
+// x), and stores 4 outputs at once.  Per element the arithmetic is that of
+// rmsnorm_kernel; the sum of squares is accumulated in another order, so the
+// two agree to rounding.
+template <int VPT>
+__global__ void rmsnorm_vec_kernel(const float* __restrict__ x, int64_t n4, int64_t ldx, float eps,
+                                   const float* __restrict__ g, void* __restrict__ out, int out_bf16, int64_t ldo,
+                                   int normalize)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    __shared__ float red[32];
+    const int64_t row = blockIdx.x;
+    const float4* xr = reinterpret_cast<const float4*>(x + row * ldx);
+    float4 v[VPT];
+    float ssq = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        const int64_t i = threadIdx.x + (int64_t)k * blockDim.x;
+        v[k] = i < n4 ? xr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        ssq = fmaf(v[k].x, v[k].x, ssq);
+        ssq = fmaf(v[k].y, v[k].y, ssq);
+        ssq = fmaf(v[k].z, v[k].z, ssq);
+        ssq = fmaf(v[k].w, v[k].w, ssq);
+    }
+    for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ssq;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float sum = 0.f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) sum += red[w];
+        red[0] = normalize ? 1.0f / sqrtf(sum / (float)(4 * n4) + eps) : 1.0f;
+    }
+    __syncthreads();
+    const float r = red[0];
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        const int64_t i = threadIdx.x + (int64_t)k * blockDim.x;
+        if (i >= n4) break;
+        float4 y = make_float4(v[k].x * r, v[k].y * r, v[k].z * r, v[k].w * r);
+        if (g) {
+            const float4 gv = reinterpret_cast<const float4*>(g)[i];
+            y = make_float4(y.x * gv.x, y.y * gv.y, y.z * gv.z, y.w * gv.w);
+        }
+        if (out_bf16) {
+            const uint2 pk = make_uint2((uint32_t)f32_to_bf16_bits(y.x) | ((uint32_t)f32_to_bf16_bits(y.y) << 16),
+                                        (uint32_t)f32_to_bf16_bits(y.z) | ((uint32_t)f32_to_bf16_bits(y.w) << 16));
+            reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + row * ldo)[i] = pk;
+        } else {
+            reinterpret_cast<float4*>(static_cast<float*>(out) + row * ldo)[i] = y;
+        }
+    }
+}
+
+// Rows of x -> out through the 16-byte kernel when the row length, strides
+// and pointers allow it, else through rmsnorm_kernel.
+static vox_status launch_rows(const float* x, int64_t m, int64_t n, int64_t ldx, float eps, const float* g, void* out,
+                              int out_bf16, int64_t ldo, int normalize, cudaStream_t s)
+{
+    auto al = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
+    const bool vec = n % 4 == 0 && ldx % 4 == 0 && ldo % 4 == 0 && al(x, 16) && (!g || al(g, 16)) &&
+                     al(out, out_bf16 ? 8 : 16) && n / 4 <= 8 * 1024;
+    if (!vec)
+        return launch_pdl(rmsnorm_kernel, dim3((unsigned)m), dim3(256), 0, s, x, n, ldx, eps, g, out, out_bf16, ldo,
+                          normalize);
+    const int64_t n4 = n / 4;
+    const int vpt = n4 <= 1024 ? 1 : n4 <= 2048 ? 2 : n4 <= 4096 ? 4 : 8;
+    const unsigned threads = (unsigned)((ceil_div(n4, vpt) + 31) / 32 * 32);
+    switch (vpt) {
+    case 1:
+        return launch_pdl(rmsnorm_vec_kernel<1>, dim3((unsigned)m), dim3(threads), 0, s, x, n4, ldx, eps, g, out,
+                          out_bf16, ldo, normalize);
+    case 2:
+        return launch_pdl(rmsnorm_vec_kernel<2>, dim3((unsigned)m), dim3(threads), 0, s, x, n4, ldx, eps, g, out,
+                          out_bf16, ldo, normalize);
+    case 4:
+        return launch_pdl(rmsnorm_vec_kernel<4>, dim3((unsigned)m), dim3(threads), 0, s, x, n4, ldx, eps, g, out,
+                          out_bf16, ldo, normalize);
+    default:
+        return launch_pdl(rmsnorm_vec_kernel<8>, dim3((unsigned)m), dim3(threads), 0, s, x, n4, ldx, eps, g, out,
+                          out_bf16, ldo, normalize);
+    }
+}
+
 vox_status launch_rmsnorm(const float* x, int64_t m, int64_t n, int64_t ldx, float eps, const float* g, void* out,
                           int out_dtype, int64_t ldo, cudaStream_t s)
 {
-    return launch_pdl(rmsnorm_kernel, dim3((unsigned)m), dim3(256), 0, s, x, n, ldx, eps, g, out,
-                      (int)(out_dtype == VOX_BF16), ldo, 1);
+    return launch_rows(x, m, n, ldx, eps, g, out, (int)(out_dtype == VOX_BF16), ldo, 1, s);
 }
 
 vox_status launch_cast_rows(const float* x, int64_t m, int64_t n, int64_t ldx, void* out, int out_dtype,
                             int64_t ldo, cudaStream_t s)
 {
-    return launch_pdl(rmsnorm_kernel, dim3((unsigned)m), dim3(256), 0, s, x, n, ldx, 0.0f,
-                      static_cast<const float*>(nullptr), out, (int)(out_dtype == VOX_BF16), ldo, 0);
+    return launch_rows(x, m, n, ldx, 0.0f, nullptr, out, (int)(out_dtype == VOX_BF16), ldo, 0, s);
 }
 
 // ------------------------------------------------------------ history roll

@@ -528,6 +528,24 @@ def test_rmsnorm(env):
     np.testing.assert_allclose(np_of(out), ref.rmsnorm(x), rtol=1e-5, atol=1e-6)
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("n", [1280, 3072, 5120, 1283])
+def test_rmsnorm_weight_bf16(env, n):
+    """RMSNorm with a weight into bf16 rows: the 16-byte path (n a multiple of
+    4, one or two float4 per thread) and the element path (n = 1283).  Each
+    value is within one bf16 rounding of the oracle's."""
+    torch, V, WL = env
+    m = 7
+    x = synth.activations(m, n, 0, 14002) * 3.0
+    g = synth.activations(1, n, 0, 14003)[0] + 1.5
+    out = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    V.vox_rmsnorm(WL.to_dev(x, "cuda"), m, n, n, 1e-5, WL.to_dev(g, "cuda"), out, V.VOX_BF16, n)
+    check_status(V)
+    want = ref.rmsnorm(x, g=g)
+    got = out.float().cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(got, want, rtol=2.0 ** -8, atol=1e-30)
+
+
 # ------------------------------------------------------------------- RoPE
 @pytest.mark.parametrize("pos,theta", [(0, 1e6), (7, 1e4), (8191, 1e6), (100000, 1e6), (123457, 500.0)])
 def test_gemv_kv_append_rope(env, pos, theta):
