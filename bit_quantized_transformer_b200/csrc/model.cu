@@ -251,8 +251,10 @@ size_t vox_decoder_batch_workspace(const vox_decoder_batch* b)
     if (!b || b->n_seq < 1 || b->n_seq > 8 || b->d.dim < 32 || b->d.vocab < 1 || b->d.n_kv_heads < 1 ||
         b->d.window < 1 || b->d.n_layers < 1 || b->d.n_q_heads < b->d.n_kv_heads)
         return 0;
+    const size_t QD = (size_t)b->d.n_q_heads * (size_t)b->d.head_dim, F = (size_t)b->d.ffn;
     return batch_gemv_ws(b) +
-           ((attn_workspace_bytes(b->d.n_kv_heads, b->d.head_dim, b->d.window, b->n_seq) + 255) & ~(size_t)255);
+           ((attn_workspace_bytes(b->d.n_kv_heads, b->d.head_dim, b->d.window, b->n_seq) + 255) & ~(size_t)255) +
+           ((b->n_seq * QD * 2 + 255) & ~(size_t)255) + ((b->n_seq * F * 2 + 255) & ~(size_t)255);
 }
 
 vox_status vox_decoder_batch_step(const vox_decoder_batch* b, void* stream)
@@ -272,7 +274,16 @@ vox_status vox_decoder_batch_step(const vox_decoder_batch* b, void* stream)
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t* ws_g = static_cast<uint8_t*>(d->workspace);
     uint8_t* ws_a = ws_g + batch_gemv_ws(b);
+    // bf16 copies of the Wo and W2 inputs for the tcgen05 GEMM (after the attention workspace)
+    uint8_t* attn16 = ws_a + ((attn_workspace_bytes(d->n_kv_heads, d->head_dim, d->window, (int)m) + 255) & ~(size_t)255);
+    uint8_t* act16 = attn16 + ((m * QD * 2 + 255) & ~(int64_t)255);
     const float scale = 1.0f / sqrtf((float)d->head_dim);
+    // Above 4 sequences the Wo and W2 projections (the long-K ones) run on the
+    // tcgen05 GEMM over bf16 copies of their inputs: there one GEMM beats the
+    // 8-row GEMV (about 11 against 19 us on 3072 x 4096, 19 against 32 on
+    // 3072 x 9216), the copy costing one short launch.
+    const char* e2 = getenv("VOX_BATCH_GEMM");
+    const bool gemm_wo_w2 = m > 4 && !(e2 && e2[0] == '0') && QD % 64 == 0 && F % 64 == 0;
 
     // x[i] = embedding row of sequence i's token (exact fp32 weights)
     if ((st = launch_q4_dequant(static_cast<const uint8_t*>(d->embedding.data), d->vocab, D, 0, d->token, m, d->x,
@@ -304,9 +315,15 @@ vox_status vox_decoder_batch_step(const vox_decoder_batch* b, void* stream)
         r.op = VOX_EP_RESIDUAL;
         r.residual = d->x;
         r.ldr = D;
-        if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->wo[l].data), D, QD, d->attn, m, QD, d->h, D, &r, ws_g,
-                                 s)))
+        if (gemm_wo_w2) {
+            if ((st = launch_cast_rows(d->attn, m, QD, QD, attn16, VOX_BF16, QD, s)) ||
+                (st = launch_q4_gemm(static_cast<const uint8_t*>(d->wo[l].data), D, QD, attn16, m, QD, d->h, VOX_F32,
+                                     D, &r, s)))
+                return st;
+        } else if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->wo[l].data), D, QD, d->attn, m, QD, d->h, D, &r,
+                                        ws_g, s))) {
             return st;
+        }
         vox_epilogue f = {};
         f.op = VOX_EP_SILU_MUL;
         f.rmsnorm = 1;
@@ -318,9 +335,15 @@ vox_status vox_decoder_batch_step(const vox_decoder_batch* b, void* stream)
         r2.op = VOX_EP_RESIDUAL;
         r2.residual = d->h;
         r2.ldr = D;
-        if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->w2[l].data), D, F, d->act, m, F, d->x, D, &r2, ws_g,
-                                 s)))
+        if (gemm_wo_w2) {
+            if ((st = launch_cast_rows(d->act, m, F, F, act16, VOX_BF16, F, s)) ||
+                (st = launch_q4_gemm(static_cast<const uint8_t*>(d->w2[l].data), D, F, act16, m, F, d->x, VOX_F32, D,
+                                     &r2, s)))
+                return st;
+        } else if ((st = launch_q4_gemv(static_cast<const uint8_t*>(d->w2[l].data), D, F, d->act, m, F, d->x, D, &r2,
+                                        ws_g, s))) {
             return st;
+        }
     }
     vox_epilogue am = {};
     am.op = VOX_EP_ARGMAX;

@@ -472,7 +472,10 @@ size_t vox_decoder_batch_workspace(const vox_decoder_batch *b);
 /* One greedy step of every sequence: the launches of vox_decoder_step_kernels
  * with m = n_seq rows (embedding rows gathered by token, the QKV epilogue
  * VOX_EP_KV_APPEND_PAGED, vox_gqa_decode_attn_paged, argmax per row, every
- * position advanced); the sequence can be captured in a CUDA graph.  Errors:
+ * position advanced); above 4 sequences the Wo and W2 projections run as the
+ * tcgen05 GEMM (vox_q4_gemm) on bf16 copies of their inputs, kept in the
+ * workspace (VOX_BATCH_GEMM=0 in the environment keeps the GEMV); the
+ * sequence can be captured in a CUDA graph.  Errors:
  * as vox_decoder_step_kernels; n_seq outside 1..8, window not a multiple of
  * 64 or n_pages < 1 -> VOX_ERR_RANGE; NULL page_table -> VOX_ERR_NULL. */
 vox_status vox_decoder_batch_step(const vox_decoder_batch *b, void *stream);
