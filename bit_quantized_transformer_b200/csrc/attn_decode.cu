@@ -467,8 +467,11 @@ __device__ __forceinline__ bool attn_cta_nonempty(int64_t bo, int64_t total, int
 
 __global__ void __launch_bounds__(32) attn_combine_kernel(const AttnArgs a, int64_t G)
 {
-    pdl_wait();
+    // The dependents (the Wo projection) may launch at once: this grid is
+    // small, so their first CTAs fit beside the attention kernel and start
+    // their weight copies; they still wait for this grid to complete.
     pdl_launch_dependents();
+    pdl_wait();
     const int group = a.group;
     const int kh = blockIdx.x / group, gi = blockIdx.x - kh * group, lane = threadIdx.x;
     const int W = a.window;

@@ -258,8 +258,10 @@ vox_status launch_hist_roll(const void* hist, int64_t ld_hist, const void* nw, i
 // --------------------------------------------------------- position advance
 __global__ void advance_pos_kernel(int64_t* pos, int n)
 {
-    pdl_wait();
+    // one CTA: the next kernels may launch at once and start their weight
+    // copies beside it; they still wait for this grid to complete
     pdl_launch_dependents();
+    pdl_wait();
     if ((int)threadIdx.x < n) pos[threadIdx.x] += 1;
 }
 

@@ -96,6 +96,10 @@ __global__ void q4_dequant_kernel(const uint8_t* __restrict__ packed, int64_t n,
                                   int64_t row0, const int32_t* __restrict__ row_dev, int64_t nrows,
                                   void* __restrict__ out, int dtype, int64_t ldo, int gather)
 {
+    // dependents may launch once every CTA has started (a one-row dequant is
+    // a few CTAs, so the next projection's CTAs start their weight copies
+    // beside it); they still wait for this grid to complete
+    pdl_launch_dependents();
     pdl_wait();
     int64_t nb = k / 32;
     int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
