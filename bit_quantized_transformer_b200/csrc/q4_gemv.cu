@@ -100,6 +100,9 @@ struct GemvSmem {
     uint32_t ring, bars, bs, cb, part, ptile, sq, best_v, best_i, total;
 };
 
+// Entries per block in the constant table: 1 at m = 1, else m rounded up to even.
+__host__ __device__ inline int gemv_cb_stride(int m) { return m == 1 ? 1 : (m + 1) & ~1; }
+
 __host__ __device__ inline GemvSmem gemv_smem_layout(int kc, int m, int stages)
 {
     GemvSmem L;
@@ -108,7 +111,9 @@ __host__ __device__ inline GemvSmem gemv_smem_layout(int kc, int m, int stages)
     L.bars = off;    off += (uint32_t)kGemvWarps * (uint32_t)stages * 8u;
     off = (off + 15u) & ~15u;
     L.bs = off;      off += (uint32_t)kc * (uint32_t)m * 128u;     // fp16 B fragments
-    L.cb = off;      off += (uint32_t)kc * (uint32_t)m * 16u;      // per (token, block): offset constant, 1/scale
+    // per (block, token), a block's tokens adjacent and padded to an even
+    // count (one 16-byte load covers tokens 2t, 2t + 1): offset constant, 1/scale
+    L.cb = off;      off += (uint32_t)kc * (uint32_t)gemv_cb_stride(m) * 16u;
     L.part = off;    off += kGemvWarps * 32 * 16;
     L.ptile = off;   off += kGemvWarps * 4;
     L.sq = off;      off += kGemvWarps * 8 * 4;
@@ -278,7 +283,7 @@ __device__ __noinline__ GemvBest gemv_epilogue(const GemvArgs& a, int64_t tile, 
 __device__ __forceinline__ void gemv_convert(const GemvArgs& a, const float* xr, int i, int f0, int nf, int nfp,
                                              int lane, uint32_t* s_bs32, float2* s_cb, float& sq)
 {
-    const int m = a.m, nblk = a.kc * 2;
+    const int m = a.m, cs = gemv_cb_stride(a.m);
     float4 v[kGemvBatch], gv[kGemvBatch];
 #pragma unroll
     for (int u = 0; u < kGemvBatch; ++u) {
@@ -318,7 +323,7 @@ __device__ __forceinline__ void gemv_convert(const GemvArgs& a, const float* xr,
             const int word = (blk * m + i) * 16 + 2 * (q & 1) * 4 + (q >> 2) * 2 + ((q & 3) >> 1);
             s_bs32[word] = *reinterpret_cast<const uint32_t*>(&h01);
             s_bs32[word + 4] = *reinterpret_cast<const uint32_t*>(&h23);
-            if (q == 0) s_cb[i * nblk + blk] = make_float2(-(1032.0f * s + 72.0f * shi), inv);
+            if (q == 0) s_cb[blk * cs + i] = make_float2(-(1032.0f * s + 72.0f * shi), inv);
         }
     }
 }
@@ -396,7 +401,7 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
     if (MT == 1 && t != 0) rr[0] = 0.f;      // token 2t of a lane with t > 0 does not exist at m = 1
 
     const int64_t pos = a.pos_dev ? *a.pos_dev : a.pos;
-    const int nblk = kc * 2;
+    const int cs = gemv_cb_stride(m);
     const uint32_t tk = smem_token();
     const uint32_t bs_a = smem_addr(s_bs32) + tk, cb_a = smem_addr(s_cb) + tk;
     const uint32_t ring_a = smem_addr(ring);
@@ -453,7 +458,7 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
                 const uint4 q = lds128(base + r * kChunkBytes + 16 * lane);
                 const uint2 e = lds64(base + r * kChunkBytes + kChunkQsBytes + 8 * g);
                 p[r][0] = p[r][1] = p[r][2] = p[r][3] = 0.f;
-                gemv_record<MT>(q, e, bs_a, cb_a, nblk, ch, m, tok, t, p[r]);
+                gemv_record<MT>(q, e, bs_a, cb_a, cs, ch, m, tok, t, p[r]);
                 ch = ch + 1 == kc ? 0 : ch + 1;
             }
             if (left > kGemvRecs && cin + kGemvRecs < kc) {

@@ -72,7 +72,7 @@ __device__ __forceinline__ float4 ld_f4(const float* p, int f, int vec)
 // block's offset constant and scaled by d / (activation scale) in fp32.
 // q, dd: this lane's code and scale words.  p[2h + e] += row g + 8h, token 2t + e.
 template <int MT>
-__device__ __forceinline__ void gemv_record(uint4 q, uint2 dd, uint32_t bs, uint32_t cb, int nblk, int chunk,
+__device__ __forceinline__ void gemv_record(uint4 q, uint2 dd, uint32_t bs, uint32_t cb, int cs, int chunk,
                                             int m, int tok, int t, float (&p)[4])
 {
     const uint32_t M_P = 0x000F000Fu, M_Q = 0x00F000F0u, C_P = 0x64006400u, C_Q = 0x54005400u;
@@ -91,9 +91,11 @@ __device__ __forceinline__ void gemv_record(uint4 q, uint2 dd, uint32_t bs, uint
             c0 = bb ? make_float2(cm.z, cm.w) : make_float2(cm.x, cm.y);
             c1 = c0;
         } else {
+            // [block][token], cs (even) entries per block: tokens 2t, 2t + 1 in one
+            // 16-byte load; a quad's lanes read adjacent words (no bank conflict)
             const int t0 = 2 * t, t1 = 2 * t + 1;
-            c0 = t0 < m ? lds64f(cb + 8u * (t0 * nblk + blk0 + bb)) : make_float2(0.f, 0.f);
-            c1 = t1 < m ? lds64f(cb + 8u * (t1 * nblk + blk0 + bb)) : make_float2(0.f, 0.f);
+            c0 = t0 < m ? lds64f(cb + 8u * ((blk0 + bb) * cs + t0)) : make_float2(0.f, 0.f);
+            c1 = t1 < m ? lds64f(cb + 8u * ((blk0 + bb) * cs + t1)) : make_float2(0.f, 0.f);
         }
         const uint32_t w0 = bb ? q.z : q.x;
         const uint32_t w1 = bb ? q.w : q.y;
