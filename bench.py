@@ -46,7 +46,7 @@ FILLED = 8192 + 300
 STEP_TRAFFIC_BYTES_PER_LAUNCH = None
 # the same for the per-projection GEMV (K1), from ncu captures of each decoder
 # shape weighted by the step's launch mix (profiles/q4_gemv_lm_head_131072x3072.md)
-GEMV_TRAFFIC_BYTES_PER_LAUNCH = 18_535_412
+GEMV_TRAFFIC_BYTES_PER_LAUNCH = 18_525_620
 
 
 def parse_args(argv=None):
