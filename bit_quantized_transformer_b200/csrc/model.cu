@@ -278,12 +278,13 @@ vox_status vox_decoder_batch_step(const vox_decoder_batch* b, void* stream)
     uint8_t* attn16 = ws_a + ((attn_workspace_bytes(d->n_kv_heads, d->head_dim, d->window, (int)m) + 255) & ~(size_t)255);
     uint8_t* act16 = attn16 + ((m * QD * 2 + 255) & ~(int64_t)255);
     const float scale = 1.0f / sqrtf((float)d->head_dim);
-    // Above 4 sequences the Wo and W2 projections (the long-K ones) run on the
-    // tcgen05 GEMM over bf16 copies of their inputs: there one GEMM beats the
-    // 8-row GEMV (about 11 against 19 us on 3072 x 4096, 19 against 32 on
-    // 3072 x 9216), the copy costing one short launch.
+    // From 4 sequences on, the Wo and W2 projections (the long-K ones) run on
+    // the tcgen05 GEMM over bf16 copies of their inputs: there one GEMM beats
+    // the multi-row GEMV (about 11 against 19 us on 3072 x 4096, 19 against 32
+    // on 3072 x 9216 at 8 rows; 11 against 13 and 19 against 21 at 4 rows), the
+    // copy costing one short launch.  At 3 rows the GEMV is still faster.
     const char* e2 = getenv("VOX_BATCH_GEMM");
-    const bool gemm_wo_w2 = m > 4 && !(e2 && e2[0] == '0') && QD % 64 == 0 && F % 64 == 0;
+    const bool gemm_wo_w2 = m > 3 && !(e2 && e2[0] == '0') && QD % 64 == 0 && F % 64 == 0;
 
     // x[i] = embedding row of sequence i's token (exact fp32 weights)
     if ((st = launch_q4_dequant(static_cast<const uint8_t*>(d->embedding.data), d->vocab, D, 0, d->token, m, d->x,

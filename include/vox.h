@@ -472,7 +472,7 @@ size_t vox_decoder_batch_workspace(const vox_decoder_batch *b);
 /* One greedy step of every sequence: the launches of vox_decoder_step_kernels
  * with m = n_seq rows (embedding rows gathered by token, the QKV epilogue
  * VOX_EP_KV_APPEND_PAGED, vox_gqa_decode_attn_paged, argmax per row, every
- * position advanced); above 4 sequences the Wo and W2 projections run as the
+ * position advanced); from 4 sequences on the Wo and W2 projections run as the
  * tcgen05 GEMM (vox_q4_gemm) on bf16 copies of their inputs, kept in the
  * workspace (VOX_BATCH_GEMM=0 in the environment keeps the GEMV); the
  * sequence can be captured in a CUDA graph.  Errors:

@@ -219,13 +219,15 @@ def check_batch_layer(shape, bm, seq, positions, tokens, seed=0):
 
 
 @pytest.mark.parametrize("positions,tokens", [
+    # 3 sequences: every projection on the multi-row GEMV
+    ([1024, 8192 + 300, 0], [17, 4242, 131071]),
+    # from 4 sequences on Wo and W2 run on the tcgen05 GEMM over bf16 inputs
     ([1024, 8192 + 300, 0, 64], [17, 4242, 131071, 9]),
-    # above 4 sequences Wo and W2 run on the tcgen05 GEMM over bf16 inputs
     ([1024, 8192 + 300, 0, 64, 63, 5000, 8191], [17, 4242, 131071, 9, 0, 77, 65536]),
 ])
 def test_batch_step_one_layer(env, positions, tokens):
-    """Four or seven sequences at different positions (fresh, mid, wrapped,
-    first and last slot of a page): every kernel checked per sequence,
+    """Three, four or seven sequences at different positions (fresh, mid,
+    wrapped, first and last slot of a page): every kernel checked per sequence,
     positions advanced, tokens = per-row argmax; a second step writes the
     next slots."""
     torch, V, WL = env
