@@ -8,6 +8,7 @@ plain torch allocations.  The objects keep every tensor alive and expose the
 from __future__ import annotations
 
 import ctypes
+import os
 
 import numpy as np
 import torch
@@ -150,7 +151,15 @@ class BatchDecoderModel:
         return self.L * 2 * self.shape.n_kv_heads * per * self.shape.head_dim * 2
 
     def launches(self) -> int:
-        return 1 + self.L * 6 + 1 + 1
+        """Kernels one batched step launches: the embedding rows, per layer
+        QKV, attention, combine, Wo, W1||W3 and W2, plus one bf16 cast before
+        each of Wo and W2 where those run on the tcgen05 GEMM (from 4
+        sequences on, unless VOX_BATCH_GEMM=0), then the LM head and the
+        position advance."""
+        sh = self.shape
+        gemm = (self.n_seq >= 4 and not os.environ.get("VOX_BATCH_GEMM", "").startswith("0")
+                and (sh.n_q_heads * sh.head_dim) % 64 == 0 and sh.ffn % 64 == 0)
+        return 1 + self.L * (8 if gemm else 6) + 1 + 1
 
 
 class DecoderModel:
