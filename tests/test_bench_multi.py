@@ -1,6 +1,7 @@
 """The N > 1 path of bench.py on CPU: two gloo ranks run the aggregation the
 benchmark uses (max-over-ranks time, whole-job throughput of independent
-replicas) and its barriers, and the reference arm leaves ranks > 0 idle."""
+replicas) and its barriers, and the reference arm leaves ranks > 0 idle;
+plus the host-side kernel count the batched workload reports."""
 import os
 import socket
 
@@ -50,3 +51,29 @@ def test_two_gloo_ranks_aggregate_max_and_whole_job_throughput():
         # 2 replicas x 10 steps x 2 GB in 150 ms
         assert value == pytest.approx(2 * 10 * 2.0 / 0.150)
         assert ref_rc == 0
+
+
+def test_batched_step_launch_count(monkeypatch):
+    """The batched step's kernel count that bench.py reports: 6 launches per
+    layer on the multi-row GEMV path, 8 (two bf16 casts) once Wo and W2 run
+    on the tcgen05 GEMM from 4 sequences on, the embedding rows, the LM head
+    and the position advance around them; 211 at 8 sequences matches the
+    launch list taken under ncu."""
+    import synth
+    from bit_quantized_transformer_b200 import workloads as WL
+
+    def model(n_seq, **kw):
+        bm = WL.BatchDecoderModel.__new__(WL.BatchDecoderModel)
+        bm.shape = synth.DecoderShape(**kw)
+        bm.n_seq, bm.L = n_seq, bm.shape.n_layers
+        return bm
+
+    monkeypatch.delenv("VOX_BATCH_GEMM", raising=False)
+    assert model(8).launches() == 211
+    assert model(4).launches() == 211
+    assert model(3).launches() == 159
+    assert model(1).launches() == 159
+    assert model(8, n_layers=2).launches() == 19
+    assert model(8, ffn=9216 + 32).launches() == 159      # W2's K not a multiple of 64: GEMV
+    monkeypatch.setenv("VOX_BATCH_GEMM", "0")
+    assert model(8).launches() == 159
