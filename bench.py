@@ -45,8 +45,9 @@ FILLED = 8192 + 300
 # kernel as it stands has been captured
 STEP_TRAFFIC_BYTES_PER_LAUNCH = None
 # the same for the per-projection GEMV (K1), from ncu captures of each decoder
-# shape weighted by the step's launch mix (profiles/q4_gemv_lm_head_131072x3072.md)
-GEMV_TRAFFIC_BYTES_PER_LAUNCH = 18_525_620
+# shape weighted by the step's launch mix (profiles/q4_gemv_lm_head_131072x3072.md);
+# None: the kernel was split into per-epilogue instances after the last capture
+GEMV_TRAFFIC_BYTES_PER_LAUNCH = None
 
 
 def parse_args(argv=None):

@@ -37,6 +37,10 @@
 //    No row statistic is needed before the main loop: the RMSNorm factor
 //    multiplies the finished dot products in the epilogue.  The prologue is
 //    one round of loads and one CTA barrier.
+//  * Instances: one row (MT = 1) or up to 8 (MT = 8), each with and without
+//    the paged KV append and the rotary embedding in its epilogue (EXT).
+//    The decode step's projections run the instances without them, which
+//    stay inside the 128-register budget with less spilling.
 //  * Build knobs (tuning, not semantics): VOX_GEMV_WARPS, VOX_GEMV_RECS,
 //    VOX_GEMV_MIN_CTAS, VOX_GEMV_BATCH at compile time; VOX_GEMV_STAGES,
 //    VOX_GEMV_PREFETCH and VOX_GEMV_CTAS_PER_SM in the environment.
@@ -160,6 +164,7 @@ struct GemvBest {
 // RMSNorm factor of token 2t + e (1 without RMSNorm).  `pre` (with use_pre)
 // holds the residual values in the same layout, loaded ahead by the caller.
 // Not inlined: it runs once per tile and keeps the record loop small.
+template <bool EXT>
 __device__ __noinline__ GemvBest gemv_epilogue(const GemvArgs& a, int64_t tile, float4 acc4, int g, int t, float r0,
                                                float r1, int64_t pos, GemvBest best, float4 pre, int use_pre)
 {
@@ -173,7 +178,7 @@ __device__ __noinline__ GemvBest gemv_epilogue(const GemvArgs& a, int64_t tile, 
     for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int e = 0; e < 2; ++e) v[2 * h + e] = acc[2 * h + e] * rr[e];
-    if (a.rope > 0.f && tile * 16 < (int64_t)a.q_rows + (int64_t)a.n_kv * a.hd) {
+    if (EXT && a.rope > 0.f && tile * 16 < (int64_t)a.q_rows + (int64_t)a.n_kv * a.hd) {
         // q or k rows (a 16-row tile lies in one region): rows 2i and 2i + 1
         // of a head sit in lanes g and g ^ 1, four lanes apart
         const int64_t base = tile * 16 < a.q_rows ? 0 : a.q_rows;
@@ -228,6 +233,7 @@ __device__ __noinline__ GemvBest gemv_epilogue(const GemvArgs& a, int64_t tile, 
             case VOX_EP_KV_APPEND_PAGED: {
                 // token mt is sequence mt: its slot pos[mt] mod window, in the page its table names
                 yr[row] = val;
+                if (!EXT) break;
                 const int64_t kvd = (int64_t)a.n_kv * a.hd;
                 const int64_t rel = row - a.q_rows;
                 if (rel >= 0 && rel < 2 * kvd) {
@@ -328,7 +334,7 @@ __device__ __forceinline__ void gemv_convert(const GemvArgs& a, const float* xr,
     }
 }
 
-template <int MT>
+template <int MT, bool EXT>
 __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kernel(const __grid_constant__ GemvArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -431,7 +437,7 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
                         make_float4(acc[0], acc[1], acc[2], acc[3]);
                     if (lane == 0) s_ptile[warp] = (int32_t)tile;
                 } else if (cin == kc) {
-                    best = gemv_epilogue(a, tile, make_float4(acc[0], acc[1], acc[2], acc[3]), g, t, rr[0], rr[1],
+                    best = gemv_epilogue<EXT>(a, tile, make_float4(acc[0], acc[1], acc[2], acc[3]), g, t, rr[0], rr[1],
                                          pos, best, make_float4(0.f, 0.f, 0.f, 0.f), 0);
                 } else {
                     tacc[0] = acc[0]; tacc[1] = acc[1]; tacc[2] = acc[2]; tacc[3] = acc[3];
@@ -525,7 +531,7 @@ __global__ void __launch_bounds__(kGemvThreads, VOX_GEMV_MIN_CTAS) q4_gemv_kerne
             const float4 pv = lds128f(smem_addr(s_part) + (uint32_t)(w2 * 32 + lane) * 16u + tk2);
             tacc[0] += pv.x; tacc[1] += pv.y; tacc[2] += pv.z; tacc[3] += pv.w;
         }
-        best = gemv_epilogue(a, tail_tile, make_float4(tacc[0], tacc[1], tacc[2], tacc[3]), g, t, rr[0], rr[1], pos,
+        best = gemv_epilogue<EXT>(a, tail_tile, make_float4(tacc[0], tacc[1], tacc[2], tacc[3]), g, t, rr[0], rr[1], pos,
                              best, tres, a.op == VOX_EP_RESIDUAL);
     }
 
@@ -618,11 +624,15 @@ vox_status launch_q4_gemv(const uint8_t* w, int64_t n, int64_t k, const float* x
     a.pre = env_int("VOX_GEMV_PREFETCH", 1, 0, stages);
     a.evict_first = env_int("VOX_GEMV_EVICT_FIRST", 1, 0, 1);
 
-    void (*kern)(GemvArgs) = m == 1 ? q4_gemv_kernel<1> : q4_gemv_kernel<8>;
-    static std::atomic<unsigned long long> attr_done1{0}, attr_done8{0};
-    vox_status st = smem_attr_per_device(reinterpret_cast<const void*>(q4_gemv_kernel<1>), 227 * 1024, attr_done1);
-    if (st == VOX_OK)
-        st = smem_attr_per_device(reinterpret_cast<const void*>(q4_gemv_kernel<8>), 227 * 1024, attr_done8);
+    // The paged append and the rotary embedding live in their own instances,
+    // so the instances the decode step runs compile without them.
+    const bool ext = ep && (ep->op == VOX_EP_KV_APPEND_PAGED || (ep->op == VOX_EP_KV_APPEND && ep->rope_theta > 0.f));
+    void (*const kerns[4])(GemvArgs) = {q4_gemv_kernel<1, false>, q4_gemv_kernel<1, true>, q4_gemv_kernel<8, false>,
+                                        q4_gemv_kernel<8, true>};
+    static std::atomic<unsigned long long> attr_done[4];
+    const int ki = (m == 1 ? 0 : 2) + (ext ? 1 : 0);
+    void (*kern)(GemvArgs) = kerns[ki];
+    vox_status st = smem_attr_per_device(reinterpret_cast<const void*>(kern), 227 * 1024, attr_done[ki]);
     if (st != VOX_OK) return st;
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemvThreads, L.total);
